@@ -1,0 +1,215 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the hybrid long-context attention step of
+ * DeepSeek-V4 (Compressed Sparse Attention, CSA, and Heavily Compressed
+ * Attention, HCA) on one NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Buffers are caller-owned DEVICE memory unless stated otherwise,
+ *    row-major and contiguous, base pointers 16-byte aligned.  The library
+ *    never allocates or frees device memory; calls that need scratch take a
+ *    caller workspace sized by the matching *_workspace_bytes() query.
+ *  * bf16 tensors are passed as `const uint16_t *` holding bf16 bit patterns.
+ *  * `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on that stream and returns after enqueueing its kernels.
+ *  * Return value: CSA_OK (0) or a negative csa_status.  Validation errors
+ *    (CSA_ERR_INVALID / CSA_ERR_UNSUPPORTED / CSA_ERR_WORKSPACE) are detected
+ *    on the host before any launch, so nothing was enqueued.  CSA_ERR_CUDA
+ *    reports a launch error.  Device-side failures (a bounded wait that ran
+ *    out) are recorded in a device status word and reported by
+ *    csa_sync_status().  No exception crosses the ABI.
+ *  * Notation: batch = independent sequences; T = tokens per sequence; m =
+ *    compression ratio; N = compressed entries per sequence (floor(T/m) when
+ *    built by csa_compress); a query at position t sees the first
+ *    n_vis(t) = min(N, floor((t+1)/m)) entries (an entry is visible once all
+ *    of its newest-m tokens are at or before t).
+ *
+ * Sources: "DeepSeek v4" (it.peoplentools.com) section "Compressed Sparse
+ * Attention" (compressed entries, lightning indexer, top-k selector, sliding
+ * window) and the hybrid-attention section (HCA, m' >> m); "DeepSeek-AI (2026)
+ * - ARXIV-2606.19348" (dmarx anthology record) "Key takeaways" (two latent KV
+ * streams, overlapping 2m-token windows, RMSNorm on query heads and on the
+ * compressed KV head); "DeepSeek-V4-Pro - Model techniques map" table
+ * "Checked in its code" (one KV head for 128 query heads, window 128, top-k
+ * 1024 with -1 for invalid slots, 64x128 indexer) and list "inference
+ * quantization" (FP4 indexer); "DeepSeek V4 paper full version is out, FP4
+ * QAT details and stability tricks [D]" (FP4 activations on the indexer QK path).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID = -1,     /* null / misaligned pointer, bad size or argument   */
+    CSA_ERR_UNSUPPORTED = -2, /* a shape outside what the compiled kernels handle   */
+    CSA_ERR_CUDA = -3,        /* a CUDA launch or runtime error                     */
+    CSA_ERR_WORKSPACE = -4,   /* workspace pointer NULL or smaller than required    */
+    CSA_ERR_TIMEOUT = -5      /* a device-side bounded wait expired (see csa_sync_status) */
+} csa_status;
+
+/* Human-readable text for a csa_status (static storage, never NULL). */
+const char *csa_strerror(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int csa_version(void);
+
+/*
+ * csa_compress -- build compressed KV entries from the two latent streams.
+ *   ("DeepSeek v4" -> "Compressed Sparse Attention" -> compressed Key-Value
+ *    entry; anthology record "Key takeaways": overlapping 2m-token windows.)
+ *
+ * For every sequence b, entry i in [0, N), N = floor(T/m), and channel c:
+ *   w_j[c]  = softmax over j = 0..2m-1 of logits[j][c]
+ *   C_i[c]  = sum_{j<m} w_j[c] * B[(i-1)m + j][c] + sum_{j<m} w_{m+j}[c] * A[im + j][c]
+ * Rows 0..m-1 of the logits weight the previous m tokens (stream B), rows
+ * m..2m-1 the newest m tokens (stream A).  Entry 0 has no previous block: its
+ * softmax runs over the A half only.  If apply_rmsnorm != 0 each entry is then
+ *   y[c] = C_i[c] / sqrt(mean_c(C_i^2) + eps) * gain[c]   (gain NULL -> 1).
+ * Arithmetic in fp32; the result is rounded to bf16 once.
+ *
+ *   A, B    [batch][T][d] bf16          stream A (newest half), stream B (previous half)
+ *   logits  [2m][d] fp32                static per-channel pooling logits
+ *   gain    [d] fp32 or NULL
+ *   out     [batch][floor(T/m)][d] bf16
+ * Requirements: batch >= 1, T >= m >= 1, d % 8 == 0, 8 <= d <= 1024, m <= 256
+ * (m > 16 or 24*m*d > 96 KiB additionally needs d % 64 == 0).
+ */
+int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
+                 int batch, long long T, int d, int m,
+                 int apply_rmsnorm, const float *gain, float eps,
+                 uint16_t *out, void *stream);
+
+/*
+ * csa_index -- lightning-indexer scores ("DeepSeek v4" -> "sparse selection
+ * Lightning Indexer": per-head weight times ReLU(q . K), summed over heads).
+ *   S[b][q][s] = sum_h w[b][q][h] * max(0, q_idx[b][q][h] . k_idx[b][s])   for s < n_vis(q_pos[b][q])
+ *   S[b][q][s] = -inf                                                      otherwise
+ * bf16 operands on the tensor cores, fp32 accumulation and epilogue.
+ *
+ *   q_idx  [batch][nq][H_I][d_I] bf16     w [batch][nq][H_I] fp32
+ *   k_idx  [batch][N][d_I] bf16           q_pos [batch][nq] int32 (0 <= t)
+ *   scores [batch][nq][N] fp32 (output)
+ * Requirements: d_I in {16, 32, 64, 128, 256}; 1 <= H_I <= 256 and
+ * H_I % 16 == 0 or H_I < 16 (padded internally); m >= 1; N >= 1.
+ */
+int csa_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx,
+              const int *q_pos, int batch, int nq, long long N, int H_I, int d_I,
+              int m, float *scores, void *stream);
+
+/*
+ * csa_quantize_fp4 -- e2m1 elements with one e4m3 scale per 16-element block
+ * (the FP4 activations of the indexer QK path; "FP4 QAT details" forum post,
+ * techniques map "FP4 precision for the attention indexer").
+ * Per block x_0..x_15:  s = e4m3_RNE_satfinite(fp32(absmax / 6));
+ *   s == 0 -> codes 0;  else q_j = e2m1_RNE_satfinite(fp32(x_j / s)), and a
+ *   code whose magnitude rounds to 0 is stored as +0.
+ *   x       [rows][d] bf16
+ *   packed  [rows][d/2] uint8   element 2i in the low nibble, 2i+1 in the high one
+ *   scales  [rows][d/16] uint8  e4m3 bit patterns
+ * Requirements: rows >= 1, d % 16 == 0.
+ */
+int csa_quantize_fp4(const uint16_t *x, long long rows, int d,
+                     uint8_t *packed, uint8_t *scales, void *stream);
+
+/*
+ * csa_index_fp4 -- csa_index on FP4 operands (layouts of csa_quantize_fp4):
+ * the score is the same formula on the dequantised values e2m1 * e4m3, with
+ * exact products and fp32 accumulation.
+ *   q4 [batch][nq][H_I][d_I/2]   q4s [batch][nq][H_I][d_I/16]   w [batch][nq][H_I] fp32
+ *   k4 [batch][N][d_I/2]         k4s [batch][N][d_I/16]         scores [batch][nq][N] fp32
+ * Requirements: as csa_index (d_I % 64 == 0 for the packed path).
+ */
+int csa_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w,
+                  const uint8_t *k4, const uint8_t *k4s, const int *q_pos,
+                  int batch, int nq, long long N, int H_I, int d_I, int m,
+                  float *scores, void *stream);
+
+/*
+ * csa_topk -- causal top-k selector ("DeepSeek v4" -> top-k selector;
+ * techniques map: indices at or beyond the causal threshold become -1).
+ * For each query the k largest scores among the first n_vis(t) entries; ties
+ * are broken towards the lower entry index.  The chosen indices are written in
+ * ascending index order; the remaining slots (when n_vis < k) are -1.
+ *   scores [batch][nq][N] fp32, q_pos [batch][nq], idx [batch][nq][k] int32.
+ * Requirements: 1 <= k <= 8192; N <= 2^19.  Workspace: csa_topk_workspace_bytes
+ * (currently 0: the selection runs in distributed shared memory).
+ */
+size_t csa_topk_workspace_bytes(int batch, int nq, long long N, int k);
+int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long N,
+             int m, int k, int *idx, void *workspace, size_t workspace_bytes,
+             void *stream);
+
+/*
+ * csa_attend -- core attention of CSA: multi-query attention with H query
+ * heads sharing one KV head (K = V) over the selected compressed entries plus
+ * a sliding window of raw stream-A rows (techniques map rows "Grouped-query
+ * attention" and "Sliding-window attention"; "DeepSeek v4" Figure 3 text).
+ *   q_hat_h = RMSNorm(q_h) (eps, q_gain [D] or NULL = unit gain)
+ *   J       = { kv[b][j] : j in idx[b][q], 0 <= j < N }
+ *             U { stream-A row of position u : max(0, t-W+1) <= u <= t }
+ *   out_h   = sum_{x in J} softmax(scale * q_hat_h . x) * x
+ * bf16 operands, fp32 softmax and accumulation, bf16 output.
+ *   q       [batch][nq][H][D] bf16      kv [batch][N][D] bf16
+ *   idx     [batch][nq][k] int32 (-1 = invalid slot; entries outside [0, N) are skipped)
+ *   win_src [batch][win_rows][D] bf16   stream-A rows of positions win_pos0 .. win_pos0+win_rows-1
+ *           (a whole stream: win_pos0 = 0, win_rows = T; a decode window cache:
+ *           win_pos0 = t-W+1, win_rows = W).  Window positions the buffer does not
+ *           hold are skipped.
+ *   q_pos   [batch][nq] int32           out [batch][nq][H][D] bf16
+ * Requirements: D in {64, 128, 256, 512}; 1 <= H <= 128; W >= 1; k >= 0.
+ * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, k + W).
+ */
+size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
+int csa_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+               const int *idx, int k, const uint16_t *win_src, long long win_pos0,
+               long long win_rows, int W,
+               const int *q_pos, int batch, int nq, int H, int D, float scale, float eps,
+               uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * hca_attend -- core attention of HCA: as csa_attend with the key set
+ * { kv[b][j] : j < n_vis(t) } U window, i.e. dense attention over every
+ * visible compressed entry ("DeepSeek v4" hybrid-attention section: HCA
+ * compresses every m' >> m tokens and keeps attention dense).
+ * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, N + W).
+ */
+int hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
+               const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
+               const int *q_pos,
+               int batch, int nq, int H, int D, float scale, float eps,
+               uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * csa_sync_status -- synchronise `stream`, then read and clear the device
+ * status word.  Returns CSA_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call, CSA_ERR_CUDA on a CUDA error, else CSA_OK.
+ */
+int csa_sync_status(void *stream);
+
+/*
+ * csa_set_wait_budget_ns -- upper bound (nanoseconds of device global time)
+ * on any single device-side wait (mbarrier or flag) in the library's kernels;
+ * 0 restores the default (2 s).  Affects kernels launched after the call.
+ */
+void csa_set_wait_budget_ns(unsigned long long ns);
+
+/*
+ * csa_selftest_wait_timeout -- launches one CTA that waits on an mbarrier
+ * nothing ever arrives on, under the current wait budget.  The wait must give
+ * up, record CSA_ERR_TIMEOUT in the status word and return; the context stays
+ * usable.  Used to test the failure path without faulting the GPU.
+ */
+int csa_selftest_wait_timeout(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,228 @@
+"""Thin Python binding of libcsa.so (include/csa.h), same names as the C ABI.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Tensors are torch CUDA tensors (PyTorch supplies device memory and the current
+stream); outputs are allocated here when not given.  If the shared library is
+missing the first call raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcsa.so")
+
+CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA, CSA_ERR_WORKSPACE, CSA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+
+_lib = None
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (where, strerror(status), status))
+
+
+def load() -> ctypes.CDLL:
+    """Load libcsa.so (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libcsa.so is not built (%s); run `python -m long_context_compressed_06_b200.build`"
+                           % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "csa_strerror": ([i32], ctypes.c_char_p),
+        "csa_version": ([], i32),
+        "csa_compress": ([P, P, P, i32, i64, i32, i32, i32, P, f32, P, P], i32),
+        "csa_index": ([P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
+        "csa_quantize_fp4": ([P, i64, i32, P, P, P], i32),
+        "csa_index_fp4": ([P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
+        "csa_topk_workspace_bytes": ([i32, i32, i64, i32], sz),
+        "csa_topk": ([P, P, i32, i32, i64, i32, i32, P, P, sz, P], i32),
+        "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
+        "csa_attend": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "hca_attend": ([P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_sync_status": ([P], i32),
+        "csa_set_wait_budget_ns": ([ctypes.c_ulonglong], None),
+        "csa_selftest_wait_timeout": ([P], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def strerror(status: int) -> str:
+    return load().csa_strerror(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != CSA_OK:
+        raise CsaError(rc, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got %s" % (name, ndim, tuple(t.shape)))
+    return t
+
+
+# --------------------------------------------------------------------------- ops
+def csa_compress(A, B, logits, m: int, apply_rmsnorm: bool = True, gain=None, eps: float = 1e-6, out=None):
+    """A, B [batch][T][d] bf16; logits [2m][d] fp32 -> compressed entries [batch][T//m][d] bf16."""
+    L = load()
+    _need(A, torch.bfloat16, "A", 3)
+    _need(B, torch.bfloat16, "B", 3)
+    _need(logits, torch.float32, "logits", 2)
+    batch, T, d = A.shape
+    if B.shape != A.shape or logits.shape != (2 * m, d):
+        raise ValueError("shape mismatch")
+    if gain is not None:
+        _need(gain, torch.float32, "gain", 1)
+    if out is None:
+        out = torch.empty((batch, T // m, d), dtype=torch.bfloat16, device=A.device)
+    _check(L.csa_compress(_p(A), _p(B), _p(logits), batch, T, d, m, int(bool(apply_rmsnorm)), _p(gain),
+                          float(eps), _p(out), _stream()), "csa_compress")
+    return out
+
+
+def csa_index(q_idx, w, k_idx, q_pos, m: int, scores=None):
+    """q_idx [b][nq][H_I][d_I] bf16, w [b][nq][H_I] fp32, k_idx [b][N][d_I] bf16 -> scores [b][nq][N] fp32."""
+    L = load()
+    _need(q_idx, torch.bfloat16, "q_idx", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(k_idx, torch.bfloat16, "k_idx", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H_I, d_I = q_idx.shape
+    N = k_idx.shape[1]
+    if scores is None:
+        scores = torch.empty((batch, nq, N), dtype=torch.float32, device=q_idx.device)
+    _check(L.csa_index(_p(q_idx), _p(w), _p(k_idx), _p(q_pos), batch, nq, N, H_I, d_I, m, _p(scores),
+                       _stream()), "csa_index")
+    return scores
+
+
+def csa_quantize_fp4(x, packed=None, scales=None):
+    """x [..., d] bf16 -> (packed [..., d/2] u8, scales [..., d/16] u8 e4m3)."""
+    L = load()
+    _need(x, torch.bfloat16, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d
+    if packed is None:
+        packed = torch.empty(x.shape[:-1] + (d // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (d // 16,), dtype=torch.uint8, device=x.device)
+    _check(L.csa_quantize_fp4(_p(x), rows, d, _p(packed), _p(scales), _stream()), "csa_quantize_fp4")
+    return packed, scales
+
+
+def csa_index_fp4(q4, q4s, w, k4, k4s, q_pos, m: int, scores=None):
+    L = load()
+    for t, n in ((q4, "q4"), (q4s, "q4s"), (k4, "k4"), (k4s, "k4s")):
+        _need(t, torch.uint8, n)
+    _need(w, torch.float32, "w", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H_I, half = q4.shape
+    N = k4.shape[1]
+    if scores is None:
+        scores = torch.empty((batch, nq, N), dtype=torch.float32, device=q4.device)
+    _check(L.csa_index_fp4(_p(q4), _p(q4s), _p(w), _p(k4), _p(k4s), _p(q_pos), batch, nq, N, H_I, half * 2, m,
+                           _p(scores), _stream()), "csa_index_fp4")
+    return scores
+
+
+def csa_topk(scores, q_pos, m: int, k: int, idx=None):
+    """scores [b][nq][N] fp32 -> idx [b][nq][k] int32 (ascending, -1 padded)."""
+    L = load()
+    _need(scores, torch.float32, "scores", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, N = scores.shape
+    if idx is None:
+        idx = torch.empty((batch, nq, k), dtype=torch.int32, device=scores.device)
+    _check(L.csa_topk(_p(scores), _p(q_pos), batch, nq, N, m, k, _p(idx), None, 0, _stream()), "csa_topk")
+    return idx
+
+
+def attend_workspace_bytes(batch: int, nq: int, H: int, D: int, max_keys: int) -> int:
+    return int(load().csa_attend_workspace_bytes(batch, nq, H, D, max_keys))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
+               workspace=None, win_pos0: int = 0):
+    """q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] (bf16, stream-A rows of positions
+    win_pos0..) -> out [b][nq][H][D] bf16."""
+    L = load()
+    _need(q, torch.bfloat16, "q", 4)
+    _need(kv, torch.bfloat16, "kv", 3)
+    _need(idx, torch.int32, "idx", 3)
+    _need(win, torch.bfloat16, "win", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H, D = q.shape
+    N, rows, k = kv.shape[1], win.shape[1], idx.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
+    _check(L.csa_attend(_p(q), _p(q_gain), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W, _p(q_pos),
+                        batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend")
+    return out
+
+
+def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
+               workspace=None, win_pos0: int = 0):
+    """Dense attention over every visible entry of kv [b][N][D] plus the window."""
+    L = load()
+    _need(q, torch.bfloat16, "q", 4)
+    _need(kv, torch.bfloat16, "kv", 3)
+    _need(win, torch.bfloat16, "win", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H, D = q.shape
+    N, rows = kv.shape[1], win.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
+    _check(L.hca_attend(_p(q), _p(q_gain), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos), batch, nq, H,
+                        D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend")
+    return out
+
+
+def csa_sync_status() -> int:
+    return int(load().csa_sync_status(_stream()))
+
+
+def csa_set_wait_budget_ns(ns: int) -> None:
+    load().csa_set_wait_budget_ns(int(ns))
+
+
+def csa_selftest_wait_timeout() -> None:
+    _check(load().csa_selftest_wait_timeout(_stream()), "csa_selftest_wait_timeout")

@@ -1,0 +1,86 @@
+// attend.cu -- csa_attend / hca_attend dispatch, workspace sizing and the
+// split-KV combine.
+//
+// The combine merges the partial results of the key splits of one (query,
+// head) with the usual log-sum-exp rule, always in split order, so the output
+// does not depend on scheduling (the pages' inference stack relies on
+// batch-invariant, deterministic split reductions; techniques map
+// "Separate split-K outputs with deterministic reduction").
+#include <algorithm>
+
+#include "attend_common.cuh"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+namespace {
+
+__global__ void __launch_bounds__(128) attend_combine_kernel(AttendArgs a) {
+    const long long bq = blockIdx.x;
+    const int h = blockIdx.y;
+    const int i = threadIdx.x * 4;
+    if (i >= a.D) return;
+    float M = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((size_t)s * a.n_bq + bq) * a.H + h].x);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < a.splits; ++s) {
+        const size_t off = ((size_t)s * a.n_bq + bq) * a.H + h;
+        const float2 ml = a.part_ml[off];
+        const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        const float4 o = *reinterpret_cast<const float4 *>(a.part_o + off * a.D + i);
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+    }
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
+    uint16_t *dst = a.out + ((size_t)bq * a.H + h) * a.D + i;
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+}
+
+size_t ws_bytes_for(long long n_bq, int H, int D, int splits) {
+    if (splits <= 1) return 0;
+    return (size_t)splits * n_bq * H * ((size_t)D * sizeof(float) + sizeof(float2));
+}
+
+}  // namespace
+
+int launch_attend_combine(const AttendArgs &a, cudaStream_t st) {
+    dim3 grid((unsigned)a.n_bq, (unsigned)a.H);
+    attend_combine_kernel<<<grid, std::max(32, a.D / 4), 0, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
+size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys) {
+    const long long n_bq = (long long)batch * nq;
+    return ws_bytes_for(n_bq, H, D, attend_simt_splits(n_bq, H, max_keys));
+}
+
+int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
+                  const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
+                  int W, const int *q_pos,
+                  int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
+                  size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
+    (void)ctx;
+    AttendArgs a = {};
+    a.q = q; a.q_gain = q_gain; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
+    a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
+    a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
+    if (a.n_bq == 0) return CSA_OK;
+    const long long max_keys = (dense ? N : (long long)k) + W;
+    a.splits = attend_simt_splits(a.n_bq, H, max_keys);
+    a.keys_per_split = (max_keys + a.splits - 1) / a.splits;
+    const size_t need = ws_bytes_for(a.n_bq, H, D, a.splits);
+    if (need > 0) {
+        if (!ws || ws_bytes < need) return CSA_ERR_WORKSPACE;
+        a.part_o = reinterpret_cast<float *>(ws);
+        a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
+                                               (size_t)a.splits * a.n_bq * H * D * sizeof(float));
+    }
+    return launch_attend_simt(a, st);
+}
+
+}  // namespace csa

@@ -1,0 +1,43 @@
+// kernels.h -- internal host-side launchers (validated arguments in, status out).
+// The C ABI in abi.cu validates every argument and then calls these.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa {
+
+struct DevCtx;
+
+int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, int batch, long long T,
+                    int d, int m, int apply_rmsnorm, const float *gain, float eps, uint16_t *out,
+                    cudaStream_t st);
+
+int launch_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos,
+                 int batch, int nq, long long N, int H_I, int d_I, int m, float *scores,
+                 const DevCtx &ctx, cudaStream_t st);
+
+int launch_quantize_fp4(const uint16_t *x, long long rows, int d, uint8_t *packed, uint8_t *scales,
+                        cudaStream_t st);
+
+int launch_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, const uint8_t *k4,
+                     const uint8_t *k4s, const int *q_pos, int batch, int nq, long long N, int H_I,
+                     int d_I, int m, float *scores, const DevCtx &ctx, cudaStream_t st);
+
+size_t topk_workspace_bytes(int batch, int nq, long long N, int k);
+int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k,
+                int *idx, cudaStream_t st);
+
+// Attention: dense selects the HCA key set of the first n_vis(t) entries;
+// otherwise the k selected entries idx (may be null when k == 0).
+size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
+int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
+                  const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
+                  int W, const int *q_pos,
+                  int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,
+                  void *ws, size_t ws_bytes, const DevCtx &ctx, cudaStream_t st);
+
+int launch_selftest_wait(const DevCtx &ctx, cudaStream_t st);
+
+}  // namespace csa

@@ -1,0 +1,239 @@
+// topk.cu -- causal top-k selector (csa_topk).
+//
+// For each query, the k largest scores among its n_vis(t) visible entries,
+// ties broken towards the lower index; invalid slots are -1 ("DeepSeek v4"
+// -> top-k selector; techniques map: indices at or beyond the causal threshold
+// become -1).  Output indices are in ascending order.
+//
+// Design: a radix select over the scores mapped to order-preserving uint32
+// keys.  One query is handled by a thread-block cluster of CS CTAs x 1024
+// threads; each thread keeps R consecutive keys in registers (CS*1024*R >= N),
+// so the scores are read from memory exactly once.  Three digit passes
+// (11, 11, 10 bits) build a histogram of the candidates that still share the
+// threshold's prefix; warps aggregate equal digits with __match_any_sync and
+// add into rank 0's shared-memory histogram through distributed shared memory.
+// A pass stops early once the threshold bin holds exactly the number of
+// elements still needed.  Selection is a stable compaction: per-thread
+// counts, a block scan, and a cluster scan over CTA totals via DSMEM.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace csa {
+namespace {
+
+constexpr int kTopkThreads = 1024;
+constexpr int kBins = 2048;
+
+// order-preserving map fp32 -> uint32 (-0 folded onto +0)
+CSA_DEVINL uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inclusive scan over the 1024 threads of the block; returns this thread's
+// inclusive prefix and writes the block total to *total.
+template <typename T>
+CSA_DEVINL T block_scan_incl(T v, T *warp_buf, T *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const T n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) warp_buf[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        T w = warp_buf[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const T n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        warp_buf[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_buf[warp - 1];
+    const T tot = warp_buf[31];
+    __syncthreads();  // warp_buf is reused by the next scan
+    *total = tot;
+    return v;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__restrict__ scores,
+                                                               const int *__restrict__ q_pos, long long N,
+                                                               int m, int k, int *__restrict__ idx, int CS) {
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const long long bq = blockIdx.x / CS;
+
+    __shared__ uint32_t hist[3][kBins];          // used in rank 0 only
+    __shared__ uint32_t warp_u32[32];
+    __shared__ unsigned long long warp_u64[32];
+    __shared__ unsigned long long cta_total;      // (gt << 32) | eq, read by higher ranks
+    __shared__ uint32_t s_bin, s_cnt;
+    __shared__ long long s_krem;
+
+    for (int i = threadIdx.x; i < 3 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
+    if (threadIdx.x == 0) {
+        s_bin = 0u;
+        s_cnt = 0u;
+        s_krem = 0;
+    }
+
+    const long long nv = n_visible(q_pos[bq], m, N);
+    const long long kk = nv < k ? nv : k;
+    const long long seg0 = ((long long)rank * kTopkThreads + threadIdx.x) * R;
+    const int nloc = (int)(nv - seg0 <= 0 ? 0 : (nv - seg0 >= R ? R : nv - seg0));
+
+    uint32_t key[R];
+    const float *row = scores + bq * N;
+    if (nloc == R && (N & 3) == 0) {
+#pragma unroll
+        for (int r = 0; r < R; r += 4) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(row + seg0 + r));
+            key[r] = order_key(v.x); key[r + 1] = order_key(v.y);
+            key[r + 2] = order_key(v.z); key[r + 3] = order_key(v.w);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) key[r] = r < nloc ? order_key(__ldg(row + seg0 + r)) : 0u;
+    }
+    cluster.sync();  // every histogram cleared before any remote add
+
+    uint32_t prefix = 0u, mask = 0u;
+    long long krem = kk;
+    bool done = nv <= k;  // every visible entry is selected
+    uint32_t *h0 = cluster.map_shared_rank(&hist[0][0], 0);
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int p = 0; p < 3 && !done; ++p) {
+        const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);
+        const uint32_t dmask = p == 2 ? 0x3ffu : 0x7ffu;
+        uint32_t *hp = h0 + p * kBins;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const bool cand = r < nloc && (key[r] & mask) == prefix;
+            const uint32_t bin = cand ? (key[r] >> sh) & dmask : 0xffffffffu;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (cand && lane == __ffs(peers) - 1) atomicAdd(hp + bin, (uint32_t)__popc(peers));
+        }
+        cluster.sync();  // histogram of this pass complete
+        // threshold bin: the highest bin b with (count above b) < krem <= (count above b) + hist[b]
+        const uint32_t c_lo = hp[2 * threadIdx.x], c_hi = hp[2 * threadIdx.x + 1];
+        uint32_t tot;
+        const uint32_t incl = block_scan_incl<uint32_t>(c_lo + c_hi, warp_u32, &tot);
+        const long long above = (long long)tot - incl;  // count in bins of higher threads
+        if (above < krem && above + c_hi >= krem) {
+            s_bin = 2 * threadIdx.x + 1; s_cnt = c_hi; s_krem = krem - above;
+        } else if (above + c_hi < krem && above + c_hi + c_lo >= krem) {
+            s_bin = 2 * threadIdx.x; s_cnt = c_lo; s_krem = krem - above - c_hi;
+        }
+        __syncthreads();
+        prefix |= s_bin << sh;
+        mask |= dmask << sh;
+        krem = s_krem;
+        done = (long long)s_cnt == krem;
+        __syncthreads();
+    }
+
+    // stable compaction in index order
+    uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (r < nloc) {
+            const uint32_t u = key[r] & mask;
+            gt += u > prefix;
+            eq += u == prefix;
+        }
+    }
+    unsigned long long blk_tot;
+    const unsigned long long mine = ((unsigned long long)gt << 32) | eq;
+    const unsigned long long excl = block_scan_incl<unsigned long long>(mine, warp_u64, &blk_tot) - mine;
+    if (threadIdx.x == 0) cta_total = blk_tot;
+    cluster.sync();
+    unsigned long long base = 0ull;
+    for (int r2 = 0; r2 < rank; ++r2) base += *cluster.map_shared_rank(&cta_total, r2);
+    long long gt_before = (long long)((base + excl) >> 32);
+    long long eq_before = (long long)((base + excl) & 0xffffffffull);
+    int *out = idx + bq * k;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (r < nloc) {
+            const uint32_t u = key[r] & mask;
+            if (u > prefix) {
+                const long long pos = gt_before + (eq_before < krem ? eq_before : krem);
+                if (pos < kk) out[pos] = (int)(seg0 + r);
+                ++gt_before;
+            } else if (u == prefix) {
+                if (eq_before < krem && gt_before + eq_before < kk) out[gt_before + eq_before] = (int)(seg0 + r);
+                ++eq_before;
+            }
+        }
+    }
+    if (rank == 0)
+        for (long long i = kk + threadIdx.x; i < k; i += kTopkThreads) out[i] = -1;
+    cluster.sync();  // peers may still read hist / cta_total of this CTA
+}
+
+struct TopkPlan {
+    int CS, R;
+};
+
+TopkPlan plan(long long n_queries, long long N) {
+    const long long need = (N + kTopkThreads - 1) / kTopkThreads;  // elements per thread with one CTA
+    int CS = 1;
+    while ((need + CS - 1) / CS > 32) CS *= 2;
+    int R = 4;
+    while ((long long)R * CS < need) R *= 2;
+    // spread small batches over more SMs (portable cluster sizes only)
+    while (n_queries * CS < 148 && CS < 8 && R > 4) {
+        CS *= 2;
+        R /= 2;
+    }
+    return {CS, R};
+}
+
+}  // namespace
+
+size_t topk_workspace_bytes(int, int, long long, int) { return 0; }
+
+int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k, int *idx,
+                cudaStream_t st) {
+    const long long nqry = (long long)batch * nq;
+    if (nqry == 0) return CSA_OK;
+    const TopkPlan pl = plan(nqry, N);
+    if (pl.CS > 16 || pl.R > 32) return CSA_ERR_UNSUPPORTED;
+    void (*kern)(const float *, const int *, long long, int, int, int *, int) = nullptr;
+    switch (pl.R) {
+        case 4: kern = topk_kernel<4>; break;
+        case 8: kern = topk_kernel<8>; break;
+        case 16: kern = topk_kernel<16>; break;
+        case 32: kern = topk_kernel<32>; break;
+        default: return CSA_ERR_UNSUPPORTED;
+    }
+    if (pl.CS > 8 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nqry * pl.CS));
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, scores, q_pos, N, m, k, idx, pl.CS);
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
+}  // namespace csa

@@ -36,9 +36,9 @@ def lib():
         L.orc_n_visible.restype = i64
         L.orc_index.argtypes = [P, P, P, P, i32, i32, i64, i32, i32, i32, P]
         L.orc_topk.argtypes = [P, P, i32, i32, i64, i32, i32, P]
-        L.orc_attend.argtypes = [P, P, P, i64, P, i32, P, i64, i32, P, i32, i32, i32, i32,
+        L.orc_attend.argtypes = [P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
                                  f64, f64, P]
-        L.orc_hca_attend.argtypes = [P, P, P, i64, i32, P, i64, i32, P, i32, i32, i32, i32,
+        L.orc_hca_attend.argtypes = [P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
                                      f64, f64, P]
         L.orc_e2m1_decode.argtypes = [ctypes.c_uint]
         L.orc_e2m1_decode.restype = f64
@@ -132,8 +132,9 @@ def topk(scores, q_pos, m, k):
     return out
 
 
-def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None):
-    """CSA attention: q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][T][D] -> float64 [b][nq][H][D]."""
+def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0):
+    """CSA attention: q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] holding stream-A
+    positions win_pos0.. -> float64 [b][nq][H][D]."""
     q, pq = _c(q, np.uint16)
     kv, pkv = _c(kv, np.uint16)
     idx, pidx = _c(idx, np.int32)
@@ -143,14 +144,14 @@ def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None):
     batch, nq, H, D = q.shape
     N = kv.shape[1]
     k = idx.shape[2]
-    T = win.shape[1]
+    rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
-    lib().orc_attend(pq, pg, pkv, N, pidx, k, pwin, T, W, pqp, batch, nq, H, D, float(scale),
-                     float(eps), out.ctypes.data_as(ctypes.c_void_p))
+    lib().orc_attend(pq, pg, pkv, N, pidx, k, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
+                     float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 
-def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None):
+def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0):
     """HCA attention over all visible entries + window -> float64 [b][nq][H][D]."""
     q, pq = _c(q, np.uint16)
     kv, pkv = _c(kv, np.uint16)
@@ -159,10 +160,10 @@ def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None):
     g, pg = _opt(q_gain, np.float32)
     batch, nq, H, D = q.shape
     N = kv.shape[1]
-    T = win.shape[1]
+    rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
-    lib().orc_hca_attend(pq, pg, pkv, N, m, pwin, T, W, pqp, batch, nq, H, D, float(scale),
-                         float(eps), out.ctypes.data_as(ctypes.c_void_p))
+    lib().orc_hca_attend(pq, pg, pkv, N, m, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
+                         float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 

@@ -285,7 +285,7 @@ void orc_topk(const double *scores, const int *q_pos, int batch, int nq, long lo
 /*
  * For one query at position t with H heads of dim D and one shared KV head:
  *   qh_hat = RMSNorm(q_h)                 (eps, optional gain [D])
- *   J      = { kv[j] : j in the key list } U { win[u] : max(0,t-W+1) <= u <= t }
+ *   J      = { kv[j] : j in the key list } U { A[u] : max(0,t-W+1) <= u <= t }
  *   o_h    = sum_{x in J} softmax_x(scale * qh_hat . x) * x
  * Keys and values are the same rows (one KV head).  Window rows are raw
  * stream-A rows (no RMSNorm); overlap with compressed entries is kept.
@@ -329,11 +329,26 @@ static void attend_one(const uint16_t *q, const float *q_gain, int H, int D, dou
     free(z);
 }
 
+/* Window rows: stream-A rows of positions u in [max(0, t-W+1), t] that the
+ * window buffer holds; win [batch][win_rows][D] holds positions
+ * win_pos0 .. win_pos0 + win_rows - 1 (win_pos0 = 0, win_rows = T for a whole
+ * stream; win_pos0 = t-W+1, win_rows = W for a decode window cache). */
+static long long window_rows(const uint16_t *win, long long win_pos0, long long win_rows, int W,
+                             long long b, long long t, int D, const uint16_t **rows)
+{
+    long long n = 0;
+    for (long long u = t - W + 1; u <= t; ++u) {
+        if (u < 0 || u < win_pos0 || u - win_pos0 >= win_rows) continue;
+        rows[n++] = win + ((size_t)b * win_rows + (u - win_pos0)) * D;
+    }
+    return n;
+}
+
 /* CSA: key list = selected compressed entries (idx != -1 and 0 <= idx < N)
  * plus the sliding window.  q [batch][nq][H][D], kv [batch][N][D],
- * idx [batch][nq][k], win [batch][T][D], out [batch][nq][H][D]. */
+ * idx [batch][nq][k], win [batch][win_rows][D], out [batch][nq][H][D]. */
 void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
-                const int *idx, int k, const uint16_t *win, long long T, int W,
+                const int *idx, int k, const uint16_t *win, long long win_pos0, long long win_rows, int W,
                 const int *q_pos, int batch, int nq, int H, int D, double scale, double eps,
                 double *out)
 {
@@ -349,10 +364,7 @@ void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long
             if (j < 0 || j >= N) continue;
             rows[n++] = kv + ((size_t)b * N + j) * D;
         }
-        for (long long u = t - W + 1; u <= t; ++u) {
-            if (u < 0 || u >= T) continue;
-            rows[n++] = win + ((size_t)b * T + u) * D;
-        }
+        n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
         attend_one(q + (size_t)bq * H * D, q_gain, H, D, scale, eps, rows, n,
                    out + (size_t)bq * H * D);
         free(rows);
@@ -363,7 +375,8 @@ void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long
  * plus the sliding window; no indexer ([DSv4-KR] hybrid-attention section:
  * HCA compresses every m' >> m tokens and keeps attention dense). */
 void orc_hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
-                    int m, const uint16_t *win, long long T, int W, const int *q_pos,
+                    int m, const uint16_t *win, long long win_pos0, long long win_rows, int W,
+                    const int *q_pos,
                     int batch, int nq, int H, int D, double scale, double eps, double *out)
 {
     const long long total = (long long)batch * nq;
@@ -375,10 +388,7 @@ void orc_hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, 
         const uint16_t **rows = (const uint16_t **)malloc(sizeof(uint16_t *) * (size_t)(nv + W + 1));
         long long n = 0;
         for (long long j = 0; j < nv; ++j) rows[n++] = kv + ((size_t)b * N + j) * D;
-        for (long long u = t - W + 1; u <= t; ++u) {
-            if (u < 0 || u >= T) continue;
-            rows[n++] = win + ((size_t)b * T + u) * D;
-        }
+        n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
         attend_one(q + (size_t)bq * H * D, q_gain, H, D, scale, eps, rows, n,
                    out + (size_t)bq * H * D);
         free(rows);

@@ -1,0 +1,118 @@
+"""C-ABI tests that need no GPU: the library loads, exports every function
+include/csa.h declares, and rejects bad arguments on the host before any
+launch (so these run in a container without a CUDA device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_compressed_06_b200 as csa
+from long_context_compressed_06_b200 import build as csa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    csa_build.build()
+    return csa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:csa|hca)_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_pipeline_calls():
+    names = declared_functions()
+    for n in ("csa_compress", "csa_index", "csa_index_fp4", "csa_quantize_fp4", "csa_topk", "csa_attend",
+              "hca_attend", "csa_sync_status", "csa_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_strerror_and_version(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert csa.strerror(code)
+    assert "unknown" in csa.strerror(17)
+    assert lib.csa_version() >= 10000
+
+
+NULL = None
+A16 = ctypes.c_void_p(0x10000)      # a 16-byte aligned fake device address (never dereferenced)
+A16b = ctypes.c_void_p(0x20000)
+MIS = ctypes.c_void_p(0x10008)      # misaligned
+
+
+def test_compress_validation(lib):
+    f = lib.csa_compress
+    assert f(NULL, A16, A16, 1, 64, 64, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_INVALID
+    assert f(MIS, A16, A16, 1, 64, 64, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, A16, A16, 1, 64, 60, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_INVALID   # d % 8
+    assert f(A16, A16, A16, 1, 3, 64, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_INVALID    # T < m
+    assert f(A16, A16, A16, 0, 64, 64, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_INVALID   # batch
+    assert f(A16, A16, A16, 1, 64, 64, 4, 1, NULL, -1.0, A16b, NULL) == csa.CSA_ERR_INVALID   # eps
+    assert f(A16, A16, A16, 1, 4096, 2048, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
+    assert f(A16, A16, A16, 1, 4096, 64, 512, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
+
+
+def test_index_validation(lib):
+    f = lib.csa_index
+    ok = (A16, A16, A16, A16)
+    assert f(NULL, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID
+    assert f(*ok, 1, 1, 100, 64, 120, 4, A16b, NULL) == csa.CSA_ERR_INVALID          # d_I % 16
+    assert f(*ok, 1, 1, 0, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID            # N
+    assert f(*ok, 1, 1, 100, 64, 128, 0, A16b, NULL) == csa.CSA_ERR_INVALID          # m
+    assert f(*ok, 1, 1, 100, 512, 128, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED     # H_I
+    assert f(*ok, 1, 1, 100, 64, 128, 4, MIS, NULL) == csa.CSA_ERR_INVALID
+    g = lib.csa_index_fp4
+    assert g(A16, NULL, A16, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID
+
+
+def test_quantize_validation(lib):
+    f = lib.csa_quantize_fp4
+    assert f(A16, 10, 24, A16b, A16, NULL) == csa.CSA_ERR_INVALID   # d % 16
+    assert f(A16, 0, 32, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+    assert f(MIS, 1, 32, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+
+
+def test_topk_validation(lib):
+    f = lib.csa_topk
+    assert f(A16, A16, 1, 1, 100, 4, 0, A16b, NULL, 0, NULL) == csa.CSA_ERR_INVALID       # k
+    assert f(A16, A16, 1, 1, 100, 4, 9000, A16b, NULL, 0, NULL) == csa.CSA_ERR_UNSUPPORTED
+    assert f(A16, A16, 1, 1, 1 << 20, 4, 64, A16b, NULL, 0, NULL) == csa.CSA_ERR_UNSUPPORTED
+    assert lib.csa_topk_workspace_bytes(8, 1, 32768, 1024) == 0
+
+
+def test_attend_validation_and_workspace(lib):
+    f = lib.csa_attend
+    args = dict(q=A16, g=NULL, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048, W=16, pos=A16, b=1, nq=1, H=8,
+                D=64, scale=0.125, eps=1e-6, out=A16b)
+
+    def call(ws=NULL, wsb=0, **kw):
+        a = dict(args, **kw)
+        return f(a["q"], a["g"], a["kv"], a["N"], a["idx"], a["k"], a["win"], a["p0"], a["T"], a["W"], a["pos"],
+                 a["b"], a["nq"], a["H"], a["D"], a["scale"], a["eps"], a["out"], ws, wsb, NULL)
+
+    assert call(q=NULL) == csa.CSA_ERR_INVALID
+    assert call(W=0) == csa.CSA_ERR_INVALID
+    assert call(p0=-1) == csa.CSA_ERR_INVALID
+    assert call(T=0) == csa.CSA_ERR_INVALID
+    assert call(D=96) == csa.CSA_ERR_UNSUPPORTED
+    assert call(H=256) == csa.CSA_ERR_UNSUPPORTED
+    need = lib.csa_attend_workspace_bytes(1, 1, 8, 64, 64 + 16)
+    assert need > 0   # a single query is split over several CTAs
+    assert call(ws=A16, wsb=need - 1) == csa.CSA_ERR_WORKSPACE
+    assert call(ws=MIS, wsb=need) == csa.CSA_ERR_WORKSPACE
+    h = lib.hca_attend
+    assert h(A16, NULL, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b, NULL, 0,
+             NULL) == csa.CSA_ERR_INVALID    # m
+    # workspace sizing is monotone in the key count and batch
+    assert lib.csa_attend_workspace_bytes(8, 1, 128, 512, 1152) >= lib.csa_attend_workspace_bytes(1, 1, 128, 512, 1152)

@@ -1,0 +1,269 @@
+"""GPU parity: every kernel, called through the C ABI, against the float64
+oracle on the same seeded input bits.
+
+Tolerances (the arithmetic is fp32 on bf16/FP4 inputs; a bf16 output carries
+a relative rounding error of at most 2^-9):
+  * compress: |gpu - oracle| <= 8e-3 * max|oracle row| per entry;
+  * index (bf16): |gpu - oracle| <= 1e-3 * max|S| per query (fp32 sums of 128
+    products, 64 heads), -inf pattern exact;
+  * top-k on identical fp32 scores: identical index sets (both sides break
+    ties towards the lower index), ascending order, same number of -1 slots;
+  * top-k on the kernel's own scores vs the oracle's float64 scores: the set
+    difference may only hold entries within 1e-4 * |s_k| of the k-th score;
+  * attention: max|err| <= 2e-2 * max|out| against the oracle on the same
+    selection;
+  * FP4 quantisation: bit-exact codes and scales; FP4 scores: 1e-5 * max|S|
+    (products are exact, only the fp32 summation order differs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_compressed_06_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def bits(t):
+    return W.bits(t)
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def seeded(shape, seed, kind="normal"):
+    if kind == "normal":
+        return W.normal_bf16(shape, seed, DEV)
+    return W.uniform_f32(shape, seed, DEV)
+
+
+def positions(batch, nq, ts):
+    return torch.tensor(np.array(ts, np.int32).reshape(batch, nq), device=DEV)
+
+
+# ----------------------------------------------------------------------------- compress
+@pytest.mark.parametrize("batch,T,d,m,rms,use_gain", [
+    (1, 2048, 64, 4, True, False),      # tiny workload shape
+    (2, 1037, 512, 4, True, True),      # ragged T, V4 width
+    (2, 777, 64, 3, False, False),      # odd m, no norm
+    (1, 4 * 128 + 77, 512, 128, True, False),   # HCA ratio (cluster kernel), ragged tail
+    (2, 300, 256, 16, True, True),
+    (3, 5, 64, 4, True, False),         # N = 1
+    (1, 1000, 1024, 64, True, False),   # cluster kernel, dc = 128
+])
+def test_compress_parity(cuda, batch, T, d, m, rms, use_gain):
+    A = seeded((batch, T, d), 11)
+    B = seeded((batch, T, d), 12)
+    L = torch.randn((2 * m, d), generator=torch.Generator(DEV).manual_seed(13), device=DEV)
+    gain = (seeded((d,), 14, "uniform") + 0.5) if use_gain else None
+    out = cuda.csa_compress(A, B, L, m, rms, gain, 1e-6)
+    ref = oracle.compress(bits(A), bits(B), L.cpu().numpy(), m, rms,
+                          None if gain is None else gain.cpu().numpy(), 1e-6)
+    got = f64(out)
+    assert got.shape == ref.shape
+    err = np.abs(got - ref).max(-1)
+    assert np.all(err <= 8e-3 * np.abs(ref).max(-1)), err.max()
+
+
+# ----------------------------------------------------------------------------- index
+def _index_case(batch, nq, H_I, d_I, N, m, ts, seed=20):
+    qI = seeded((batch, nq, H_I, d_I), seed)
+    w = seeded((batch, nq, H_I), seed + 1, "uniform")
+    kI = seeded((batch, N, d_I), seed + 2)
+    qp = positions(batch, nq, ts)
+    return qI, w, kI, qp
+
+
+def _check_scores(got, ref, rel):
+    assert np.array_equal(np.isneginf(got), np.isneginf(ref))
+    fin = np.isfinite(ref)
+    for q in np.ndindex(ref.shape[:-1]):
+        f = fin[q]
+        if f.any():
+            scale = np.abs(ref[q][f]).max()
+            assert np.abs(got[q][f] - ref[q][f]).max() <= rel * max(scale, 1e-30), q
+
+
+@pytest.mark.parametrize("batch,nq,H_I,d_I,N,m,ts", [
+    (1, 1, 4, 32, 512, 4, [2047]),                              # tiny workload
+    (2, 3, 64, 128, 1000, 4, [3999, 1500, 2, 3, 2222, 3998]),     # ragged N, near-zero positions
+    (1, 2, 16, 64, 130, 1, [129, 64]),
+    (1, 4, 64, 128, 4096 + 33, 4, [16531, 16500, 8000, 3]),
+    (2, 1, 8, 256, 300, 2, [599, 100]),
+])
+def test_index_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
+    qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts)
+    got = f64(cuda.csa_index(qI, w, kI, qp, m))
+    ref = oracle.index(bits(qI), w.cpu().numpy(), bits(kI), qp.cpu().numpy(), m)
+    _check_scores(got, ref, 1e-3)
+
+
+# ----------------------------------------------------------------------------- top-k
+def _check_topk_exact(got, ref, qp, m, N):
+    for q in np.ndindex(ref.shape[:-1]):
+        g, r = got[q], ref[q]
+        nv = oracle.n_visible(int(qp[q]), m, N)
+        assert np.sum(g == -1) == np.sum(r == -1) == max(0, len(r) - nv)
+        gv = g[g >= 0]
+        assert np.all(np.diff(gv) > 0), "indices must be ascending"
+        assert np.array_equal(gv, np.sort(r[r >= 0])), q
+
+
+@pytest.mark.parametrize("batch,nq,N,m,k,ts,levels", [
+    (1, 1, 512, 4, 64, [2047], 0),
+    (2, 2, 1000, 4, 64, [3999, 100, 20, 3], 0),          # n_vis < k and n_vis = 0/1
+    (1, 3, 5000, 1, 1024, [4999, 1023, 3000], 7),        # heavy ties (7 score levels)
+    (8, 1, 32768, 4, 1024, [131071] * 8, 0),             # CSA decode shape
+    (1, 2, 262144, 4, 1024, [1048575, 900000], 0),       # FP4 decode shape (cluster of 8-16)
+    (3, 1, 777, 1, 1024, [776, 500, 1023], 3),
+])
+def test_topk_exact_on_identical_scores(cuda, batch, nq, N, m, k, ts, levels):
+    r = np.random.default_rng(30 + N)
+    s = r.standard_normal((batch, nq, N)).astype(np.float32)
+    if levels:
+        s = np.floor(s * levels / 2).astype(np.float32)
+    s[0, 0, :7] = 0.0
+    s[0, 0, 7] = -0.0            # signed zero ties with +0
+    qp = positions(batch, nq, ts)
+    got = cuda.csa_topk(torch.from_numpy(s).to(DEV), qp, m, k).cpu().numpy()
+    ref = oracle.topk(s.astype(np.float64), qp.cpu().numpy(), m, k)
+    _check_topk_exact(got, ref, qp.cpu().numpy(), m, N)
+
+
+def _check_topk_band(got, ref_scores, qp, m, k, N):
+    """Set difference only inside the 1e-4 relative band around the k-th oracle score."""
+    for q in np.ndindex(ref_scores.shape[:-1]):
+        nv = oracle.n_visible(int(qp[q]), m, N)
+        s = ref_scores[q][:nv]
+        g = got[q]
+        gset = set(g[g >= 0].tolist())
+        assert len(gset) == min(k, nv)
+        if nv <= k:
+            assert gset == set(range(nv))
+            continue
+        sk = np.sort(s)[::-1][k - 1]
+        band = 1e-4 * abs(sk)
+        oset = set(oracle.topk(ref_scores[q][None, None], np.array([[qp[q]]], np.int32), m, k)[0, 0].tolist())
+        for j in gset ^ oset:
+            assert abs(s[j] - sk) <= band, (q, j, s[j], sk)
+
+
+# ----------------------------------------------------------------------------- attention
+def _random_selection(batch, nq, k, ts, m, N, seed):
+    r = np.random.default_rng(seed)
+    idx = np.full((batch, nq, k), -1, np.int32)
+    for b in range(batch):
+        for q in range(nq):
+            nv = oracle.n_visible(ts[b * nq + q], m, N)
+            n = min(k, nv)
+            idx[b, q, :n] = r.choice(nv, n, replace=False)
+            r.shuffle(idx[b, q])
+    return idx
+
+
+@pytest.mark.parametrize("batch,nq,H,D,N,T,k,Wn,m,ts,gain", [
+    (1, 1, 8, 64, 512, 2048, 64, 16, 4, [2047], False),                      # tiny workload
+    (2, 2, 128, 512, 300, 1200, 100, 128, 4, [1199, 1100, 700, 5], True),    # V4 heads, n_vis < k
+    (1, 3, 128, 512, 1024, 4096, 1024, 128, 4, [4095, 2000, 0], False),      # k = 1024, t = 0
+    (2, 1, 40, 128, 97, 400, 33, 7, 4, [399, 13], False),                    # ragged heads
+    (1, 1, 128, 256, 64, 256, 16, 1, 4, [255], False),                       # W = 1
+])
+def test_csa_attend_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts, gain):
+    q = seeded((batch, nq, H, D), 40)
+    kv = seeded((batch, N, D), 41)
+    win = seeded((batch, T, D), 42)
+    qp = positions(batch, nq, ts)
+    g = (seeded((D,), 43, "uniform") + 0.5) if gain else None
+    idx = _random_selection(batch, nq, k, ts, m, N, 44)
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale, 1e-6, g)
+    ref = oracle.attend(bits(q), bits(kv), idx, bits(win), qp.cpu().numpy(), Wn, scale, 1e-6,
+                        None if g is None else g.cpu().numpy())
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
+def test_csa_attend_window_cache_equals_full_stream(cuda):
+    """A decode window cache (win_pos0 = t-W+1, W rows) gives the same output as the whole stream."""
+    batch, H, D, N, T, k, Wn, m = 2, 128, 512, 256, 1024, 64, 128, 4
+    q = seeded((batch, 1, H, D), 50)
+    kv = seeded((batch, N, D), 51)
+    A = seeded((batch, T, D), 52)
+    qp = positions(batch, 1, [T - 1, T - 1])
+    idx = torch.from_numpy(_random_selection(batch, 1, k, [T - 1] * 2, m, N, 53)).to(DEV)
+    full = cuda.csa_attend(q, kv, idx, A, qp, Wn, D ** -0.5)
+    cache = A[:, T - Wn:].contiguous()
+    part = cuda.csa_attend(q, kv, idx, cache, qp, Wn, D ** -0.5, win_pos0=T - Wn)
+    torch.cuda.synchronize()
+    assert torch.equal(full, part)
+
+
+@pytest.mark.parametrize("batch,nq,H,D,N,m,T,Wn,ts", [
+    (2, 1, 128, 512, 600, 128, 600 * 128, 128, [600 * 128 - 1, 300 * 128 + 5]),
+    (1, 2, 8, 64, 512, 4, 2048, 16, [2047, 9]),
+    (3, 1, 64, 256, 1000, 4, 4000, 50, [3999, 2, 1234]),
+])
+def test_hca_attend_parity(cuda, batch, nq, H, D, N, m, T, Wn, ts):
+    q = seeded((batch, nq, H, D), 60)
+    kv = seeded((batch, N, D), 61)
+    qp = positions(batch, nq, ts)
+    p0 = max(0, min(ts) - Wn + 1)
+    win = seeded((batch, T - p0, D), 62)
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.hca_attend(q, kv, m, win, qp, Wn, scale, win_pos0=p0)
+    ref = oracle.hca_attend(bits(q), bits(kv), m, bits(win), qp.cpu().numpy(), Wn, scale, win_pos0=p0)
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
+# ----------------------------------------------------------------------------- FP4
+def test_quantize_fp4_bit_exact(cuda):
+    x = seeded((4096, 128), 70).float()
+    x[:, 5] *= 8
+    x[:, 77] *= 8
+    x[0:3, 0:16] = 0                                    # zero blocks
+    x[3, 0:16] = 1e-5                                   # scale underflows to e4m3 0
+    x[4, 0:16] = torch.linspace(-3e-3, 3e-3, 16)        # subnormal e4m3 scales
+    x[5, 16:32] = torch.linspace(-3000, 3000, 16)       # satfinite scale
+    x[6, 32:48] = torch.tensor([6, 3, 1.5, 0.75, 0.25, -0.25, -0.75, 5, 2.5, -5, 1.25, 1.75, 3.5, -0.1, 0, -6.])
+    xb = x.to(torch.bfloat16).contiguous()
+    p, s = cuda.csa_quantize_fp4(xb)
+    rp, rs = oracle.quantize_fp4(bits(xb))
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(p.cpu().numpy(), rp)
+
+
+@pytest.mark.parametrize("batch,nq,H_I,d_I,N,m,ts", [
+    (1, 1, 64, 128, 4096, 4, [16383]),
+    (2, 2, 16, 64, 777, 4, [3107, 50, 3000, 7]),
+])
+def test_index_fp4_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
+    qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts, seed=80)
+    q4, q4s = cuda.csa_quantize_fp4(qI)
+    k4, k4s = cuda.csa_quantize_fp4(kI)
+    got = f64(cuda.csa_index_fp4(q4, q4s, w, k4, k4s, qp, m))
+    rq4, rq4s = oracle.quantize_fp4(bits(qI))
+    rk4, rk4s = oracle.quantize_fp4(bits(kI))
+    ref = oracle.index_fp4(rq4, rq4s, w.cpu().numpy(), rk4, rk4s, qp.cpu().numpy(), m)
+    _check_scores(got, ref, 1e-5)
+
+
+# ----------------------------------------------------------------------------- failure path
+def test_bounded_wait_times_out_and_context_survives(cuda):
+    assert cuda.csa_sync_status() == 0
+    cuda.csa_set_wait_budget_ns(2_000_000)      # 2 ms
+    try:
+        cuda.csa_selftest_wait_timeout()
+        assert cuda.csa_sync_status() == cuda.CSA_ERR_TIMEOUT
+        assert cuda.csa_sync_status() == 0       # read-and-clear
+    finally:
+        cuda.csa_set_wait_budget_ns(0)
+    # the context is still usable
+    A = seeded((1, 64, 64), 90)
+    out = cuda.csa_compress(A, A, torch.zeros((8, 64), device=DEV), 4)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
