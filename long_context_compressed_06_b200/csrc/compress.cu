@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -230,17 +231,6 @@ cudaError_t run_small(const uint16_t *A, const uint16_t *B, const float *logits,
     }
     k<<<grid, 256, smem, st>>>(A, B, logits, batch, T, d, m, apply_rms, gain, eps, out, N);
     return cudaGetLastError();
-}
-
-int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
 }
 
 }  // namespace

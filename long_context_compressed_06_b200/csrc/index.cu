@@ -11,10 +11,16 @@ int launch_index_fp4_simt(const uint8_t *q4, const uint8_t *q4s, const float *w,
                           const uint8_t *k4s, const int *q_pos, int batch, int nq, long long N, int H_I,
                           int d_I, int m, float *scores, cudaStream_t st);
 
+bool index_tc_supported(int H_I, int d_I);
+int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
+                    int nq, long long N, int H_I, int d_I, int m, float *scores, const DevCtx &ctx,
+                    cudaStream_t st);
+
 int launch_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
                  int nq, long long N, int H_I, int d_I, int m, float *scores, const DevCtx &ctx,
                  cudaStream_t st) {
-    (void)ctx;
+    if (index_tc_supported(H_I, d_I))
+        return launch_index_tc(q_idx, w, k_idx, q_pos, batch, nq, N, H_I, d_I, m, scores, ctx, st);
     return launch_index_simt(q_idx, w, k_idx, q_pos, batch, nq, N, H_I, d_I, m, scores, st);
 }
 

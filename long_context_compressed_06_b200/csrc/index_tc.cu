@@ -1,0 +1,292 @@
+// index_tc.cu -- lightning-indexer scores on the 5th-generation tensor cores.
+//
+//   S[q][s] = sum_h w[q][h] * max(0, q_I[q][h] . K_I[s])   (s < n_vis(t_q), else -inf)
+// ("DeepSeek v4" -> "sparse selection Lightning Indexer").
+//
+// GEMM view per sequence: D[s][(q,h)] = K_I[s] . q_I[q][h], M = 128 keys per
+// tile, N = NQ queries x H_pad heads (<= 256), K = d_I.  The keys are the
+// streamed operand (A); the NQ queries' heads (B) stay in shared memory while
+// the CTA walks key tiles.  Each TMEM lane holds one key, so the epilogue
+// sum_h w_h * ReLU(.) is a loop over columns inside one thread, and a warp
+// stores 32 consecutive scores.
+//
+// Warp roles (192 threads):  warp 0 -- TMA producer (key tiles into a STAGES
+// ring, query tile once per query group); warp 1 -- TMEM owner and MMA issuer
+// (one thread; tcgen05.mma kind::f16, fp32 accumulate, two accumulator
+// buffers); warps 2..5 -- epilogue (tcgen05.ld, ReLU, weighted head sum,
+// causal mask, store).  Every mbarrier wait is bounded (csa_sync_status
+// reports a timeout).  Decode is HBM bound on the key stream (the MMA work per
+// tile is ~1/5 of the time the tile takes to arrive), prefill is bound by the
+// tensor cores and the epilogue.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTileKeys = 128;
+constexpr int kMaxStages = 6;
+
+struct IndexTcParams {
+    const float *w;       // [batch][nq][H_I]
+    const int *q_pos;     // [batch][nq]
+    float *scores;        // [batch][nq][N]
+    long long N;
+    int nq, H_I, H_pad, d_I, m, NQ;
+    int groups_per_batch, n_ktiles;
+    long long total_work;
+    int stages, nchunk, chunk_elems, row_bytes, layout;
+    uint32_t stage_bytes, q_bytes, idesc;
+    int n_cols;           // N of the MMA = NQ * H_pad
+    uint32_t tmem_cols;   // allocated columns (2 accumulators)
+    DevCtx ctx;
+};
+
+struct WorkItem {
+    long long grp;
+    int kt;
+    bool first_of_group, last_of_group;
+};
+
+CSA_DEVINL WorkItem work_item(const IndexTcParams &p, long long w, long long w0, long long w1) {
+    WorkItem it;
+    it.grp = w / p.n_ktiles;
+    it.kt = (int)(w - it.grp * p.n_ktiles);
+    it.first_of_group = (w == w0) || it.kt == 0;
+    it.last_of_group = (w == w1 - 1) || it.kt == p.n_ktiles - 1;
+    return it;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                    const IndexTcParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned carve-up: key stages | query tile | weights | barriers
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *k_smem = base;
+    uint8_t *q_smem = k_smem + (size_t)p.stages * p.stage_bytes;
+    float *w_s = reinterpret_cast<float *>(q_smem + p.q_bytes);          // [NQ][H_pad]
+    int *nvis_s = reinterpret_cast<int *>(w_s + p.NQ * p.H_pad);         // [NQ]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+        (reinterpret_cast<uintptr_t>(nvis_s + p.NQ) + 7) & ~uintptr_t(7));
+    uint64_t *full = bars, *empty = bars + kMaxStages;
+    uint64_t *tfull = bars + 2 * kMaxStages, *tempty = tfull + 2;
+    uint64_t *qfull = tempty + 2, *qempty = qfull + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long w0 = (long long)blockIdx.x * p.total_work / gridDim.x;
+    const long long w1 = (long long)(blockIdx.x + 1) * p.total_work / gridDim.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 4);
+        }
+        mbar_init(qfull, 1);
+        mbar_init(qempty, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tc::prefetch_tmap(&kmap);
+        tc::prefetch_tmap(&qmap);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ TMA producer
+        long long it = 0, gi = 0;
+        for (long long w = w0; w < w1; ++w) {
+            const WorkItem wi = work_item(p, w, w0, w1);
+            const int b = (int)(wi.grp / p.groups_per_batch);
+            const int g = (int)(wi.grp - (long long)b * p.groups_per_batch);
+            if (wi.first_of_group) {
+                if (!mbar_wait(smem_u32(qempty), (uint32_t)((gi & 1) ^ 1), p.ctx, abort_flag)) break;
+                mbar_arrive_expect_tx(smem_u32(qfull), p.q_bytes);
+                for (int c = 0; c < p.nchunk; ++c)
+                    tc::tma_load_4d(smem_u32(q_smem + (size_t)c * p.n_cols * p.row_bytes), &qmap, smem_u32(qfull),
+                                    c * p.chunk_elems, 0, g * p.NQ, b);
+                ++gi;
+            }
+            const int st = (int)(it % p.stages);
+            const uint32_t ph = (uint32_t)((it / p.stages) & 1);
+            if (!mbar_wait(smem_u32(empty + st), ph ^ 1u, p.ctx, abort_flag)) break;
+            mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes);
+            uint8_t *dst = k_smem + (size_t)st * p.stage_bytes;
+            for (int c = 0; c < p.nchunk; ++c)
+                tc::tma_load_3d(smem_u32(dst + (size_t)c * kTileKeys * p.row_bytes), &kmap, smem_u32(full + st),
+                                c * p.chunk_elems, wi.kt * kTileKeys, b);
+            ++it;
+        }
+        // drain: wait (bounded) for the copies this thread issued last into each stage
+        for (long long j = std::max(0LL, it - p.stages); j < it; ++j)
+            mbar_wait(smem_u32(full + (j % p.stages)), (uint32_t)((j / p.stages) & 1), p.ctx, nullptr);
+        if (gi > 0) mbar_wait(smem_u32(qfull), (uint32_t)((gi - 1) & 1), p.ctx, nullptr);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        long long it = 0, gi = 0;
+        const uint32_t sbo = 8u * p.row_bytes;
+        for (long long w = w0; w < w1; ++w) {
+            const WorkItem wi = work_item(p, w, w0, w1);
+            if (wi.first_of_group) {
+                if (!mbar_wait(smem_u32(qfull), (uint32_t)(gi & 1), p.ctx, abort_flag)) break;
+                ++gi;
+            }
+            const int acc = (int)(it & 1);
+            const uint32_t aph = (uint32_t)((it >> 1) & 1);
+            if (!mbar_wait(smem_u32(tempty + acc), aph ^ 1u, p.ctx, abort_flag)) break;
+            const int st = (int)(it % p.stages);
+            const uint32_t ph = (uint32_t)((it / p.stages) & 1);
+            if (!mbar_wait(smem_u32(full + st), ph, p.ctx, abort_flag)) break;
+            tc::fence_after_sync();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols);
+            const uint32_t a0 = smem_u32(k_smem + (size_t)st * p.stage_bytes);
+            const uint32_t b0 = smem_u32(q_smem);
+            uint32_t accumulate = 0;
+            for (int c = 0; c < p.nchunk; ++c) {
+                for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
+                    const uint64_t ad = tc::smem_desc(a0 + c * kTileKeys * p.row_bytes + kk * 32, sbo, p.layout);
+                    const uint64_t bd = tc::smem_desc(b0 + c * p.n_cols * p.row_bytes + kk * 32, sbo, p.layout);
+                    tc::mma_f16(d_tmem, ad, bd, p.idesc, accumulate);
+                    accumulate = 1;
+                }
+            }
+            tc::mma_commit(smem_u32(empty + st));
+            tc::mma_commit(smem_u32(tfull + acc));
+            if (wi.last_of_group) tc::mma_commit(smem_u32(qempty));
+            ++it;
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int row = quarter * 32 + lane;
+        const int et = threadIdx.x - 64;  // 0..127
+        long long it = 0;
+        for (long long w = w0; w < w1; ++w) {
+            const WorkItem wi = work_item(p, w, w0, w1);
+            const int b = (int)(wi.grp / p.groups_per_batch);
+            const int g = (int)(wi.grp - (long long)b * p.groups_per_batch);
+            if (wi.first_of_group) {
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                for (int i = et; i < p.NQ * p.H_pad; i += 128) {
+                    const int qi = i / p.H_pad, h = i - qi * p.H_pad;
+                    const int q = g * p.NQ + qi;
+                    w_s[i] = (q < p.nq && h < p.H_I) ? __ldg(p.w + ((size_t)b * p.nq + q) * p.H_I + h) : 0.f;
+                }
+                for (int qi = et; qi < p.NQ; qi += 128) {
+                    const int q = g * p.NQ + qi;
+                    nvis_s[qi] = q < p.nq ? (int)n_visible(__ldg(p.q_pos + (size_t)b * p.nq + q), p.m, p.N) : 0;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            }
+            const int acc = (int)(it & 1);
+            const uint32_t aph = (uint32_t)((it >> 1) & 1);
+            if (!mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag)) break;
+            tc::fence_after_sync();
+            const long long s = (long long)wi.kt * kTileKeys + row;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.n_cols);
+            for (int qi = 0; qi < p.NQ; ++qi) {
+                const int q = g * p.NQ + qi;
+                if (q >= p.nq) break;
+                float score = 0.f;
+                for (int hc = 0; hc < p.H_pad; hc += 16) {
+                    float v[16];
+                    tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc), v);
+                    tc::tmem_wait_ld();
+                    const float *ws = w_s + qi * p.H_pad + hc;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) score = fmaf(ws[i], fmaxf(v[i], 0.f), score);
+                }
+                if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nvis_s[qi] ? score : -INFINITY;
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
+            ++it;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+}
+
+}  // namespace
+
+// The tensor-core path takes d_I in {32, 64, 128, 256} and up to 256 heads.
+bool index_tc_supported(int H_I, int d_I) {
+    return (d_I == 32 || d_I == 64 || d_I == 128 || d_I == 256) && H_I >= 1 && H_I <= 256;
+}
+
+int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
+                    int nq, long long N, int H_I, int d_I, int m, float *scores, const DevCtx &ctx,
+                    cudaStream_t st) {
+    IndexTcParams p = {};
+    p.w = w; p.q_pos = q_pos; p.scores = scores; p.N = N; p.nq = nq; p.H_I = H_I; p.d_I = d_I; p.m = m;
+    p.ctx = ctx;
+    p.H_pad = std::max(16, (H_I + 15) / 16 * 16);
+    p.chunk_elems = d_I >= 64 ? 64 : d_I;           // one swizzle row of bf16
+    p.row_bytes = p.chunk_elems * 2;
+    p.layout = p.row_bytes == 128 ? tc::kLayoutSw128 : tc::kLayoutSw64;
+    p.nchunk = d_I / p.chunk_elems;
+    p.stage_bytes = (uint32_t)(kTileKeys * d_I * 2);
+    // queries per tile: as many as fit in N <= 256 and in shared memory
+    const size_t smem_cap = 200 * 1024;
+    int NQ = std::max(1, std::min(nq, std::min(16, 256 / p.H_pad)));
+    while (NQ > 1 && (size_t)NQ * p.H_pad * d_I * 2 + 2 * p.stage_bytes > smem_cap) NQ /= 2;
+    p.NQ = NQ;
+    p.n_cols = NQ * p.H_pad;
+    p.q_bytes = (uint32_t)(p.n_cols * d_I * 2);
+    p.stages = (int)std::min<size_t>(kMaxStages, (smem_cap - p.q_bytes) / p.stage_bytes);
+    if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
+    p.idesc = tc::idesc_f16(p.n_cols, true);
+    uint32_t cols = 32;
+    while (cols < 2u * (uint32_t)p.n_cols) cols *= 2;
+    p.tmem_cols = cols;
+    p.groups_per_batch = (nq + NQ - 1) / NQ;
+    p.n_ktiles = (int)((N + kTileKeys - 1) / kTileKeys);
+    p.total_work = (long long)batch * p.groups_per_batch * p.n_ktiles;
+
+    const CUtensorMapSwizzle sw = p.row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap kmap, qmap;
+    {
+        const uint64_t dims[3] = {(uint64_t)d_I, (uint64_t)N, (uint64_t)batch};
+        const uint64_t strides[2] = {(uint64_t)d_I * 2, (uint64_t)N * d_I * 2};
+        const uint32_t box[3] = {(uint32_t)p.chunk_elems, (uint32_t)kTileKeys, 1};
+        if (!encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k_idx, dims, strides, box, sw))
+            return CSA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[4] = {(uint64_t)d_I, (uint64_t)H_I, (uint64_t)nq, (uint64_t)batch};
+        const uint64_t strides[3] = {(uint64_t)d_I * 2, (uint64_t)H_I * d_I * 2, (uint64_t)nq * H_I * d_I * 2};
+        const uint32_t box[4] = {(uint32_t)p.chunk_elems, (uint32_t)p.H_pad, (uint32_t)NQ, 1};
+        if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q_idx, dims, strides, box, sw))
+            return CSA_ERR_CUDA;
+    }
+    const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + p.q_bytes + (size_t)NQ * p.H_pad * 4 + NQ * 4 +
+                        8 + (2 * kMaxStages + 6) * 8 + 16;
+    if (cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const int grid = (int)std::min<long long>(p.total_work, num_sms());
+    index_tc_kernel<<<grid, kThreads, smem, st>>>(kmap, qmap, p);
+    return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
+}  // namespace csa

@@ -94,6 +94,10 @@ def _check_scores(got, ref, rel):
     (1, 2, 16, 64, 130, 1, [129, 64]),
     (1, 4, 64, 128, 4096 + 33, 4, [16531, 16500, 8000, 3]),
     (2, 1, 8, 256, 300, 2, [599, 100]),
+    (1, 9, 64, 128, 2000, 4, [7999 - 3 * i for i in range(9)]),     # query groups of 4 (+1 ragged)
+    (3, 5, 4, 32, 700, 4, [2799, 2000, 1000, 10, 3] * 3),          # H_I padded to 16, 5 queries per tile
+    (1, 2, 8, 48, 200, 4, [799, 400]),                             # d_I = 48: CUDA-core kernel
+    (8, 1, 64, 128, 32768, 4, [131071] * 8),                       # CSA decode shape
 ])
 def test_index_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
     qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts)
