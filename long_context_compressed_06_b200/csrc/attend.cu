@@ -54,9 +54,27 @@ int launch_attend_combine(const AttendArgs &a, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
+bool attend_tc_supported(int H, int D);
+void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long long *kps);
+int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st);
+
+// Split plan of the kernel that will run for these shapes (the tensor-core
+// kernel whenever it supports them).
+static void plan_splits(long long n_bq, int H, int D, long long max_keys, int *splits, long long *kps) {
+    if (attend_tc_supported(H, D)) {
+        attend_tc_plan(n_bq, H, max_keys, splits, kps);
+    } else {
+        *splits = attend_simt_splits(n_bq, H, max_keys);
+        *kps = (max_keys + *splits - 1) / *splits;
+    }
+}
+
 size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys) {
     const long long n_bq = (long long)batch * nq;
-    return ws_bytes_for(n_bq, H, D, attend_simt_splits(n_bq, H, max_keys));
+    int splits;
+    long long kps;
+    plan_splits(n_bq, H, D, max_keys, &splits, &kps);
+    return ws_bytes_for(n_bq, H, D, splits);
 }
 
 int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
@@ -64,15 +82,13 @@ int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, lo
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
                   size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
-    (void)ctx;
     AttendArgs a = {};
     a.q = q; a.q_gain = q_gain; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
     a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
     a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
     if (a.n_bq == 0) return CSA_OK;
     const long long max_keys = (dense ? N : (long long)k) + W;
-    a.splits = attend_simt_splits(a.n_bq, H, max_keys);
-    a.keys_per_split = (max_keys + a.splits - 1) / a.splits;
+    plan_splits(a.n_bq, H, D, max_keys, &a.splits, &a.keys_per_split);
     const size_t need = ws_bytes_for(a.n_bq, H, D, a.splits);
     if (need > 0) {
         if (!ws || ws_bytes < need) return CSA_ERR_WORKSPACE;
@@ -80,6 +96,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, lo
         a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(float));
     }
+    if (attend_tc_supported(H, D)) return launch_attend_tc(a, ctx, st);
     return launch_attend_simt(a, st);
 }
 

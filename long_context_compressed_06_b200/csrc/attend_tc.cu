@@ -1,0 +1,580 @@
+// attend_tc.cu -- CSA / HCA core attention on the 5th-generation tensor cores.
+//
+// One query at a time: H (<= 128) RMSNorm'd query heads share one KV head of
+// dim D (K = V); the key set is the selected compressed entries (CSA) or all
+// visible entries (HCA) plus the sliding window of raw stream-A rows
+// (techniques map rows "Grouped-query attention", "Sliding-window attention",
+// "QK normalization").  Flash-style, per tile of 64 keys:
+//   S = Q_hat K^T   (tcgen05.mma M = 64 heads, N = 64 keys, fp32 in TMEM)
+//   online softmax in fp32, log2 domain; the running max is raised only when
+//   it grows by more than 2^8, so the O rescale in TMEM is rare
+//   O += P V        (tcgen05.mma M = 64 heads, N <= 256 dims per MMA, V read
+//                    MN-major from the same shared-memory tile as K)
+//
+// TMEM budget: O for 128 heads x 512 dims in fp32 would take all of one SM's
+// tensor memory, so each CTA owns 64 heads (M = 64).  An M = 64 accumulator
+// occupies lanes 0-15 of every 32-lane sub-partition; O sits there (all D
+// columns) and the two S buffers sit at lane offset 16 (columns 0..127).  The
+// 16x32bx2 TMEM access shape keeps every warp inside the lane half it means
+// to touch.  The two head halves of a query are independent CTAs: no cluster,
+// no exchange; each streams the gathered rows itself (the second read of a
+// row is an L2 hit).
+//
+// Warp roles (256 threads): warp 0 TMEM owner + MMA issuer (one thread);
+// warps 1..3 gather the key rows with 16-byte cp.async into the 128-byte
+// swizzled layout (one 512-byte coalesced row segment per warp instruction);
+// warps 4..7 softmax and output, two threads per head (keys 0-31 / 32-63,
+// D/2 output columns each); all eight warps build Q_hat for each query.  Work
+// items are (query, key split, head half); splits write fp32 partials +
+// (max, sum) that attend_combine merges in a fixed order.  Every wait is
+// bounded.
+#include <algorithm>
+
+#include "attend_common.cuh"
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTileKeys = 64;
+constexpr int kHeads = 64;          // heads per CTA (M of every MMA)
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kProducerWarp0 = 1, kProducerWarps = 3;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kMaxStages = 4;
+
+struct AttTcParams {
+    AttendArgs a;
+    int HH;             // head halves per query (1 or 2)
+    int stages;
+    uint32_t idesc_qk, idesc_pv;
+    long long n_work;   // n_bq * splits * HH
+    DevCtx ctx;
+};
+
+template <int D>
+struct Layout {
+    static constexpr int kChunks = D / 64;                       // 64-dim, 128-byte swizzle rows
+    static constexpr uint32_t kQBytes = kHeads * D * 2;          // [kChunks][64 heads][128 B]
+    static constexpr uint32_t kStageBytes = kTileKeys * D * 2;   // [kChunks][64 keys][128 B]
+    static constexpr uint32_t kPBytes = kHeads * kTileKeys * 2;  // [64 heads][128 B]
+    static constexpr int kPvN = D < 256 ? D : 256;               // N of one P.V MMA
+};
+
+struct Smem {
+    uint8_t *q, *k, *p;
+    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready;
+    uint32_t *tmem_slot;
+    int *abort_flag;
+};
+
+template <int D>
+CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
+    using Lt = Layout<D>;
+    Smem s;
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    s.q = base;
+    s.k = s.q + Lt::kQBytes;
+    s.p = s.k + (size_t)stages * Lt::kStageBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s.p + 2 * Lt::kPBytes);
+    s.kfull = bars;
+    s.kempty = bars + kMaxStages;
+    s.sfull = bars + 2 * kMaxStages;
+    s.sempty = s.sfull + 2;
+    s.pfull = s.sempty + 2;
+    s.pempty = s.pfull + 2;
+    s.oready = s.pempty + 2;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.oready + 1);
+    s.abort_flag = reinterpret_cast<int *>(s.tmem_slot + 1);
+    return s;
+}
+
+template <int D>
+size_t smem_bytes(int stages) {
+    using Lt = Layout<D>;
+    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (2 * kMaxStages + 9) * 8 + 16;
+}
+
+// ---------------------------------------------------------------- TMEM, 16-lane access shape
+// 16x32bx2 with a split offset of 32 columns: threads 0-15 read lanes
+// base..base+15 at columns [c, c+32), threads 16-31 the same lanes at
+// columns [c+32, c+64).
+CSA_DEVINL void tmem_ld_half32(uint32_t taddr, float v[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+CSA_DEVINL void tmem_st_half32(uint32_t taddr, const float v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+// ---------------------------------------------------------------- key enumeration
+// Key e of one query: e < nsel4 -> selection slot e (slots >= nsel are padding),
+// else window row e - nsel4.  nsel4 = nsel rounded up to a multiple of 4.
+struct Keys {
+    long long nsel, nsel4, nwin, u0, total;
+};
+
+CSA_DEVINL Keys query_keys(const AttendArgs &a, long long t) {
+    Keys k;
+    k.nsel = a.dense ? n_visible(t, a.m, a.N) : a.k;
+    k.nsel4 = (k.nsel + 3) & ~3LL;
+    long long u0 = t - a.W + 1;
+    u0 = u0 < 0 ? 0 : u0;
+    k.u0 = u0 < a.win_pos0 ? a.win_pos0 : u0;
+    const long long last = a.win_pos0 + a.win_rows - 1;
+    const long long u1 = t < last ? t : last;
+    k.nwin = u1 >= k.u0 ? u1 - k.u0 + 1 : 0;
+    k.total = k.nsel4 + k.nwin;
+    return k;
+}
+
+// Row of key e (invalid keys read a valid row; their scores are masked).
+CSA_DEVINL const uint16_t *key_ptr(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e) {
+    if (e < ks.nsel4) {
+        long long j = 0;
+        if (e < ks.nsel) {
+            j = a.dense ? e : (long long)__ldg(a.idx + bq * a.k + e);
+            if (j < 0 || j >= a.N) j = 0;
+        }
+        return a.kv + ((size_t)b * a.N + j) * a.D;
+    }
+    long long w = e - ks.nsel4;
+    w = w < ks.nwin ? w : ks.nwin - 1;
+    w = w < 0 ? 0 : w;
+    return a.win + ((size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + w) * a.D;
+}
+
+CSA_DEVINL bool key_valid(const AttendArgs &a, const Keys &ks, long long bq, long long e, long long e_end) {
+    if (e >= e_end) return false;
+    if (e < ks.nsel4) {
+        if (e >= ks.nsel) return false;
+        if (a.dense) return true;
+        const int j = __ldg(a.idx + bq * a.k + e);
+        return j >= 0 && j < a.N;
+    }
+    return e - ks.nsel4 < ks.nwin;
+}
+
+// Validity of the 64 keys of a tile as a bit mask (every lane of the warp gets it).
+CSA_DEVINL uint64_t tile_mask(const AttendArgs &a, const Keys &ks, long long bq, long long ebase, long long e_end) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lo = __ballot_sync(0xffffffffu, key_valid(a, ks, bq, ebase + lane, e_end));
+    const uint32_t hi = __ballot_sync(0xffffffffu, key_valid(a, ks, bq, ebase + 32 + lane, e_end));
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the outcome is broadcast.
+CSA_DEVINL bool warp_wait(uint32_t bar, uint32_t parity, const DevCtx &ctx, volatile int *abort) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ctx, abort);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+// ---------------------------------------------------------------- Q_hat
+// Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16, for this CTA's 64 heads,
+// into the swizzled K-major tile [D/64][64 heads][128 B].  Each warp loads all
+// of its 8 heads before reducing (8 rows in flight).
+template <int D>
+CSA_DEVINL void build_q(const AttendArgs &a, const Smem &s, long long bq, int head0) {
+    constexpr int DPL = D / 32;   // dims per lane
+    constexpr int HPW = kHeads / (kThreads / 32);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float x[HPW][DPL];
+#pragma unroll
+    for (int i = 0; i < HPW; ++i) {
+        const int h = head0 + warp * HPW + i;
+        if (h < a.H) {
+            const uint16_t *row = a.q + ((size_t)bq * a.H + h) * D + lane * DPL;
+            if constexpr (DPL >= 8) {
+#pragma unroll
+                for (int c = 0; c < DPL; c += 8) unpack8(ldg16(row + c), x[i] + c);
+            } else {
+#pragma unroll
+                for (int c = 0; c < DPL; c += 2) {
+                    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(row + c));
+                    x[i][c] = bf16_lo(v);
+                    x[i][c + 1] = bf16_hi(v);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < DPL; ++c) x[i][c] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < HPW; ++i) {
+        const int hl = warp * HPW + i;
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < DPL; ++c) ss = fmaf(x[i][c], x[i][c], ss);
+        ss = warp_sum(ss);
+        const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
+#pragma unroll
+        for (int c = 0; c < DPL; c += 2) {
+            const int d = lane * DPL + c;
+            const float g0 = a.q_gain ? __ldg(a.q_gain + d) : 1.f;
+            const float g1 = a.q_gain ? __ldg(a.q_gain + d + 1) : 1.f;
+            uint8_t *dst = s.q + (size_t)(d >> 6) * kHeads * 128 + hl * 128 + ((((d & 63) >> 3) ^ (hl & 7)) << 4) +
+                           (d & 7) * 2;
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(x[i][c] * r * g0, x[i][c + 1] * r * g1);
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParams p) {
+    using Lt = Layout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const Smem s = carve<D>(smem_raw, p.stages);
+    const AttendArgs &a = p.a;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.stages; ++i) {
+            mbar_init(s.kfull + i, kProducerWarps * 32);  // one cp.async completion arrive per producer thread
+            mbar_init(s.kempty + i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s.sfull + i, 1);
+            mbar_init(s.sempty + i, 128);
+            mbar_init(s.pfull + i, 128);
+            mbar_init(s.pempty + i, 1);
+        }
+        mbar_init(s.oready, 1);
+        *s.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(smem_u32(s.tmem_slot), 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *s.tmem_slot;
+    const uint32_t tmem_o = tmem;                  // lanes 0-15 of each sub-partition, columns 0..D-1
+    const uint32_t tmem_s = tmem + (16u << 16);    // lanes 16-31, columns 0..127 (two S buffers)
+
+    long long jt = 0;  // tiles processed by this CTA (ring and phase position, identical in every role)
+    for (long long wi = blockIdx.x; wi < p.n_work; wi += gridDim.x) {
+        const int hh = (int)(wi % p.HH);
+        const long long rest = wi / p.HH;
+        const int split = (int)(rest % a.splits);
+        const long long bq = rest / a.splits;
+        const long long b = bq / a.nq;
+        const int head0 = hh * kHeads;
+        const long long t = __ldg(a.q_pos + bq);
+        const Keys ks = query_keys(a, t);
+        const long long e0 = (long long)split * a.keys_per_split;
+        const long long e1 = std::min(ks.total, e0 + a.keys_per_split);
+        const int ntiles = e1 > e0 ? (int)((e1 - e0 + kTileKeys - 1) / kTileKeys) : 0;
+
+        build_q<D>(a, s, bq, head0);
+        tc::fence_proxy_async_smem();
+        __syncthreads();
+
+        if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
+            // -------------------------------------------------------- producers (cp.async gather)
+            const int pw = warp - kProducerWarp0;
+            for (int j = 0; j < ntiles; ++j) {
+                const long long g = jt + j;
+                const int st = (int)(g % p.stages);
+                if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag))
+                    break;
+                uint8_t *stage = s.k + (size_t)st * Lt::kStageBytes;
+                const long long ebase = e0 + (long long)j * kTileKeys;
+                for (int key = pw; key < kTileKeys; key += kProducerWarps) {
+                    const uint16_t *row = key_ptr(a, ks, b, bq, std::min(ebase + key, e1 - 1));
+#pragma unroll
+                    for (int u = lane; u < D / 8; u += 32) {  // 16-byte units of the row
+                        const uint32_t dst = smem_u32(stage + (size_t)(u >> 3) * kTileKeys * 128 + key * 128 +
+                                                      (((u & 7) ^ (key & 7)) << 4));
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(row + u * 8)
+                                     : "memory");
+                    }
+                }
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
+                             : "memory");
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        } else if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- MMA issuer
+            auto pv = [&](long long g, bool first) -> bool {
+                const int pb = (int)(g & 1);
+                if (!mbar_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1), p.ctx, s.abort_flag)) return false;
+                tc::fence_after_sync();
+                const int st = (int)(g % p.stages);
+                const uint32_t pa = smem_u32(s.p + pb * Lt::kPBytes);
+                const uint32_t vb = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+#pragma unroll
+                for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+                    const uint64_t ad = tc::smem_desc(pa + kk * 32, 1024, tc::kLayoutSw128);
+#pragma unroll
+                    for (int n0 = 0; n0 < D; n0 += Lt::kPvN) {
+                        // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes apart (LBO),
+                        // 8-key groups 1024 bytes apart (SBO); a K step is 16 keys
+                        const uint64_t bd = tc::smem_desc_lbo(vb + (n0 / 64) * kTileKeys * 128 + kk * 16 * 128,
+                                                              kTileKeys * 128, 1024, tc::kLayoutSw128);
+                        tc::mma_f16(tmem_o + n0, ad, bd, p.idesc_pv, (first && kk == 0) ? 0u : 1u);
+                    }
+                }
+                tc::mma_commit(smem_u32(s.kempty + st));
+                tc::mma_commit(smem_u32(s.pempty + pb));
+                tc::mma_commit(smem_u32(s.oready));
+                return true;
+            };
+            bool ok = true;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const long long g = jt + j;
+                const int st = (int)(g % p.stages);
+                const int sb = (int)(g & 1);
+                if (!mbar_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1), p.ctx, s.abort_flag)) break;
+                if (!mbar_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1), p.ctx, s.abort_flag)) break;
+                tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+                tc::fence_after_sync();
+                const uint32_t qa = smem_u32(s.q), kb = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+#pragma unroll
+                for (int c = 0; c < Lt::kChunks; ++c)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = tc::smem_desc(qa + c * kHeads * 128 + kk * 32, 1024, tc::kLayoutSw128);
+                        const uint64_t bd = tc::smem_desc(kb + c * kTileKeys * 128 + kk * 32, 1024, tc::kLayoutSw128);
+                        tc::mma_f16(tmem_s + sb * kTileKeys, ad, bd, p.idesc_qk, (c | kk) ? 1u : 0u);
+                    }
+                tc::mma_commit(smem_u32(s.sfull + sb));
+                if (j > 0) ok = pv(g - 1, j == 1);
+            }
+            if (ok && ntiles > 0) pv(jt + ntiles - 1, ntiles == 1);
+        } else if (warp >= kSoftmaxWarp0) {
+            // -------------------------------------------------------- softmax + output
+            // Thread (quarter sp, lane l): head 16*sp + l%16 of this CTA's 64,
+            // keys 32*(l/16) .. +31 of each tile; the two threads of a head
+            // combine their row max / sum with one shuffle.
+            const int sp = warp & 3;
+            const int hl = sp * 16 + (lane & 15), kh = lane >> 4;
+            const int h = head0 + hl;
+            const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+            float m_run = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const long long g = jt + j;
+                const int sb = (int)(g & 1);
+                const long long ebase = e0 + (long long)j * kTileKeys;
+                const uint64_t vmask = tile_mask(a, ks, bq, ebase, e1) >> (32 * kh);
+                if (!warp_wait(smem_u32(s.sfull + sb), (uint32_t)((g >> 1) & 1), p.ctx, s.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                float sc[32];
+                tmem_ld_half32(tmem_s + lane_base + sb * kTileKeys, sc);
+                tc::tmem_wait_ld();
+                tc::fence_before_sync();
+                mbar_arrive(smem_u32(s.sempty + sb));
+                float mt = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if (!((vmask >> i) & 1u)) sc[i] = -INFINITY;
+                    mt = fmaxf(mt, sc[i]);
+                }
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                // raise the running max only when it grows by more than 2^8: O (after the
+                // previous P.V) and l are then scaled by 2^(m_old - m_new)
+                const bool mine = m_run != -INFINITY && mt > m_run + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, mine)) {
+                    if (!warp_wait(smem_u32(s.oready), (uint32_t)((g - 1) & 1), p.ctx, s.abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const float f = mine ? exp2f(m_run - mt) : 1.0f;
+                    for (int c = 0; c < D; c += 64) {
+                        float v[32];
+                        tmem_ld_half32(tmem_o + lane_base + c, v);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= f;
+                        tmem_st_half32(tmem_o + lane_base + c, v);
+                    }
+                    tc::tmem_wait_st();
+                    if (mine) {
+                        l *= f;
+                        m_run = mt;
+                    }
+                }
+                if (m_run == -INFINITY) m_run = mt;
+                const float mref = m_run == -INFINITY ? 0.f : m_run;
+                float ps = 0.f;
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 = exp2f(sc[i] - mref), p1 = exp2f(sc[i + 1] - mref);
+                    ps += p0 + p1;
+                    pk[i / 2] = pack_bf16x2(p0, p1);
+                }
+                l += ps + __shfl_xor_sync(0xffffffffu, ps, 16);
+                const int pb = (int)(g & 1);
+                if (!warp_wait(smem_u32(s.pempty + pb), (uint32_t)(((g >> 1) & 1) ^ 1), p.ctx, s.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *prow = s.p + pb * Lt::kPBytes + hl * 128;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    *reinterpret_cast<uint4 *>(prow + (((4 * kh + u) ^ (hl & 7)) << 4)) =
+                        make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                tc::fence_proxy_async_smem();
+                tc::fence_before_sync();
+                mbar_arrive(smem_u32(s.pfull + pb));
+            }
+            // output: O / l (one split) or the unnormalised partial + (max, sum)
+            if (ok && ntiles > 0) {
+                ok = warp_wait(smem_u32(s.oready), (uint32_t)((jt + ntiles - 1) & 1), p.ctx, s.abort_flag);
+                tc::fence_after_sync();
+            }
+            if (ok) {
+                const float inv = l > 0.f ? 1.0f / l : 0.f;
+                const bool store = h < a.H;
+                for (int c = 0; c < D; c += 64) {
+                    float v[32];
+                    if (ntiles > 0) {
+                        tmem_ld_half32(tmem_o + lane_base + c, v);  // every lane (warp-collective)
+                        tc::tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    }
+                    if (!store) continue;
+                    const int col = c + 32 * kh;
+                    if (a.splits == 1) {
+                        uint16_t *dst = a.out + ((size_t)bq * a.H + h) * D + col;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            float o[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o[e] = v[i + e] * inv;
+                            *reinterpret_cast<uint4 *>(dst + i) = pack8(o);
+                        }
+                    } else {
+                        float *dst = a.part_o + (((size_t)split * a.n_bq + bq) * a.H + h) * D + col;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    }
+                }
+                if (store && a.splits > 1 && kh == 0)
+                    a.part_ml[((size_t)split * a.n_bq + bq) * a.H + h] =
+                        ntiles > 0 ? make_float2(m_run, l) : make_float2(-INFINITY, 0.f);
+            }
+        }
+        jt += ntiles;
+        tc::fence_before_sync();
+        __syncthreads();  // Q_hat, O and the buffers are reused by the next work item
+        tc::fence_after_sync();
+        if (*s.abort_flag) break;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// M = 64 instruction descriptor (kind::f16, bf16 operands, fp32 accumulate)
+constexpr uint32_t idesc_m64(int n, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn ? (1u << 16) : 0u) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(64 >> 4) << 24);
+}
+
+template <int D>
+int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
+    AttTcParams p = {};
+    p.a = a;
+    p.ctx = ctx;
+    p.HH = (a.H + kHeads - 1) / kHeads;
+    p.idesc_qk = idesc_m64(kTileKeys, false);
+    p.idesc_pv = idesc_m64(Layout<D>::kPvN, true);
+    p.n_work = a.n_bq * a.splits * p.HH;
+    int stages = kMaxStages;
+    while (stages > 2 && smem_bytes<D>(stages) > 225 * 1024) --stages;
+    p.stages = stages;
+    // at least 120 KiB so that one CTA owns an SM (it allocates all 512 TMEM columns)
+    const size_t smem = std::max<size_t>(smem_bytes<D>(stages), 120 * 1024);
+    auto kern = attend_tc_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const int grid = (int)std::min<long long>(p.n_work, num_sms());
+    kern<<<grid, kThreads, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+    return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
+}
+
+}  // namespace
+
+bool attend_tc_supported(int H, int D) { return H >= 1 && H <= 128 && (D == 64 || D == 128 || D == 256 || D == 512); }
+
+// Key splits per query: enough (query, split, head half) items to fill the
+// SMs, splits aligned to 64-key tiles, chosen to minimise the tiles of the
+// busiest CTA (plus a small per-item and per-split overhead).
+void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long long *kps) {
+    const long long HH = (H + kHeads - 1) / kHeads;
+    const long long ctas = num_sms();
+    const long long tiles = (max_keys + 3 + kTileKeys - 1) / kTileKeys + 1;
+    long long best_cost = -1;
+    int best = 1;
+    for (int sp = 1; sp <= 64; ++sp) {
+        const long long per = (tiles + sp - 1) / sp;
+        const long long items = n_bq * HH * sp;
+        const long long waves = (items + ctas - 1) / ctas;
+        const long long cost = waves * (per + 3) + (sp > 1 ? 1 : 0);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = sp;
+        }
+        if (per <= 1) break;
+    }
+    *splits = best;
+    *kps = ((tiles + best - 1) / best) * kTileKeys;
+}
+
+int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st) {
+    switch (a.D) {
+        case 64: return launch_d<64>(a, ctx, st);
+        case 128: return launch_d<128>(a, ctx, st);
+        case 256: return launch_d<256>(a, ctx, st);
+        case 512: return launch_d<512>(a, ctx, st);
+        default: return CSA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace csa

@@ -196,7 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int acc = (int)(it & 1);
             const uint32_t aph = (uint32_t)((it >> 1) & 1);
-            if (!mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag)) break;
+            // lane 0 polls, the warp follows (tcgen05.ld below is warp-collective)
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            __syncwarp();
+            if (!ok) break;
             tc::fence_after_sync();
             const long long s = (long long)wi.kt * kTileKeys + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.n_cols);

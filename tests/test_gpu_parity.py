@@ -191,6 +191,46 @@ def test_csa_attend_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts, gain):
     assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
 
 
+@pytest.mark.parametrize("batch,nq,H,D,N,T,k,Wn,m", [
+    (8, 1, 128, 512, 32768, 131072, 1024, 128, 4),     # CSA decode shape (split keys + combine)
+    (1, 200, 128, 512, 2048, 8192, 128, 16, 4),        # many queries per cluster (prefill-like loop)
+    (1, 150, 64, 256, 1000, 4000, 200, 32, 4),         # D = 256: one CTA per query, several per SM slot
+])
+def test_csa_attend_parity_large(cuda, batch, nq, H, D, N, T, k, Wn, m):
+    q = seeded((batch, nq, H, D), 45)
+    kv = seeded((batch, N, D), 46)
+    ts = [T - 1 - (i % 7) * 3 for i in range(batch * nq)]
+    qp = positions(batch, nq, ts)
+    p0 = T - 64 - Wn
+    win = seeded((batch, T - p0, D), 47)
+    idx = _random_selection(batch, nq, k, ts, m, N, 48)
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale, win_pos0=p0)
+    ref = oracle.attend(bits(q), bits(kv), idx, bits(win), qp.cpu().numpy(), Wn, scale, win_pos0=p0)
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
+def test_attend_running_max_rescale(cuda):
+    """Entries whose norms grow along the key order (logit scale 0.01 -> 5) push
+    the running max up by more than 2^8 after the first tiles (the O rescale
+    path).  Logits stay in the range where bf16 query operands keep the
+    softmax weights within tolerance."""
+    batch, H, D, N, m, Wn = 2, 128, 512, 640, 4, 8
+    T = N * m
+    q = seeded((batch, 1, H, D), 55)
+    base = seeded((batch, N, D), 56).float()
+    grow = torch.logspace(-2.0, float(np.log10(5.0)), N, device=DEV).view(1, N, 1)
+    kv = (base * grow).to(torch.bfloat16).contiguous()
+    win = seeded((batch, Wn, D), 57)
+    qp = positions(batch, 1, [T - 1, T - 1])
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.hca_attend(q, kv, m, win, qp, Wn, scale, win_pos0=T - Wn)
+    ref = oracle.hca_attend(bits(q), bits(kv), m, bits(win), qp.cpu().numpy(), Wn, scale, win_pos0=T - Wn)
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
 def test_csa_attend_window_cache_equals_full_stream(cuda):
     """A decode window cache (win_pos0 = t-W+1, W rows) gives the same output as the whole stream."""
     batch, H, D, N, T, k, Wn, m = 2, 128, 512, 256, 1024, 64, 128, 4
