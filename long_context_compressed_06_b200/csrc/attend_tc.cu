@@ -304,20 +304,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
 
         if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
             // -------------------------------------------------------- producers (cp.async gather)
+            // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l, l+32,
+            // .. of the row (coalesced 512 B per instruction).  Row pointers of the
+            // tile's 64 keys are computed once per tile, two per lane.
             const int pw = warp - kProducerWarp0;
             for (int j = 0; j < ntiles; ++j) {
                 const long long g = jt + j;
                 const int st = (int)(g % p.stages);
+                const long long ebase = e0 + (long long)j * kTileKeys;
+                const uint16_t *r0 = key_ptr(a, ks, b, bq, std::min(ebase + lane, e1 - 1));
+                const uint16_t *r1 = key_ptr(a, ks, b, bq, std::min(ebase + 32 + lane, e1 - 1));
                 if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag))
                     break;
-                uint8_t *stage = s.k + (size_t)st * Lt::kStageBytes;
-                const long long ebase = e0 + (long long)j * kTileKeys;
+                const uint32_t stage = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+#pragma unroll 2
                 for (int key = pw; key < kTileKeys; key += kProducerWarps) {
-                    const uint16_t *row = key_ptr(a, ks, b, bq, std::min(ebase + key, e1 - 1));
+                    const uint16_t *row = reinterpret_cast<const uint16_t *>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? r0 : r1), key & 31));
+                    const uint32_t krow = stage + key * 128;
 #pragma unroll
                     for (int u = lane; u < D / 8; u += 32) {  // 16-byte units of the row
-                        const uint32_t dst = smem_u32(stage + (size_t)(u >> 3) * kTileKeys * 128 + key * 128 +
-                                                      (((u & 7) ^ (key & 7)) << 4));
+                        const uint32_t dst = krow + (u >> 3) * (kTileKeys * 128) + (((u & 7) ^ (key & 7)) << 4);
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(row + u * 8)
                                      : "memory");
                     }
@@ -328,52 +335,73 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
             asm volatile("cp.async.wait_all;" ::: "memory");
         } else if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- MMA issuer
-            auto pv = [&](long long g, bool first) -> bool {
-                const int pb = (int)(g & 1);
-                if (!mbar_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1), p.ctx, s.abort_flag)) return false;
-                tc::fence_after_sync();
-                const int st = (int)(g % p.stages);
-                const uint32_t pa = smem_u32(s.p + pb * Lt::kPBytes);
-                const uint32_t vb = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+            // Event driven: P.V for tile i as soon as P_i is written, QK for the
+            // next tile as soon as its keys have landed and an S buffer is free.
+            // Descriptors are built once and advanced by constant offsets.
+            const uint64_t qdesc = tc::smem_desc(smem_u32(s.q), 1024, tc::kLayoutSw128);
+            const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
+            const uint64_t vdesc0 = tc::smem_desc_lbo(smem_u32(s.k), kTileKeys * 128, 1024, tc::kLayoutSw128);
+            const uint64_t pdesc0 = tc::smem_desc(smem_u32(s.p), 1024, tc::kLayoutSw128);
+            int nqk = 0, npv = 0;
+            uint64_t t_idle = 0;
+            while (npv < ntiles) {
+                bool progressed = false;
+                if (nqk < ntiles && nqk < npv + 2) {
+                    const long long g = jt + nqk;
+                    const int st = (int)(g % p.stages), sb = (int)(g & 1);
+                    if (mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1)) &&
+                        mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1))) {
+                        tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+                        tc::fence_after_sync();
+                        const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-                    const uint64_t ad = tc::smem_desc(pa + kk * 32, 1024, tc::kLayoutSw128);
+                        for (int c = 0; c < Lt::kChunks; ++c)
 #pragma unroll
-                    for (int n0 = 0; n0 < D; n0 += Lt::kPvN) {
-                        // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes apart (LBO),
-                        // 8-key groups 1024 bytes apart (SBO); a K step is 16 keys
-                        const uint64_t bd = tc::smem_desc_lbo(vb + (n0 / 64) * kTileKeys * 128 + kk * 16 * 128,
-                                                              kTileKeys * 128, 1024, tc::kLayoutSw128);
-                        tc::mma_f16(tmem_o + n0, ad, bd, p.idesc_pv, (first && kk == 0) ? 0u : 1u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                                            kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
+                                            (c | kk) ? 1u : 0u);
+                        tc::mma_commit(smem_u32(s.sfull + sb));
+                        ++nqk;
+                        progressed = true;
                     }
                 }
-                tc::mma_commit(smem_u32(s.kempty + st));
-                tc::mma_commit(smem_u32(s.pempty + pb));
-                tc::mma_commit(smem_u32(s.oready));
-                return true;
-            };
-            bool ok = true;
-            for (int j = 0; j < ntiles && ok; ++j) {
-                const long long g = jt + j;
-                const int st = (int)(g % p.stages);
-                const int sb = (int)(g & 1);
-                if (!mbar_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1), p.ctx, s.abort_flag)) break;
-                if (!mbar_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1), p.ctx, s.abort_flag)) break;
-                tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
-                tc::fence_after_sync();
-                const uint32_t qa = smem_u32(s.q), kb = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+                if (npv < nqk) {
+                    const long long g = jt + npv;
+                    const int pb = (int)(g & 1), st = (int)(g % p.stages);
+                    if (mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1))) {
+                        tc::fence_after_sync();
+                        const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
+                        const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
 #pragma unroll
-                for (int c = 0; c < Lt::kChunks; ++c)
+                        for (int kk = 0; kk < kTileKeys / 16; ++kk)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = tc::smem_desc(qa + c * kHeads * 128 + kk * 32, 1024, tc::kLayoutSw128);
-                        const uint64_t bd = tc::smem_desc(kb + c * kTileKeys * 128 + kk * 32, 1024, tc::kLayoutSw128);
-                        tc::mma_f16(tmem_s + sb * kTileKeys, ad, bd, p.idesc_qk, (c | kk) ? 1u : 0u);
+                            for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
+                                // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
+                                // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
+                                tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
+                                            vd + (((n0 / 64) * kTileKeys * 128 + kk * 16 * 128) >> 4), p.idesc_pv,
+                                            (npv == 0 && kk == 0) ? 0u : 1u);
+                        tc::mma_commit(smem_u32(s.kempty + st));
+                        tc::mma_commit(smem_u32(s.pempty + pb));
+                        tc::mma_commit(smem_u32(s.oready));
+                        ++npv;
+                        progressed = true;
                     }
-                tc::mma_commit(smem_u32(s.sfull + sb));
-                if (j > 0) ok = pv(g - 1, j == 1);
+                }
+                if (progressed) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = global_timer_ns();
+                    if (t_idle == 0) {
+                        t_idle = now;
+                    } else if (now - t_idle > p.ctx.budget_ns || *s.abort_flag) {
+                        record_status(p.ctx.status, CSA_ERR_TIMEOUT);
+                        *s.abort_flag = 1;
+                        break;
+                    }
+                }
             }
-            if (ok && ntiles > 0) pv(jt + ntiles - 1, ntiles == 1);
         } else if (warp >= kSoftmaxWarp0) {
             // -------------------------------------------------------- softmax + output
             // Thread (quarter sp, lane l): head 16*sp + l%16 of this CTA's 64,

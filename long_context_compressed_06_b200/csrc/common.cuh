@@ -103,6 +103,19 @@ CSA_DEVINL bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of a phase (for loops that poll several barriers).
+CSA_DEVINL bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of the mbarrier at shared address `bar`.  Gives up
 // after ctx.budget_ns of global time, or at once if *abort (a CTA-wide flag in
 // shared memory) is set; on giving up it records CSA_ERR_TIMEOUT, sets *abort
