@@ -209,13 +209,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int q = g * p.NQ + qi;
                 if (q >= p.nq) break;
                 float score = 0.f;
-                for (int hc = 0; hc < p.H_pad; hc += 16) {
-                    float v[16];
-                    tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc), v);
+                for (int hc = 0; hc < p.H_pad; hc += 64) {
+                    // up to four 16-column loads in flight per wait
+                    float v[64];
+                    const int nl = min(4, (p.H_pad - hc) >> 4);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
                     tc::tmem_wait_ld();
                     const float *ws = w_s + qi * p.H_pad + hc;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) score = fmaf(ws[i], fmaxf(v[i], 0.f), score);
+                    for (int u = 0; u < 4; ++u)
+                        if (u < nl) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                score = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), score);
+                        }
                 }
                 if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nvis_s[qi] ? score : -INFINITY;
             }

@@ -8,11 +8,12 @@
 // Design: a radix select over the scores mapped to order-preserving uint32
 // keys.  One query is handled by a thread-block cluster of CS CTAs x 1024
 // threads; each thread keeps R consecutive keys in registers (CS*1024*R >= N),
-// so the scores are read from memory exactly once.  Three digit passes
-// (11, 11, 10 bits) build a histogram of the candidates that still share the
-// threshold's prefix; warps aggregate equal digits with __match_any_sync and
-// add into rank 0's shared-memory histogram through distributed shared memory.
-// A pass stops early once the threshold bin holds exactly the number of
+// so the scores are read from memory exactly once.  The digits start at the
+// highest bit where the cluster-wide smallest and largest key differ (the bits
+// above are shared by every candidate), 11 bits per pass; each CTA counts its
+// candidates into its own shared-memory histogram and, after one cluster
+// barrier, reads its peers' histograms through distributed shared memory.
+// The selection stops once the threshold bin holds exactly the number of
 // elements still needed.  Selection is a stable compaction: per-thread
 // counts, a block scan, and a cluster scan over CTA totals via DSMEM.
 #include <cooperative_groups.h>
@@ -71,20 +72,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const long long bq = blockIdx.x / CS;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    __shared__ uint32_t hist[3][kBins];          // used in rank 0 only
+    __shared__ __align__(8) uint32_t hist[2][kBins];  // this CTA's histogram, double-buffered over passes
     __shared__ uint32_t warp_u32[32];
     __shared__ unsigned long long warp_u64[32];
-    __shared__ unsigned long long cta_total;      // (gt << 32) | eq, read by higher ranks
-    __shared__ uint32_t s_bin, s_cnt;
+    __shared__ unsigned long long cta_total;           // (gt << 32) | eq, read by higher ranks
+    __shared__ uint32_t cta_min, cta_max;               // this CTA's key range, read by peers
+    __shared__ uint32_t s_min, s_max, s_bin, s_cnt;
     __shared__ long long s_krem;
 
-    for (int i = threadIdx.x; i < 3 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
-    if (threadIdx.x == 0) {
-        s_bin = 0u;
-        s_cnt = 0u;
-        s_krem = 0;
-    }
+    for (int i = threadIdx.x; i < 2 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
 
     const long long nv = n_visible(q_pos[bq], m, N);
     const long long kk = nv < k ? nv : k;
@@ -104,28 +102,81 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
 #pragma unroll
         for (int r = 0; r < R; ++r) key[r] = r < nloc ? order_key(__ldg(row + seg0 + r)) : 0u;
     }
-    cluster.sync();  // every histogram cleared before any remote add
+    // key range of the visible entries (cluster-wide)
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        if (r < nloc) {
+            kmin = min(kmin, key[r]);
+            kmax = max(kmax, key[r]);
+        }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+        warp_u32[warp] = kmin;
+        reinterpret_cast<uint32_t *>(warp_u64)[warp] = kmax;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t a = __reduce_min_sync(0xffffffffu, warp_u32[lane]);
+        const uint32_t b = __reduce_max_sync(0xffffffffu, reinterpret_cast<uint32_t *>(warp_u64)[lane]);
+        if (lane == 0) {
+            cta_min = a;
+            cta_max = b;
+        }
+    }
+    cluster.sync();  // key ranges published, histograms cleared
+    if (warp == 0) {
+        const uint32_t a = lane < CS ? *cluster.map_shared_rank(&cta_min, lane) : 0xffffffffu;
+        const uint32_t b = lane < CS ? *cluster.map_shared_rank(&cta_max, lane) : 0u;
+        const uint32_t ga = __reduce_min_sync(0xffffffffu, a), gb = __reduce_max_sync(0xffffffffu, b);
+        if (lane == 0) {
+            s_min = ga;
+            s_max = gb;
+            s_bin = 0u;
+            s_cnt = 0u;
+            s_krem = 0;
+        }
+    }
+    __syncthreads();
 
+    // Radix select from the highest bit where the smallest and largest key
+    // differ (bits above it are shared by every candidate), 11 bits per pass.
     uint32_t prefix = 0u, mask = 0u;
     long long krem = kk;
     bool done = nv <= k;  // every visible entry is selected
-    uint32_t *h0 = cluster.map_shared_rank(&hist[0][0], 0);
-    const int lane = threadIdx.x & 31;
-#pragma unroll 1
-    for (int p = 0; p < 3 && !done; ++p) {
-        const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);
-        const uint32_t dmask = p == 2 ? 0x3ffu : 0x7ffu;
-        uint32_t *hp = h0 + p * kBins;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const bool cand = r < nloc && (key[r] & mask) == prefix;
-            const uint32_t bin = cand ? (key[r] >> sh) & dmask : 0xffffffffu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (cand && lane == __ffs(peers) - 1) atomicAdd(hp + bin, (uint32_t)__popc(peers));
+    int top = -1;
+    if (!done) {
+        if (s_min == s_max) {
+            prefix = s_max;
+            mask = 0xffffffffu;  // all keys equal: the lowest indices win
+            done = true;
+        } else {
+            top = 31 - __clz(s_min ^ s_max);
+            mask = top == 31 ? 0u : ~((2u << top) - 1u);
+            prefix = s_max & mask;
         }
-        cluster.sync();  // histogram of this pass complete
+    }
+#pragma unroll 1
+    for (int p = 0; !done && top >= 0; ++p) {
+        const int width = top + 1 < 11 ? top + 1 : 11;
+        const int sh = top - width + 1;
+        const uint32_t dmask = (1u << width) - 1u;
+        uint32_t *hloc = hist[p & 1];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if (r < nloc && (key[r] & mask) == prefix) atomicAdd(hloc + ((key[r] >> sh) & dmask), 1u);
+        cluster.sync();  // every CTA's histogram of this pass is complete
+        // cluster-wide counts of this thread's two bins: read every rank's histogram
+        uint32_t c_lo = 0u, c_hi = 0u;
+        for (int r2 = 0; r2 < CS; ++r2) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(cluster.map_shared_rank(hloc, r2) + 2 * threadIdx.x);
+            c_lo += v.x;
+            c_hi += v.y;
+        }
+        hist[(p + 1) & 1][2 * threadIdx.x] = 0u;      // peers finished reading it in the previous pass
+        hist[(p + 1) & 1][2 * threadIdx.x + 1] = 0u;
         // threshold bin: the highest bin b with (count above b) < krem <= (count above b) + hist[b]
-        const uint32_t c_lo = hp[2 * threadIdx.x], c_hi = hp[2 * threadIdx.x + 1];
         uint32_t tot;
         const uint32_t incl = block_scan_incl<uint32_t>(c_lo + c_hi, warp_u32, &tot);
         const long long above = (long long)tot - incl;  // count in bins of higher threads
@@ -139,6 +190,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         mask |= dmask << sh;
         krem = s_krem;
         done = (long long)s_cnt == krem;
+        top = sh - 1;
         __syncthreads();
     }
 
@@ -178,7 +230,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     }
     if (rank == 0)
         for (long long i = kk + threadIdx.x; i < k; i += kTopkThreads) out[i] = -1;
-    cluster.sync();  // peers may still read hist / cta_total of this CTA
+    cluster.sync();  // peers may still read this CTA's histogram / cta_total
 }
 
 struct TopkPlan {
