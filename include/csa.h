@@ -187,6 +187,36 @@ int hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long 
                uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * csa_attend_noalloc -- csa_attend for callers that cannot allocate device
+ * memory.  No passage of the pages corresponds to it: it is a deployment
+ * convenience of this library.
+ *
+ * Who needs it: a plugin or embedded runtime handed only a stream and tensor
+ * pointers; a serving loop that must not call cudaMalloc on its hot path (it
+ * synchronises the whole device); code being recorded into a CUDA graph,
+ * where allocation is not allowed.  csa_attend needs caller scratch for its
+ * split-KV partial results; here that scratch is a file-scope device array of
+ * CSA_ATTEND_NOALLOC_MAX_BYTES per device, held by every GPU that loads the
+ * library until the process exits.
+ *
+ * Arguments, layouts and results are those of csa_attend without the
+ * workspace.  Returns CSA_ERR_WORKSPACE when csa_attend_workspace_bytes(batch,
+ * nq, H, D, k + W) exceeds CSA_ATTEND_NOALLOC_MAX_BYTES (use csa_attend with
+ * a caller workspace then).  Nothing is allocated or freed.
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls share the array and it keeps the last call's contents
+ * (nothing in it needs clearing: every slot read is written by the same
+ * call); calls that overlap on the GPU -- different streams or host threads --
+ * race on it, so serialise them.
+ */
+#define CSA_ATTEND_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+                       const int *idx, int k, const uint16_t *win_src, long long win_pos0,
+                       long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
+                       float scale, float eps, uint16_t *out, void *stream);
+
+/*
  * csa_sync_status -- synchronise `stream`, then read and clear the device
  * status word.  Returns CSA_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call, CSA_ERR_CUDA on a CUDA error, else CSA_OK.

@@ -49,6 +49,8 @@ def load() -> ctypes.CDLL:
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
         "csa_attend": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
         "hca_attend": ([P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_attend_noalloc": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
+                               i32),
         "csa_sync_status": ([P], i32),
         "csa_set_wait_budget_ns": ([ctypes.c_ulonglong], None),
         "csa_selftest_wait_timeout": ([P], i32),
@@ -213,6 +215,26 @@ def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
     _check(L.hca_attend(_p(q), _p(q_gain), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos), batch, nq, H,
                         D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend")
+    return out
+
+
+def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
+                       win_pos0: int = 0):
+    """csa_attend without a caller workspace: the library's own fixed device
+    scratch is used (for callers that cannot allocate; see include/csa.h)."""
+    L = load()
+    _need(q, torch.bfloat16, "q", 4)
+    _need(kv, torch.bfloat16, "kv", 3)
+    _need(idx, torch.int32, "idx", 3)
+    _need(win, torch.bfloat16, "win", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H, D = q.shape
+    N, rows, k = kv.shape[1], win.shape[1], idx.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
+                                _p(q_pos), batch, nq, H, D, float(scale), float(eps), _p(out), _stream()),
+           "csa_attend_noalloc")
     return out
 
 

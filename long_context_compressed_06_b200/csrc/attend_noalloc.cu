@@ -1,0 +1,54 @@
+// attend_noalloc.cu -- csa_attend for callers that cannot allocate device memory.
+//
+// Some callers of this library have no way to allocate: a plugin or embedded
+// runtime that is handed only a stream and pointers to its tensors, a serving
+// loop that forbids cudaMalloc on its hot path (it synchronises the device),
+// or code recording work into a CUDA graph, where allocation is not permitted.
+// csa_attend needs caller scratch for its split-KV partial results; this entry
+// point supplies it from a file-scope device array instead, so the caller
+// passes only inputs and outputs.
+//
+// The array is a fixed CSA_ATTEND_NOALLOC_MAX_BYTES per device; every GPU that
+// loads the library holds it until the process exits.  All calls share it and
+// it keeps the last call's contents; nothing needs clearing (every slot the
+// combine step reads is written earlier in the same call), but calls that
+// overlap on the GPU -- on different streams, or from several host threads --
+// race on it.
+#include <cuda_runtime.h>
+
+#include "../../include/csa.h"
+
+namespace {
+
+__device__ __align__(256) unsigned char g_attend_scratch[CSA_ATTEND_NOALLOC_MAX_BYTES];
+
+// Device address of the array on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress; it is looked up once per device, with that device
+// current, on the first call made on it.
+void *scratch_on_current_device() {
+    static void *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_attend_scratch) != cudaSuccess) return nullptr;
+        cache[dev] = p;
+    }
+    return cache[dev];
+}
+
+}  // namespace
+
+extern "C" int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+                                  const int *idx, int k, const uint16_t *win_src, long long win_pos0,
+                                  long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
+                                  float scale, float eps, uint16_t *out, void *stream) {
+    if (batch < 1 || nq < 1 || H < 1 || D < 1 || k < 0 || W < 1) return CSA_ERR_INVALID;
+    const size_t need = csa_attend_workspace_bytes(batch, nq, H, D, (long long)k + W);
+    if (need > (size_t)CSA_ATTEND_NOALLOC_MAX_BYTES) return CSA_ERR_WORKSPACE;
+    void *scratch = scratch_on_current_device();
+    if (!scratch) return CSA_ERR_CUDA;
+    return csa_attend(q, q_gain, kv, N, idx, k, win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, scale, eps,
+                      out, scratch, (size_t)CSA_ATTEND_NOALLOC_MAX_BYTES, stream);
+}
