@@ -44,6 +44,7 @@ from long_context_compressed_06_b200 import workloads as W  # noqa: E402
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 PROFILES = os.path.join(ROOT, "profiles")
+METRIC = "CSA decode queries/s @128K ctx + HBM GB/s vs peak; prefill TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -73,6 +74,11 @@ def max_over_ranks(x: float, world: int, device) -> float:
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_rank_step: int, steps: int, world: int, t_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / t_max
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
@@ -275,8 +281,7 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
     torch.cuda.synchronize()
     barrier(world)
     t_max = max_over_ranks(t_graph, world, device)
-    n_units = wl.batch * wl.nq * args.steps * world
-    value = n_units / t_max
+    value = job_rate(wl.batch * wl.nq, args.steps, world, t_max)
     # per-kernel breakdown (eager launches, events between kernels)
     _, seg = timer.run(lambda mark: csa_decode_step(csa, st, mark), args.steps, args.warmup, marks=2)
     t_index = seg[0]
@@ -317,7 +322,7 @@ def e2e_csa_decode(csa, st, args, device, world):
 
     t, _ = timer.run(step, args.steps, args.warmup)
     t_max = max_over_ranks(t, world, device)
-    return {"value": wl.batch * wl.nq * args.steps * world / t_max, "unit": "queries/s",
+    return {"value": job_rate(wl.batch * wl.nq, args.steps, world, t_max), "unit": "queries/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
@@ -498,17 +503,24 @@ def run_reference(args):
         dt, threads = oracle_decode_sample(wl)
         total += dt
     value = steps / total
-    line = {"impl": "reference", "metric": "CSA decode queries/s @128K ctx", "value": value, "unit": "queries/s",
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
             "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup, "ms_per_step": total / steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "context": wl.T, "m": wl.m, "top_k": wl.k,
-                       "heads": wl.H, "head_dim": wl.D, "indexer": [wl.H_I, wl.d_I], "window": wl.W},
+            "config": decode_config(wl, args.gpus),
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads, "kind": "oracle",
                              "sample": "one decode query of the 128K workload per step (index over 32768 entries, "
                                        "full-sort top-1024, 128x512 attention over 1152 keys)"},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
+
+
+def decode_config(wl: W.Workload, world: int) -> dict:
+    """The headline workload as both arms name it."""
+    return {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.T, "m": wl.m, "entries": wl.N,
+            "top_k": wl.k, "heads": wl.H, "head_dim": wl.D, "indexer": [wl.H_I, wl.d_I], "window": wl.W,
+            "parallelism": "replicas x%d" % world, "l2": "flushed (256 MiB write) before every timed step",
+            "cuda_graph": True}
 
 
 # ----------------------------------------------------------------------------- main
@@ -560,14 +572,11 @@ def main():
     if rank == 0:
         wl = W.CSA_DECODE
         head["roofline"]["peak_source"] = peak_kind + " (burst, kernel timed alone)"
-        line = {"metric": "CSA decode queries/s @128K ctx + HBM GB/s vs peak; prefill TFLOP/s",
+        line = {"metric": METRIC,
                 "value": head["value"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.T, "m": wl.m,
-                           "entries": wl.N, "top_k": wl.k, "heads": wl.H, "head_dim": wl.D,
-                           "indexer": [wl.H_I, wl.d_I], "window": wl.W, "parallelism": "replicas x%d" % world,
-                           "l2": "flushed (256 MiB write) before every timed step", "cuda_graph": True},
+                "config": decode_config(wl, world),
                 "roofline": head["roofline"], "step": head["step"], "cpu_baseline": cpu, "e2e": head["e2e"],
                 "gpu_launches": head["launches"], "clocks": head["clocks"], "workloads": extra}
         print(json.dumps(line))
