@@ -66,7 +66,7 @@ struct Layout {
 
 struct Smem {
     uint8_t *q, *k, *p;
-    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready;
+    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready, *qready, *qempty;
     uint32_t *tmem_slot;
     int *abort_flag;
 };
@@ -87,7 +87,9 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
     s.pfull = s.sempty + 2;
     s.pempty = s.pfull + 2;
     s.oready = s.pempty + 2;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.oready + 1);
+    s.qready = s.oready + 2;
+    s.qempty = s.qready + 1;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.qempty + 1);
     s.abort_flag = reinterpret_cast<int *>(s.tmem_slot + 1);
     return s;
 }
@@ -95,7 +97,7 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
 template <int D>
 size_t smem_bytes(int stages) {
     using Lt = Layout<D>;
-    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (2 * kMaxStages + 9) * 8 + 16;
+    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (2 * kMaxStages + 12) * 8 + 16;
 }
 
 // ---------------------------------------------------------------- TMEM, 16-lane access shape
@@ -200,54 +202,91 @@ CSA_DEVINL bool warp_wait(uint32_t bar, uint32_t parity, const DevCtx &ctx, vola
 }
 
 // ---------------------------------------------------------------- Q_hat
-// Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16, for this CTA's 64 heads,
-// into the swizzled K-major tile [D/64][64 heads][128 B].  Each warp loads all
-// of its 8 heads before reducing (8 rows in flight).
+// Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16, into the swizzled
+// K-major tile [D/64][64 heads][128 B].  Built by the four softmax warps, 16
+// heads each, while the producers already gather the first key tiles.  A lane
+// owns whole 16-byte units (8 dims) of a row, so the loads are coalesced and
+// every shared-memory store is a conflict-free 16-byte store.
 template <int D>
-CSA_DEVINL void build_q(const AttendArgs &a, const Smem &s, long long bq, int head0) {
-    constexpr int DPL = D / 32;   // dims per lane
-    constexpr int HPW = kHeads / (kThreads / 32);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float x[HPW][DPL];
+CSA_DEVINL void build_q(const AttendArgs &a, const Smem &s, long long bq, int head0, int sw) {
+    constexpr int UR = D / 8;                   // 16-byte units per row
+    constexpr int LPR = UR < 32 ? UR : 32;      // lanes per row
+    constexpr int RPI = 32 / LPR;               // rows per warp instruction
+    constexpr int UPL = UR / LPR;               // units per lane
+    constexpr int HPW = kHeads / 4;             // heads per softmax warp
+    constexpr int PASSES = HPW / RPI;
+    constexpr int BATCH = PASSES * UPL <= 16 ? PASSES : 16 / UPL;  // rows in flight per lane
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPR, ul = lane % LPR;
+    float g[UPL][8];
 #pragma unroll
-    for (int i = 0; i < HPW; ++i) {
-        const int h = head0 + warp * HPW + i;
-        if (h < a.H) {
-            const uint16_t *row = a.q + ((size_t)bq * a.H + h) * D + lane * DPL;
-            if constexpr (DPL >= 8) {
+    for (int u = 0; u < UPL; ++u) {
+        const int d0 = (ul + u * LPR) * 8;
 #pragma unroll
-                for (int c = 0; c < DPL; c += 8) unpack8(ldg16(row + c), x[i] + c);
-            } else {
+        for (int e = 0; e < 8; ++e) g[u][e] = a.q_gain ? __ldg(a.q_gain + d0 + e) : 1.f;
+    }
 #pragma unroll
-                for (int c = 0; c < DPL; c += 2) {
-                    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(row + c));
-                    x[i][c] = bf16_lo(v);
-                    x[i][c + 1] = bf16_hi(v);
-                }
+    for (int p0 = 0; p0 < PASSES; p0 += BATCH) {
+        uint4 raw[BATCH][UPL];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int h = head0 + sw * HPW + (p0 + i) * RPI + sub;
+#pragma unroll
+            for (int u = 0; u < UPL; ++u)
+                raw[i][u] = h < a.H ? ldg16(a.q + ((size_t)bq * a.H + h) * D + (ul + u * LPR) * 8)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int hl = sw * HPW + (p0 + i) * RPI + sub;
+            float x[UPL][8];
+            float ss = 0.f;
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) {
+                unpack8(raw[i][u], x[u]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(x[u][e], x[u][e], ss);
             }
-        } else {
 #pragma unroll
-            for (int c = 0; c < DPL; ++c) x[i][c] = 0.f;
+            for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) {
+                const int unit = ul + u * LPR;
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = x[u][e] * r * g[u][e];
+                uint8_t *dst = s.q + (size_t)(unit >> 3) * kHeads * 128 + hl * 128 + (((unit & 7) ^ (hl & 7)) << 4);
+                *reinterpret_cast<uint4 *>(dst) = pack8(y);
+            }
         }
     }
-#pragma unroll
-    for (int i = 0; i < HPW; ++i) {
-        const int hl = warp * HPW + i;
-        float ss = 0.f;
-#pragma unroll
-        for (int c = 0; c < DPL; ++c) ss = fmaf(x[i][c], x[i][c], ss);
-        ss = warp_sum(ss);
-        const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
-#pragma unroll
-        for (int c = 0; c < DPL; c += 2) {
-            const int d = lane * DPL + c;
-            const float g0 = a.q_gain ? __ldg(a.q_gain + d) : 1.f;
-            const float g1 = a.q_gain ? __ldg(a.q_gain + d + 1) : 1.f;
-            uint8_t *dst = s.q + (size_t)(d >> 6) * kHeads * 128 + hl * 128 + ((((d & 63) >> 3) ^ (hl & 7)) << 4) +
-                           (d & 7) * 2;
-            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(x[i][c] * r * g0, x[i][c + 1] * r * g1);
-        }
-    }
+}
+
+// One work item: (query, key split, head half).  The query's tiles of 64 keys
+// are dealt to the splits in balanced contiguous ranges.
+struct Item {
+    long long bq, b, e0, e1;
+    Keys ks;
+    int split, head0, ntiles;
+};
+
+CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
+    const AttendArgs &a = p.a;
+    Item it;
+    const int hh = (int)(wi % p.HH);
+    const long long rest = wi / p.HH;
+    it.split = (int)(rest % a.splits);
+    it.bq = rest / a.splits;
+    it.b = it.bq / a.nq;
+    it.head0 = hh * kHeads;
+    it.ks = query_keys(a, __ldg(a.q_pos + it.bq));
+    const long long T = (it.ks.total + kTileKeys - 1) / kTileKeys;
+    const long long t0 = T * it.split / a.splits, t1 = T * (it.split + 1) / a.splits;
+    it.e0 = t0 * kTileKeys;
+    it.e1 = std::min(it.ks.total, t1 * kTileKeys);
+    it.ntiles = (int)(t1 - t0);
+    return it;
 }
 
 template <int D>
@@ -270,6 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
             mbar_init(s.pempty + i, 1);
         }
         mbar_init(s.oready, 1);
+        mbar_init(s.oready + 1, 1);
+        mbar_init(s.qready, 128);
+        mbar_init(s.qempty, 1);
         *s.abort_flag = 0;
         fence_mbar_init();
     }
@@ -284,38 +326,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
     const uint32_t tmem_o = tmem;                  // lanes 0-15 of each sub-partition, columns 0..D-1
     const uint32_t tmem_s = tmem + (16u << 16);    // lanes 16-31, columns 0..127 (two S buffers)
 
-    long long jt = 0;  // tiles processed by this CTA (ring and phase position, identical in every role)
-    for (long long wi = blockIdx.x; wi < p.n_work; wi += gridDim.x) {
-        const int hh = (int)(wi % p.HH);
-        const long long rest = wi / p.HH;
-        const int split = (int)(rest % a.splits);
-        const long long bq = rest / a.splits;
-        const long long b = bq / a.nq;
-        const int head0 = hh * kHeads;
-        const long long t = __ldg(a.q_pos + bq);
-        const Keys ks = query_keys(a, t);
-        const long long e0 = (long long)split * a.keys_per_split;
-        const long long e1 = std::min(ks.total, e0 + a.keys_per_split);
-        const int ntiles = e1 > e0 ? (int)((e1 - e0 + kTileKeys - 1) / kTileKeys) : 0;
-
-        build_q<D>(a, s, bq, head0);
-        tc::fence_proxy_async_smem();
-        __syncthreads();
-
-        if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
-            // -------------------------------------------------------- producers (cp.async gather)
-            // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l, l+32,
-            // .. of the row (coalesced 512 B per instruction).  Row pointers of the
-            // tile's 64 keys are computed once per tile, two per lane.
-            const int pw = warp - kProducerWarp0;
-            for (int j = 0; j < ntiles; ++j) {
+    // The roles run decoupled across work items; their only contacts are the
+    // mbarriers (key ring kfull/kempty, S buffers sfull/sempty, P buffers
+    // pfull/pempty, Q_hat qready/qempty, and oready[g & 1], committed after the
+    // P.V of tile g).  A parity wait is exact only if the barrier's previous
+    // phase is known complete; oready alternates between two barriers because
+    // the softmax may wait for P.V g while P.V g-1 is still running, whereas
+    // P.V g-2 is known complete (the P buffer it read was released before P_g
+    // was written).  jt counts the tiles this CTA has processed, identically in
+    // every role.
+    if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
+        // ------------------------------------------------------------ producers (cp.async gather)
+        // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l, l+32,
+        // .. of the row (coalesced 512 B per instruction).  Row pointers of the
+        // tile's 64 keys are computed once per tile, two per lane.
+        const int pw = warp - kProducerWarp0;
+        long long jt = 0;
+        bool ok = true;
+        for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x) {
+            const Item it = work_item(p, wi);
+            for (int j = 0; j < it.ntiles; ++j) {
                 const long long g = jt + j;
                 const int st = (int)(g % p.stages);
-                const long long ebase = e0 + (long long)j * kTileKeys;
-                const uint16_t *r0 = key_ptr(a, ks, b, bq, std::min(ebase + lane, e1 - 1));
-                const uint16_t *r1 = key_ptr(a, ks, b, bq, std::min(ebase + 32 + lane, e1 - 1));
-                if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag))
+                const long long ebase = it.e0 + (long long)j * kTileKeys;
+                const uint16_t *r0 = key_ptr(a, it.ks, it.b, it.bq, std::min(ebase + lane, it.e1 - 1));
+                const uint16_t *r1 = key_ptr(a, it.ks, it.b, it.bq, std::min(ebase + 32 + lane, it.e1 - 1));
+                if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag)) {
+                    ok = false;
                     break;
+                }
                 const uint32_t stage = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
 #pragma unroll 2
                 for (int key = pw; key < kTileKeys; key += kProducerWarps) {
@@ -332,8 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
                              : "memory");
             }
-            asm volatile("cp.async.wait_all;" ::: "memory");
-        } else if (warp == 0 && lane == 0) {
+            jt += it.ntiles;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 0) {
+        if (lane == 0) {
             // -------------------------------------------------------- MMA issuer
             // Event driven: P.V for tile i as soon as P_i is written, QK for the
             // next tile as soon as its keys have landed and an S buffer is free.
@@ -342,82 +384,106 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
             const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
             const uint64_t vdesc0 = tc::smem_desc_lbo(smem_u32(s.k), kTileKeys * 128, 1024, tc::kLayoutSw128);
             const uint64_t pdesc0 = tc::smem_desc(smem_u32(s.p), 1024, tc::kLayoutSw128);
-            int nqk = 0, npv = 0;
-            uint64_t t_idle = 0;
-            while (npv < ntiles) {
-                bool progressed = false;
-                if (nqk < ntiles && nqk < npv + 2) {
-                    const long long g = jt + nqk;
-                    const int st = (int)(g % p.stages), sb = (int)(g & 1);
-                    if (mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1)) &&
-                        mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1))) {
-                        tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
-                        tc::fence_after_sync();
-                        const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
-#pragma unroll
-                        for (int c = 0; c < Lt::kChunks; ++c)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
-                                            kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
-                                            (c | kk) ? 1u : 0u);
-                        tc::mma_commit(smem_u32(s.sfull + sb));
-                        ++nqk;
-                        progressed = true;
-                    }
-                }
-                if (npv < nqk) {
-                    const long long g = jt + npv;
-                    const int pb = (int)(g & 1), st = (int)(g % p.stages);
-                    if (mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1))) {
-                        tc::fence_after_sync();
-                        const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
-                        const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < kTileKeys / 16; ++kk)
-#pragma unroll
-                            for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
-                                // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
-                                // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
-                                tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
-                                            vd + (((n0 / 64) * kTileKeys * 128 + kk * 16 * 128) >> 4), p.idesc_pv,
-                                            (npv == 0 && kk == 0) ? 0u : 1u);
-                        tc::mma_commit(smem_u32(s.kempty + st));
-                        tc::mma_commit(smem_u32(s.pempty + pb));
-                        tc::mma_commit(smem_u32(s.oready));
-                        ++npv;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    t_idle = 0;
-                } else {
-                    const uint64_t now = global_timer_ns();
-                    if (t_idle == 0) {
-                        t_idle = now;
-                    } else if (now - t_idle > p.ctx.budget_ns || *s.abort_flag) {
-                        record_status(p.ctx.status, CSA_ERR_TIMEOUT);
-                        *s.abort_flag = 1;
-                        break;
-                    }
-                }
-            }
-        } else if (warp >= kSoftmaxWarp0) {
-            // -------------------------------------------------------- softmax + output
-            // Thread (quarter sp, lane l): head 16*sp + l%16 of this CTA's 64,
-            // keys 32*(l/16) .. +31 of each tile; the two threads of a head
-            // combine their row max / sum with one shuffle.
-            const int sp = warp & 3;
-            const int hl = sp * 16 + (lane & 15), kh = lane >> 4;
-            const int h = head0 + hl;
-            const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-            float m_run = -INFINITY, l = 0.f;
+            long long jt = 0;
+            uint32_t n_items = 0;
             bool ok = true;
-            for (int j = 0; j < ntiles && ok; ++j) {
+            for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
+                const Item it = work_item(p, wi);
+                if (!mbar_wait(smem_u32(s.qready), n_items & 1u, p.ctx, s.abort_flag)) break;
+                tc::fence_after_sync();
+                if (it.ntiles == 0) mbar_arrive(smem_u32(s.qempty));
+                int nqk = 0, npv = 0;
+                uint64_t t_idle = 0;
+                while (npv < it.ntiles) {
+                    bool progressed = false;
+                    if (nqk < it.ntiles && nqk < npv + 2) {
+                        const long long g = jt + nqk;
+                        const int st = (int)(g % p.stages), sb = (int)(g & 1);
+                        if (mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1)) &&
+                            mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1))) {
+                            tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+                            tc::fence_after_sync();
+                            const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
+#pragma unroll
+                            for (int c = 0; c < Lt::kChunks; ++c)
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                                                kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
+                                                (c | kk) ? 1u : 0u);
+                            tc::mma_commit(smem_u32(s.sfull + sb));
+                            ++nqk;
+                            if (nqk == it.ntiles) tc::mma_commit(smem_u32(s.qempty));  // Q_hat no longer read
+                            progressed = true;
+                        }
+                    }
+                    if (npv < nqk) {
+                        const long long g = jt + npv;
+                        const int pb = (int)(g & 1), st = (int)(g % p.stages);
+                        if (mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1))) {
+                            tc::fence_after_sync();
+                            const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
+                            const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
+#pragma unroll
+                            for (int kk = 0; kk < kTileKeys / 16; ++kk)
+#pragma unroll
+                                for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
+                                    // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
+                                    // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
+                                    tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
+                                                vd + (((n0 / 64) * kTileKeys * 128 + kk * 16 * 128) >> 4),
+                                                p.idesc_pv, (npv == 0 && kk == 0) ? 0u : 1u);
+                            tc::mma_commit(smem_u32(s.kempty + st));
+                            tc::mma_commit(smem_u32(s.pempty + pb));
+                            tc::mma_commit(smem_u32(s.oready + pb));
+                            ++npv;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        t_idle = 0;
+                    } else {
+                        const uint64_t now = global_timer_ns();
+                        if (t_idle == 0) {
+                            t_idle = now;
+                        } else if (now - t_idle > p.ctx.budget_ns || *s.abort_flag) {
+                            record_status(p.ctx.status, CSA_ERR_TIMEOUT);
+                            *s.abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+                jt += it.ntiles;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + output (warps 4..7)
+        // Thread (quarter sp, lane l): head 16*sp + l%16 of this CTA's 64,
+        // keys 32*(l/16) .. +31 of each tile; the two threads of a head
+        // combine their row max / sum with one shuffle.
+        const int sp = warp & 3;
+        const int hl = sp * 16 + (lane & 15), kh = lane >> 4;
+        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        long long jt = 0;
+        uint32_t n_items = 0;
+        bool ok = true;
+        for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
+            const Item it = work_item(p, wi);
+            const int h = it.head0 + hl;
+            // Q_hat of the previous item must have been consumed by its QK MMAs
+            if (n_items > 0 && !warp_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx, s.abort_flag)) break;
+            build_q<D>(a, s, it.bq, it.head0, sp);
+            tc::fence_proxy_async_smem();
+            mbar_arrive(smem_u32(s.qready));
+
+            float m_run = -INFINITY, l = 0.f;
+            for (int j = 0; j < it.ntiles && ok; ++j) {
                 const long long g = jt + j;
                 const int sb = (int)(g & 1);
-                const long long ebase = e0 + (long long)j * kTileKeys;
-                const uint64_t vmask = tile_mask(a, ks, bq, ebase, e1) >> (32 * kh);
+                const long long ebase = it.e0 + (long long)j * kTileKeys;
+                const uint64_t vmask = tile_mask(a, it.ks, it.bq, ebase, it.e1) >> (32 * kh);
                 if (!warp_wait(smem_u32(s.sfull + sb), (uint32_t)((g >> 1) & 1), p.ctx, s.abort_flag)) {
                     ok = false;
                     break;
@@ -439,7 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                 // previous P.V) and l are then scaled by 2^(m_old - m_new)
                 const bool mine = m_run != -INFINITY && mt > m_run + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, mine)) {
-                    if (!warp_wait(smem_u32(s.oready), (uint32_t)((g - 1) & 1), p.ctx, s.abort_flag)) {
+                    if (!warp_wait(smem_u32(s.oready + ((g - 1) & 1)), (uint32_t)(((g - 1) >> 1) & 1), p.ctx,
+                                   s.abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -484,51 +551,62 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                 tc::fence_before_sync();
                 mbar_arrive(smem_u32(s.pfull + pb));
             }
-            // output: O / l (one split) or the unnormalised partial + (max, sum)
-            if (ok && ntiles > 0) {
-                ok = warp_wait(smem_u32(s.oready), (uint32_t)((jt + ntiles - 1) & 1), p.ctx, s.abort_flag);
+            if (!ok) break;
+            // output: O / l (one split) or the unnormalised partial + (max, sum).
+            // After the last P.V both P buffers are free; they stage one 64-column
+            // slab of O (64 heads x 64 fp32, 16-byte units swizzled by head) so the
+            // global stores are whole row segments.
+            if (it.ntiles > 0) {
+                const long long gl = jt + it.ntiles - 1;
+                if (!warp_wait(smem_u32(s.oready + (gl & 1)), (uint32_t)((gl >> 1) & 1), p.ctx, s.abort_flag)) break;
                 tc::fence_after_sync();
             }
-            if (ok) {
-                const float inv = l > 0.f ? 1.0f / l : 0.f;
-                const bool store = h < a.H;
-                for (int c = 0; c < D; c += 64) {
-                    float v[32];
-                    if (ntiles > 0) {
-                        tmem_ld_half32(tmem_o + lane_base + c, v);  // every lane (warp-collective)
-                        tc::tmem_wait_ld();
-                    } else {
+            const float inv = a.splits == 1 ? (l > 0.f ? 1.0f / l : 0.f) : 1.0f;
+            uint8_t *stg = s.p;
+            for (int c = 0; c < D; c += 64) {
+                float v[32];
+                if (it.ntiles > 0) {
+                    tmem_ld_half32(tmem_o + lane_base + c, v);  // every lane (warp-collective)
+                    tc::tmem_wait_ld();
+                } else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4 *>(stg + hl * 256 + (((8 * kh + u) ^ (hl & 7)) << 4)) =
+                        make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
+                __syncwarp();  // a warp stages and stores only its own 16 heads
+                if (a.splits == 1) {
+                    // bf16 rows: 4 heads per instruction, 8 lanes x 8 columns each
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        const int r = sp * 16 + i + (lane >> 3), cu = lane & 7, hr = it.head0 + r;
+                        const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
+                        const float4 hi =
+                            *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
+                        const float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        if (hr < a.H)
+                            *reinterpret_cast<uint4 *>(a.out + ((size_t)it.bq * a.H + hr) * D + c + 8 * cu) = pack8(o);
                     }
-                    if (!store) continue;
-                    const int col = c + 32 * kh;
-                    if (a.splits == 1) {
-                        uint16_t *dst = a.out + ((size_t)bq * a.H + h) * D + col;
+                } else {
+                    // fp32 partial rows: 2 heads per instruction, 16 lanes x 4 columns each
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            float o[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) o[e] = v[i + e] * inv;
-                            *reinterpret_cast<uint4 *>(dst + i) = pack8(o);
-                        }
-                    } else {
-                        float *dst = a.part_o + (((size_t)split * a.n_bq + bq) * a.H + h) * D + col;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    for (int i = 0; i < 16; i += 2) {
+                        const int r = sp * 16 + i + (lane >> 4), cu = lane & 15, hr = it.head0 + r;
+                        const float4 v4 = *reinterpret_cast<const float4 *>(stg + r * 256 + ((cu ^ (r & 7)) << 4));
+                        if (hr < a.H)
+                            *reinterpret_cast<float4 *>(
+                                a.part_o + (((size_t)it.split * a.n_bq + it.bq) * a.H + hr) * D + c + 4 * cu) = v4;
                     }
                 }
-                if (store && a.splits > 1 && kh == 0)
-                    a.part_ml[((size_t)split * a.n_bq + bq) * a.H + h] =
-                        ntiles > 0 ? make_float2(m_run, l) : make_float2(-INFINITY, 0.f);
+                __syncwarp();  // a warp stages and stores only its own 16 heads
             }
+            if (h < a.H && a.splits > 1 && kh == 0)
+                a.part_ml[((size_t)it.split * a.n_bq + it.bq) * a.H + h] =
+                    it.ntiles > 0 ? make_float2(m_run, l) : make_float2(-INFINITY, 0.f);
+            jt += it.ntiles;
         }
-        jt += ntiles;
-        tc::fence_before_sync();
-        __syncthreads();  // Q_hat, O and the buffers are reused by the next work item
-        tc::fence_after_sync();
-        if (*s.abort_flag) break;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -572,12 +650,13 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
 bool attend_tc_supported(int H, int D) { return H >= 1 && H <= 128 && (D == 64 || D == 128 || D == 256 || D == 512); }
 
 // Key splits per query: enough (query, split, head half) items to fill the
-// SMs, splits aligned to 64-key tiles, chosen to minimise the tiles of the
-// busiest CTA (plus a small per-item and per-split overhead).
+// SMs, chosen to minimise the tiles of the busiest CTA (plus a small per-item
+// and per-split overhead).  The kernel deals each query's 64-key tiles to its
+// splits in balanced contiguous ranges, so the plan only needs the count.
 void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long long *kps) {
     const long long HH = (H + kHeads - 1) / kHeads;
     const long long ctas = num_sms();
-    const long long tiles = (max_keys + 3 + kTileKeys - 1) / kTileKeys + 1;
+    const long long tiles = (max_keys + kTileKeys - 1) / kTileKeys;
     long long best_cost = -1;
     int best = 1;
     for (int sp = 1; sp <= 64; ++sp) {

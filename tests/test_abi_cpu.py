@@ -107,10 +107,10 @@ def test_attend_validation_and_workspace(lib):
     assert call(T=0) == csa.CSA_ERR_INVALID
     assert call(D=96) == csa.CSA_ERR_UNSUPPORTED
     assert call(H=256) == csa.CSA_ERR_UNSUPPORTED
-    need = lib.csa_attend_workspace_bytes(1, 1, 8, 64, 64 + 16)
-    assert need > 0   # a single query is split over several CTAs
-    assert call(ws=A16, wsb=need - 1) == csa.CSA_ERR_WORKSPACE
-    assert call(ws=MIS, wsb=need) == csa.CSA_ERR_WORKSPACE
+    need = lib.csa_attend_workspace_bytes(1, 1, 8, 64, 1024 + 16)
+    assert need > 0   # a single query with 1040 keys is split over several CTAs
+    assert call(ws=A16, wsb=need - 1, k=1024) == csa.CSA_ERR_WORKSPACE
+    assert call(ws=MIS, wsb=need, k=1024) == csa.CSA_ERR_WORKSPACE
     h = lib.hca_attend
     assert h(A16, NULL, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b, NULL, 0,
              NULL) == csa.CSA_ERR_INVALID    # m
