@@ -20,7 +20,7 @@
 // no exchange; each streams the gathered rows itself (the second read of a
 // row is an L2 hit).
 //
-// Warp roles (256 threads): warp 0 TMEM owner + MMA issuer (one thread);
+// Warp roles (256 threads): warp 0 TMEM owner + MMA issuer (lane 0 issues);
 // warps 1..3 gather the key rows with 16-byte cp.async into the 128-byte
 // swizzled layout (one 512-byte coalesced row segment per warp instruction);
 // warps 4..7 softmax and output, two threads per head (keys 0-31 / 32-63,
@@ -66,7 +66,8 @@ struct Layout {
 
 struct Smem {
     uint8_t *q, *k, *p;
-    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready, *qready, *qempty;
+    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready, *qready, *qempty, *qfull;
+    uint64_t *kmask;  // [stage] validity of the 64 keys in the stage
     uint32_t *tmem_slot;
     int *abort_flag;
 };
@@ -89,7 +90,9 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
     s.oready = s.pempty + 2;
     s.qready = s.oready + 2;
     s.qempty = s.qready + 1;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.qempty + 1);
+    s.qfull = s.qempty + 1;
+    s.kmask = s.qfull + 1;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.kmask + kMaxStages);
     s.abort_flag = reinterpret_cast<int *>(s.tmem_slot + 1);
     return s;
 }
@@ -97,7 +100,7 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
 template <int D>
 size_t smem_bytes(int stages) {
     using Lt = Layout<D>;
-    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (2 * kMaxStages + 12) * 8 + 16;
+    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (3 * kMaxStages + 13) * 8 + 16;
 }
 
 // ---------------------------------------------------------------- TMEM, 16-lane access shape
@@ -157,108 +160,85 @@ CSA_DEVINL Keys query_keys(const AttendArgs &a, long long t) {
     return k;
 }
 
-// Row of key e (invalid keys read a valid row; their scores are masked).
-CSA_DEVINL const uint16_t *key_ptr(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e) {
+// Row of key e and whether it takes part (keys past e_end, selection padding
+// and out-of-range indices read a valid row; their scores are masked).
+CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
+                                    long long e_end, bool &valid) {
+    valid = e < e_end;
+    if (!valid) e = e_end - 1;  // e_end >= 1 whenever a tile exists
     if (e < ks.nsel4) {
         long long j = 0;
         if (e < ks.nsel) {
             j = a.dense ? e : (long long)__ldg(a.idx + bq * a.k + e);
-            if (j < 0 || j >= a.N) j = 0;
+            if (j < 0 || j >= a.N) {
+                j = 0;
+                valid = false;
+            }
+        } else {
+            valid = false;
         }
         return a.kv + ((size_t)b * a.N + j) * a.D;
     }
     long long w = e - ks.nsel4;
+    if (w >= ks.nwin) valid = false;
     w = w < ks.nwin ? w : ks.nwin - 1;
     w = w < 0 ? 0 : w;
     return a.win + ((size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + w) * a.D;
 }
 
-CSA_DEVINL bool key_valid(const AttendArgs &a, const Keys &ks, long long bq, long long e, long long e_end) {
-    if (e >= e_end) return false;
-    if (e < ks.nsel4) {
-        if (e >= ks.nsel) return false;
-        if (a.dense) return true;
-        const int j = __ldg(a.idx + bq * a.k + e);
-        return j >= 0 && j < a.N;
-    }
-    return e - ks.nsel4 < ks.nwin;
-}
-
-// Validity of the 64 keys of a tile as a bit mask (every lane of the warp gets it).
-CSA_DEVINL uint64_t tile_mask(const AttendArgs &a, const Keys &ks, long long bq, long long ebase, long long e_end) {
-    const int lane = threadIdx.x & 31;
-    const uint32_t lo = __ballot_sync(0xffffffffu, key_valid(a, ks, bq, ebase + lane, e_end));
-    const uint32_t hi = __ballot_sync(0xffffffffu, key_valid(a, ks, bq, ebase + 32 + lane, e_end));
-    return ((uint64_t)hi << 32) | lo;
-}
-
-// Warp-uniform bounded wait: lane 0 polls, the outcome is broadcast.
+// Warp-uniform bounded wait.  Every lane polls and the outcome is voted: a
+// wait polled by one lane while the others park at a shuffle leaves the warp
+// running its following code far slower (measured: 4x on the Q_hat pass).
 CSA_DEVINL bool warp_wait(uint32_t bar, uint32_t parity, const DevCtx &ctx, volatile int *abort) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ctx, abort);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();
-    return ok;
+    const bool ok = mbar_wait(bar, parity, ctx, abort);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------- Q_hat
-// Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16, into the swizzled
-// K-major tile [D/64][64 heads][128 B].  Built by the four softmax warps, 16
-// heads each, while the producers already gather the first key tiles.  A lane
-// owns whole 16-byte units (8 dims) of a row, so the loads are coalesced and
-// every shared-memory store is a conflict-free 16-byte store.
+// The raw query rows of a work item arrive by TMA, already in the swizzled
+// K-major tile [D/64][64 heads][128 B] (heads past H are zero-filled).  The
+// four softmax warps then normalise them in place, 16 heads each:
+//   Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16.
+// A lane owns whole 16-byte units (8 dims) of a row; every shared-memory
+// access is a conflict-free 16-byte access.
 template <int D>
-CSA_DEVINL void build_q(const AttendArgs &a, const Smem &s, long long bq, int head0, int sw) {
-    constexpr int UR = D / 8;                   // 16-byte units per row
-    constexpr int LPR = UR < 32 ? UR : 32;      // lanes per row
-    constexpr int RPI = 32 / LPR;               // rows per warp instruction
-    constexpr int UPL = UR / LPR;               // units per lane
-    constexpr int HPW = kHeads / 4;             // heads per softmax warp
-    constexpr int PASSES = HPW / RPI;
-    constexpr int BATCH = PASSES * UPL <= 16 ? PASSES : 16 / UPL;  // rows in flight per lane
+struct QLanes {
+    static constexpr int UR = D / 8;               // 16-byte units per row
+    static constexpr int LPR = UR < 32 ? UR : 32;  // lanes per row
+    static constexpr int RPI = 32 / LPR;           // rows per warp instruction
+    static constexpr int UPL = UR / LPR;           // units per lane
+    static constexpr int PASSES = (kHeads / 4) / RPI;
+};
+
+template <int D>
+CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8]) {
+    using QL = QLanes<D>;
     const int lane = threadIdx.x & 31;
-    const int sub = lane / LPR, ul = lane % LPR;
-    float g[UPL][8];
+    const int sub = lane / QL::LPR, ul = lane % QL::LPR;
+#pragma unroll 4
+    for (int pass = 0; pass < QL::PASSES; ++pass) {
+        const int hl = sw * (kHeads / 4) + pass * QL::RPI + sub;
+        uint4 *ptr[QL::UPL];
+        float x[QL::UPL][8];
+        float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < UPL; ++u) {
-        const int d0 = (ul + u * LPR) * 8;
+        for (int u = 0; u < QL::UPL; ++u) {
+            const int unit = ul + u * QL::LPR;
+            ptr[u] = reinterpret_cast<uint4 *>(s.q + (size_t)(unit >> 3) * kHeads * 128 + hl * 128 +
+                                               (((unit & 7) ^ (hl & 7)) << 4));
+            unpack8(*ptr[u], x[u]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) g[u][e] = a.q_gain ? __ldg(a.q_gain + d0 + e) : 1.f;
-    }
-#pragma unroll
-    for (int p0 = 0; p0 < PASSES; p0 += BATCH) {
-        uint4 raw[BATCH][UPL];
-#pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-            const int h = head0 + sw * HPW + (p0 + i) * RPI + sub;
-#pragma unroll
-            for (int u = 0; u < UPL; ++u)
-                raw[i][u] = h < a.H ? ldg16(a.q + ((size_t)bq * a.H + h) * D + (ul + u * LPR) * 8)
-                                    : make_uint4(0u, 0u, 0u, 0u);
+            for (int e = 0; e < 8; ++e) ss = fmaf(x[u][e], x[u][e], ss);
         }
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-            const int hl = sw * HPW + (p0 + i) * RPI + sub;
-            float x[UPL][8];
-            float ss = 0.f;
+        for (int o = QL::LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
 #pragma unroll
-            for (int u = 0; u < UPL; ++u) {
-                unpack8(raw[i][u], x[u]);
+        for (int u = 0; u < QL::UPL; ++u) {
+            float y[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(x[u][e], x[u][e], ss);
-            }
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
-#pragma unroll
-            for (int u = 0; u < UPL; ++u) {
-                const int unit = ul + u * LPR;
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = x[u][e] * r * g[u][e];
-                uint8_t *dst = s.q + (size_t)(unit >> 3) * kHeads * 128 + hl * 128 + (((unit & 7) ^ (hl & 7)) << 4);
-                *reinterpret_cast<uint4 *>(dst) = pack8(y);
-            }
+            for (int e = 0; e < 8; ++e) y[e] = x[u][e] * r * g[u][e];
+            *ptr[u] = pack8(y);
         }
     }
 }
@@ -290,7 +270,8 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const AttTcParams p) {
     using Lt = Layout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem s = carve<D>(smem_raw, p.stages);
@@ -299,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) {
-            mbar_init(s.kfull + i, kProducerWarps * 32);  // one cp.async completion arrive per producer thread
+            // one cp.async completion arrive per producer thread + the key-mask arrive
+            mbar_init(s.kfull + i, kProducerWarps * 32 + 1);
             mbar_init(s.kempty + i, 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -312,9 +294,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
         mbar_init(s.oready + 1, 1);
         mbar_init(s.qready, 128);
         mbar_init(s.qempty, 1);
+        mbar_init(s.qfull, 1);
         *s.abort_flag = 0;
         fence_mbar_init();
+        tc::prefetch_tmap(&qmap);
     }
+    // per-dimension query gains of this lane's units (softmax warps), read once
+    float qg[QLanes<D>::UPL][8];
+#pragma unroll
+    for (int u = 0; u < QLanes<D>::UPL; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            qg[u][e] = (warp >= kSoftmaxWarp0 && a.q_gain)
+                           ? __ldg(a.q_gain + (lane % QLanes<D>::LPR + u * QLanes<D>::LPR) * 8 + e)
+                           : 1.f;
     if (warp == 0) {
         tc::tmem_alloc(smem_u32(s.tmem_slot), 512);
         tc::tmem_relinquish();
@@ -349,8 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                 const long long g = jt + j;
                 const int st = (int)(g % p.stages);
                 const long long ebase = it.e0 + (long long)j * kTileKeys;
-                const uint16_t *r0 = key_ptr(a, it.ks, it.b, it.bq, std::min(ebase + lane, it.e1 - 1));
-                const uint16_t *r1 = key_ptr(a, it.ks, it.b, it.bq, std::min(ebase + 32 + lane, it.e1 - 1));
+                bool v0, v1;
+                const uint16_t *r0 = key_slot(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0);
+                const uint16_t *r1 = key_slot(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1);
+                const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
                 if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag)) {
                     ok = false;
                     break;
@@ -370,37 +365,57 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
                              : "memory");
+                if (pw == 0 && lane == 0) {  // the mask travels with the tile (release by this arrive)
+                    s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
+                    mbar_arrive(smem_u32(s.kfull + st));
+                }
             }
             jt += it.ntiles;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 0) {
-        if (lane == 0) {
-            // -------------------------------------------------------- MMA issuer
-            // Event driven: P.V for tile i as soon as P_i is written, QK for the
-            // next tile as soon as its keys have landed and an S buffer is free.
-            // Descriptors are built once and advanced by constant offsets.
-            const uint64_t qdesc = tc::smem_desc(smem_u32(s.q), 1024, tc::kLayoutSw128);
-            const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
-            const uint64_t vdesc0 = tc::smem_desc_lbo(smem_u32(s.k), kTileKeys * 128, 1024, tc::kLayoutSw128);
-            const uint64_t pdesc0 = tc::smem_desc(smem_u32(s.p), 1024, tc::kLayoutSw128);
-            long long jt = 0;
-            uint32_t n_items = 0;
-            bool ok = true;
-            for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
-                const Item it = work_item(p, wi);
-                if (!mbar_wait(smem_u32(s.qready), n_items & 1u, p.ctx, s.abort_flag)) break;
-                tc::fence_after_sync();
-                if (it.ntiles == 0) mbar_arrive(smem_u32(s.qempty));
-                int nqk = 0, npv = 0;
-                uint64_t t_idle = 0;
-                while (npv < it.ntiles) {
-                    bool progressed = false;
-                    if (nqk < it.ntiles && nqk < npv + 2) {
-                        const long long g = jt + nqk;
-                        const int st = (int)(g % p.stages), sb = (int)(g & 1);
-                        if (mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1)) &&
-                            mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1))) {
+        // ------------------------------------------------------------ MMA issuer
+        // Event driven: P.V for tile i as soon as P_i is written, QK for the
+        // next tile as soon as its keys have landed and an S buffer is free.
+        // The whole warp runs the loop and polls (decisions are lane 0's, made
+        // warp-uniform by a shuffle); lane 0 issues.  Descriptors are built
+        // once and advanced by constant offsets.
+        const uint64_t qdesc = tc::smem_desc(smem_u32(s.q), 1024, tc::kLayoutSw128);
+        const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
+        const uint64_t vdesc0 = tc::smem_desc_lbo(smem_u32(s.k), kTileKeys * 128, 1024, tc::kLayoutSw128);
+        const uint64_t pdesc0 = tc::smem_desc(smem_u32(s.p), 1024, tc::kLayoutSw128);
+        const auto ready = [&](bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; };
+        long long jt = 0;
+        uint32_t n_items = 0;
+        bool ok = true;
+        for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
+            const Item it = work_item(p, wi);
+            // raw query rows of this item by TMA, once the previous item's QK MMAs are done with Q_hat
+            if (n_items > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx,
+                                                                 s.abort_flag)))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(smem_u32(s.qfull), Lt::kQBytes);
+                for (int c = 0; c < Lt::kChunks; ++c)
+                    tc::tma_load_3d(smem_u32(s.q + (size_t)c * kHeads * 128), &qmap, smem_u32(s.qfull), c * 64,
+                                    it.head0, (int)it.bq);
+            }
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qready), n_items & 1u, p.ctx, s.abort_flag))) break;
+            tc::fence_after_sync();
+            if (it.ntiles == 0 && lane == 0) mbar_arrive(smem_u32(s.qempty));
+            __syncwarp();
+            int nqk = 0, npv = 0;
+            uint64_t t_idle = 0;
+            while (npv < it.ntiles) {
+                bool progressed = false;
+                if (nqk < it.ntiles && nqk < npv + 2) {
+                    const long long g = jt + nqk;
+                    const int st = (int)(g % p.stages), sb = (int)(g & 1);
+                    const bool k_in = mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1));
+                    const bool s_free = mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1));
+                    if (ready(k_in && s_free)) {
+                        if (lane == 0) {
                             tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
                             tc::fence_after_sync();
                             const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
@@ -412,15 +427,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                                                 kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
                                                 (c | kk) ? 1u : 0u);
                             tc::mma_commit(smem_u32(s.sfull + sb));
-                            ++nqk;
-                            if (nqk == it.ntiles) tc::mma_commit(smem_u32(s.qempty));  // Q_hat no longer read
-                            progressed = true;
+                            if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty));  // Q_hat no longer read
                         }
+                        __syncwarp();
+                        ++nqk;
+                        progressed = true;
                     }
-                    if (npv < nqk) {
-                        const long long g = jt + npv;
-                        const int pb = (int)(g & 1), st = (int)(g % p.stages);
-                        if (mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1))) {
+                }
+                if (npv < nqk) {
+                    const long long g = jt + npv;
+                    const int pb = (int)(g & 1), st = (int)(g % p.stages);
+                    if (ready(mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1)))) {
+                        if (lane == 0) {
                             tc::fence_after_sync();
                             const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
                             const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
@@ -436,28 +454,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
                             tc::mma_commit(smem_u32(s.kempty + st));
                             tc::mma_commit(smem_u32(s.pempty + pb));
                             tc::mma_commit(smem_u32(s.oready + pb));
-                            ++npv;
-                            progressed = true;
                         }
-                    }
-                    if (progressed) {
-                        t_idle = 0;
-                    } else {
-                        const uint64_t now = global_timer_ns();
-                        if (t_idle == 0) {
-                            t_idle = now;
-                        } else if (now - t_idle > p.ctx.budget_ns || *s.abort_flag) {
-                            record_status(p.ctx.status, CSA_ERR_TIMEOUT);
-                            *s.abort_flag = 1;
-                            ok = false;
-                            break;
-                        }
+                        __syncwarp();
+                        ++npv;
+                        progressed = true;
                     }
                 }
-                jt += it.ntiles;
+                if (progressed) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = global_timer_ns();
+                    if (t_idle == 0) {
+                        t_idle = now;
+                    } else if (ready(now - t_idle > p.ctx.budget_ns || *s.abort_flag)) {
+                        if (lane == 0) {
+                            record_status(p.ctx.status, CSA_ERR_TIMEOUT);
+                            *s.abort_flag = 1;
+                        }
+                        __syncwarp();
+                        ok = false;
+                        break;
+                    }
+                }
             }
+            jt += it.ntiles;
         }
-        __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + output (warps 4..7)
         // Thread (quarter sp, lane l): head 16*sp + l%16 of this CTA's 64,
@@ -472,9 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
         for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
             const Item it = work_item(p, wi);
             const int h = it.head0 + hl;
-            // Q_hat of the previous item must have been consumed by its QK MMAs
-            if (n_items > 0 && !warp_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx, s.abort_flag)) break;
-            build_q<D>(a, s, it.bq, it.head0, sp);
+            if (!warp_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag)) break;
+            normalize_q<D>(a, s, sp, qg);
             tc::fence_proxy_async_smem();
             mbar_arrive(smem_u32(s.qready));
 
@@ -482,12 +502,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const AttTcParam
             for (int j = 0; j < it.ntiles && ok; ++j) {
                 const long long g = jt + j;
                 const int sb = (int)(g & 1);
-                const long long ebase = it.e0 + (long long)j * kTileKeys;
-                const uint64_t vmask = tile_mask(a, it.ks, it.bq, ebase, it.e1) >> (32 * kh);
                 if (!warp_wait(smem_u32(s.sfull + sb), (uint32_t)((g >> 1) & 1), p.ctx, s.abort_flag)) {
                     ok = false;
                     break;
                 }
+                // the stage's key mask (completed phase: acquires the producer's write)
+                const int st = (int)(g % p.stages);
+                if (!warp_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1), p.ctx, s.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t vmask = s.kmask[st] >> (32 * kh);
                 tc::fence_after_sync();
                 float sc[32];
                 tmem_ld_half32(tmem_s + lane_base + sb * kTileKeys, sc);
@@ -639,8 +664,17 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
     auto kern = attend_tc_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
+    CUtensorMap qmap;
+    {
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.n_bq};
+        const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2};
+        const uint32_t box[3] = {64, (uint32_t)kHeads, 1};
+        if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.q, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B))
+            return CSA_ERR_CUDA;
+    }
     const int grid = (int)std::min<long long>(p.n_work, num_sms());
-    kern<<<grid, kThreads, smem, st>>>(p);
+    kern<<<grid, kThreads, smem, st>>>(qmap, p);
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
     return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
 }

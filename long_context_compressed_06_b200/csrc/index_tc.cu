@@ -12,7 +12,7 @@
 //
 // Warp roles (192 threads):  warp 0 -- TMA producer (key tiles into a STAGES
 // ring, query tile once per query group); warp 1 -- TMEM owner and MMA issuer
-// (one thread; tcgen05.mma kind::f16, fp32 accumulate, two accumulator
+// (lane 0 issues; tcgen05.mma kind::f16, fp32 accumulate, two accumulator
 // buffers); warps 2..5 -- epilogue (tcgen05.ld, ReLU, weighted head sum,
 // causal mask, store).  Every mbarrier wait is bounded (csa_sync_status
 // reports a timeout).  Decode is HBM bound on the key stream (the MMA work per
@@ -108,7 +108,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0 && lane == 0) {
+    // The single-thread roles keep their whole warp in the loop: every lane
+    // polls the barriers (votes keep the warp converged), lane 0 issues.
+    const auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, p.ctx, abort_flag));
+    };
+    if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         long long it = 0, gi = 0;
         for (long long w = w0; w < w1; ++w) {
@@ -116,59 +121,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = (int)(wi.grp / p.groups_per_batch);
             const int g = (int)(wi.grp - (long long)b * p.groups_per_batch);
             if (wi.first_of_group) {
-                if (!mbar_wait(smem_u32(qempty), (uint32_t)((gi & 1) ^ 1), p.ctx, abort_flag)) break;
-                mbar_arrive_expect_tx(smem_u32(qfull), p.q_bytes);
-                for (int c = 0; c < p.nchunk; ++c)
-                    tc::tma_load_4d(smem_u32(q_smem + (size_t)c * p.n_cols * p.row_bytes), &qmap, smem_u32(qfull),
-                                    c * p.chunk_elems, 0, g * p.NQ, b);
+                if (!wait_all(qempty, (uint32_t)((gi & 1) ^ 1))) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(smem_u32(qfull), p.q_bytes);
+                    for (int c = 0; c < p.nchunk; ++c)
+                        tc::tma_load_4d(smem_u32(q_smem + (size_t)c * p.n_cols * p.row_bytes), &qmap,
+                                        smem_u32(qfull), c * p.chunk_elems, 0, g * p.NQ, b);
+                }
+                __syncwarp();
                 ++gi;
             }
             const int st = (int)(it % p.stages);
             const uint32_t ph = (uint32_t)((it / p.stages) & 1);
-            if (!mbar_wait(smem_u32(empty + st), ph ^ 1u, p.ctx, abort_flag)) break;
-            mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes);
-            uint8_t *dst = k_smem + (size_t)st * p.stage_bytes;
-            for (int c = 0; c < p.nchunk; ++c)
-                tc::tma_load_3d(smem_u32(dst + (size_t)c * kTileKeys * p.row_bytes), &kmap, smem_u32(full + st),
-                                c * p.chunk_elems, wi.kt * kTileKeys, b);
+            if (!wait_all(empty + st, ph ^ 1u)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes);
+                uint8_t *dst = k_smem + (size_t)st * p.stage_bytes;
+                for (int c = 0; c < p.nchunk; ++c)
+                    tc::tma_load_3d(smem_u32(dst + (size_t)c * kTileKeys * p.row_bytes), &kmap, smem_u32(full + st),
+                                    c * p.chunk_elems, wi.kt * kTileKeys, b);
+            }
+            __syncwarp();
             ++it;
         }
-        // drain: wait (bounded) for the copies this thread issued last into each stage
+        // drain: wait (bounded) for the copies this warp issued last into each stage
         for (long long j = std::max(0LL, it - p.stages); j < it; ++j)
             mbar_wait(smem_u32(full + (j % p.stages)), (uint32_t)((j / p.stages) & 1), p.ctx, nullptr);
         if (gi > 0) mbar_wait(smem_u32(qfull), (uint32_t)((gi - 1) & 1), p.ctx, nullptr);
-    } else if (warp == 1 && lane == 0) {
+        __syncwarp();
+    } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         long long it = 0, gi = 0;
         const uint32_t sbo = 8u * p.row_bytes;
         for (long long w = w0; w < w1; ++w) {
             const WorkItem wi = work_item(p, w, w0, w1);
             if (wi.first_of_group) {
-                if (!mbar_wait(smem_u32(qfull), (uint32_t)(gi & 1), p.ctx, abort_flag)) break;
+                if (!wait_all(qfull, (uint32_t)(gi & 1))) break;
                 ++gi;
             }
             const int acc = (int)(it & 1);
             const uint32_t aph = (uint32_t)((it >> 1) & 1);
-            if (!mbar_wait(smem_u32(tempty + acc), aph ^ 1u, p.ctx, abort_flag)) break;
+            if (!wait_all(tempty + acc, aph ^ 1u)) break;
             const int st = (int)(it % p.stages);
             const uint32_t ph = (uint32_t)((it / p.stages) & 1);
-            if (!mbar_wait(smem_u32(full + st), ph, p.ctx, abort_flag)) break;
+            if (!wait_all(full + st, ph)) break;
             tc::fence_after_sync();
             const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols);
             const uint32_t a0 = smem_u32(k_smem + (size_t)st * p.stage_bytes);
             const uint32_t b0 = smem_u32(q_smem);
-            uint32_t accumulate = 0;
-            for (int c = 0; c < p.nchunk; ++c) {
-                for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
-                    const uint64_t ad = tc::smem_desc(a0 + c * kTileKeys * p.row_bytes + kk * 32, sbo, p.layout);
-                    const uint64_t bd = tc::smem_desc(b0 + c * p.n_cols * p.row_bytes + kk * 32, sbo, p.layout);
-                    tc::mma_f16(d_tmem, ad, bd, p.idesc, accumulate);
-                    accumulate = 1;
+            if (lane == 0) {
+                uint32_t accumulate = 0;
+                for (int c = 0; c < p.nchunk; ++c) {
+                    for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
+                        const uint64_t ad = tc::smem_desc(a0 + c * kTileKeys * p.row_bytes + kk * 32, sbo, p.layout);
+                        const uint64_t bd = tc::smem_desc(b0 + c * p.n_cols * p.row_bytes + kk * 32, sbo, p.layout);
+                        tc::mma_f16(d_tmem, ad, bd, p.idesc, accumulate);
+                        accumulate = 1;
+                    }
                 }
+                tc::mma_commit(smem_u32(empty + st));
+                tc::mma_commit(smem_u32(tfull + acc));
+                if (wi.last_of_group) tc::mma_commit(smem_u32(qempty));
             }
-            tc::mma_commit(smem_u32(empty + st));
-            tc::mma_commit(smem_u32(tfull + acc));
-            if (wi.last_of_group) tc::mma_commit(smem_u32(qempty));
+            __syncwarp();
             ++it;
         }
     } else if (warp >= 2) {
@@ -196,11 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int acc = (int)(it & 1);
             const uint32_t aph = (uint32_t)((it >> 1) & 1);
-            // lane 0 polls, the warp follows (tcgen05.ld below is warp-collective)
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            __syncwarp();
+            // every lane polls and the warp votes (tcgen05.ld below is warp-collective;
+            // a single polling lane leaves the warp's following code much slower)
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag));
             if (!ok) break;
             tc::fence_after_sync();
             const long long s = (long long)wi.kt * kTileKeys + row;
@@ -231,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
+            __syncwarp();
             ++it;
         }
     }
