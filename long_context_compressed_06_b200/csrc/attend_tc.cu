@@ -365,9 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
                              : "memory");
-                if (pw == 0 && lane == 0) {  // the mask travels with the tile (release by this arrive)
-                    s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
-                    mbar_arrive(smem_u32(s.kfull + st));
+                if (pw == 0) {  // the mask travels with the tile (release by lane 0's arrive)
+                    if (lane == 0) s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
+                    mbar_arrive(smem_u32(s.kfull + st), lane == 0);
                 }
             }
             jt += it.ntiles;
@@ -378,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Event driven: P.V for tile i as soon as P_i is written, QK for the
         // next tile as soon as its keys have landed and an S buffer is free.
         // The whole warp runs the loop and polls (decisions are lane 0's, made
-        // warp-uniform by a shuffle); lane 0 issues.  Descriptors are built
+        // warp-uniform by a shuffle); lane 0 issues through guarded
+        // instructions, never a branch.  Descriptors are built
         // once and advanced by constant offsets.
         const uint64_t qdesc = tc::smem_desc(smem_u32(s.q), 1024, tc::kLayoutSw128);
         const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
@@ -394,17 +395,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n_items > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx,
                                                                  s.abort_flag)))
                 break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(smem_u32(s.qfull), Lt::kQBytes);
-                for (int c = 0; c < Lt::kChunks; ++c)
-                    tc::tma_load_3d(smem_u32(s.q + (size_t)c * kHeads * 128), &qmap, smem_u32(s.qfull), c * 64,
-                                    it.head0, (int)it.bq);
-            }
-            __syncwarp();
+            mbar_arrive_expect_tx(smem_u32(s.qfull), Lt::kQBytes, lane == 0);
+            for (int c = 0; c < Lt::kChunks; ++c)
+                tc::tma_load_3d(smem_u32(s.q + (size_t)c * kHeads * 128), &qmap, smem_u32(s.qfull), c * 64,
+                                it.head0, (int)it.bq, lane == 0);
             if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qready), n_items & 1u, p.ctx, s.abort_flag))) break;
             tc::fence_after_sync();
-            if (it.ntiles == 0 && lane == 0) mbar_arrive(smem_u32(s.qempty));
-            __syncwarp();
+            if (it.ntiles == 0) mbar_arrive(smem_u32(s.qempty), lane == 0);
             int nqk = 0, npv = 0;
             uint64_t t_idle = 0;
             while (npv < it.ntiles) {
@@ -415,21 +412,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool k_in = mbar_test_wait(smem_u32(s.kfull + st), (uint32_t)((g / p.stages) & 1));
                     const bool s_free = mbar_test_wait(smem_u32(s.sempty + sb), (uint32_t)(((g >> 1) & 1) ^ 1));
                     if (ready(k_in && s_free)) {
-                        if (lane == 0) {
-                            tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
-                            tc::fence_after_sync();
-                            const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
+                        const bool issuer = lane == 0;
+                        tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+                        tc::fence_after_sync();
+                        const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
 #pragma unroll
-                            for (int c = 0; c < Lt::kChunks; ++c)
+                        for (int c = 0; c < Lt::kChunks; ++c)
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
-                                                kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
-                                                (c | kk) ? 1u : 0u);
-                            tc::mma_commit(smem_u32(s.sfull + sb));
-                            if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty));  // Q_hat no longer read
-                        }
-                        __syncwarp();
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                                            kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
+                                            (c | kk) ? 1u : 0u, issuer);
+                        tc::mma_commit(smem_u32(s.sfull + sb), issuer);
+                        if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty), issuer);  // Q_hat no longer read
                         ++nqk;
                         progressed = true;
                     }
@@ -438,24 +433,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const long long g = jt + npv;
                     const int pb = (int)(g & 1), st = (int)(g % p.stages);
                     if (ready(mbar_test_wait(smem_u32(s.pfull + pb), (uint32_t)((g >> 1) & 1)))) {
-                        if (lane == 0) {
-                            tc::fence_after_sync();
-                            const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
-                            const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
+                        const bool issuer = lane == 0;
+                        tc::fence_after_sync();
+                        const uint64_t pd = pdesc0 + ((uint64_t)(pb * Lt::kPBytes) >> 4);
+                        const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
 #pragma unroll
-                            for (int kk = 0; kk < kTileKeys / 16; ++kk)
+                        for (int kk = 0; kk < kTileKeys / 16; ++kk)
 #pragma unroll
-                                for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
-                                    // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
-                                    // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
-                                    tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
-                                                vd + (((n0 / 64) * kTileKeys * 128 + kk * 16 * 128) >> 4),
-                                                p.idesc_pv, (npv == 0 && kk == 0) ? 0u : 1u);
-                            tc::mma_commit(smem_u32(s.kempty + st));
-                            tc::mma_commit(smem_u32(s.pempty + pb));
-                            tc::mma_commit(smem_u32(s.oready + pb));
-                        }
-                        __syncwarp();
+                            for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
+                                // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
+                                // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
+                                tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
+                                            vd + (((n0 / 64) * kTileKeys * 128 + kk * 16 * 128) >> 4), p.idesc_pv,
+                                            (npv == 0 && kk == 0) ? 0u : 1u, issuer);
+                        tc::mma_commit(smem_u32(s.kempty + st), issuer);
+                        tc::mma_commit(smem_u32(s.pempty + pb), issuer);
+                        tc::mma_commit(smem_u32(s.oready + pb), issuer);
                         ++npv;
                         progressed = true;
                     }

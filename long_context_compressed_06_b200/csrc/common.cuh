@@ -134,12 +134,18 @@ CSA_DEVINL bool mbar_wait(uint32_t bar, uint32_t parity, const DevCtx &ctx, vola
     }
 }
 
-CSA_DEVINL void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+// `pred` guards the arrive (one lane of a converged warp arrives).
+CSA_DEVINL void mbar_arrive(uint32_t bar, bool pred = true) {
+    asm volatile(
+        "{\n\t.reg .pred g;\n\tsetp.ne.b32 g, %1, 0;\n\t@g mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}"
+        ::"r"(bar), "r"((int)pred) : "memory");
 }
 
-CSA_DEVINL void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+CSA_DEVINL void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes, bool pred = true) {
+    asm volatile(
+        "{\n\t.reg .pred g;\n\tsetp.ne.b32 g, %2, 0;\n\t"
+        "@g mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}"
+        ::"r"(bar), "r"(bytes), "r"((int)pred) : "memory");
 }
 
 // ---------------------------------------------------------------- warp helpers

@@ -10,14 +10,14 @@
 // sum_h w_h * ReLU(.) is a loop over columns inside one thread, and a warp
 // stores 32 consecutive scores.
 //
-// Warp roles (192 threads):  warp 0 -- TMA producer (key tiles into a STAGES
+// Warp roles (320 threads):  warp 0 -- TMA producer (key tiles into a STAGES
 // ring, query tile once per query group); warp 1 -- TMEM owner and MMA issuer
-// (lane 0 issues; tcgen05.mma kind::f16, fp32 accumulate, two accumulator
-// buffers); warps 2..5 -- epilogue (tcgen05.ld, ReLU, weighted head sum,
-// causal mask, store).  Every mbarrier wait is bounded (csa_sync_status
-// reports a timeout).  Decode is HBM bound on the key stream (the MMA work per
-// tile is ~1/5 of the time the tile takes to arrive), prefill is bound by the
-// tensor cores and the epilogue.
+// (lane 0 issues; tcgen05.mma kind::f16, fp32 accumulate, four accumulator
+// buffers when N <= 128, else two); warps 2..9 -- two epilogue groups of four
+// warps taking alternate tiles (tcgen05.ld, ReLU, weighted head sum, causal
+// mask, store).  Every mbarrier wait is bounded (csa_sync_status reports a
+// timeout).  Decode streams the key cache from HBM; prefill is bound by the
+// epilogue (64 FMAs per key per query) rather than the tensor cores.
 #include <algorithm>
 
 #include "common.cuh"
@@ -27,9 +27,10 @@
 namespace csa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer warp, MMA warp, two epilogue groups of four warps
 constexpr int kTileKeys = 128;
 constexpr int kMaxStages = 6;
+constexpr int kMaxAcc = 4;   // TMEM accumulators (two when N = NQ x H_pad > 128)
 
 struct IndexTcParams {
     const float *w;       // [batch][nq][H_I]
@@ -42,24 +43,58 @@ struct IndexTcParams {
     int stages, nchunk, chunk_elems, row_bytes, layout;
     uint32_t stage_bytes, q_bytes, idesc;
     int n_cols;           // N of the MMA = NQ * H_pad
-    uint32_t tmem_cols;   // allocated columns (2 accumulators)
+    int n_acc;            // TMEM accumulators (2 or 4)
+    uint32_t tmem_cols;   // allocated columns (n_acc accumulators)
     DevCtx ctx;
 };
 
-struct WorkItem {
-    long long grp;
-    int kt;
-    bool first_of_group, last_of_group;
+// Position in a CTA's work range (sequence b, query group g, key tile kt),
+// advanced without divisions.
+struct Cursor {
+    long long w;
+    int kt, g, b;
 };
 
-CSA_DEVINL WorkItem work_item(const IndexTcParams &p, long long w, long long w0, long long w1) {
-    WorkItem it;
-    it.grp = w / p.n_ktiles;
-    it.kt = (int)(w - it.grp * p.n_ktiles);
-    it.first_of_group = (w == w0) || it.kt == 0;
-    it.last_of_group = (w == w1 - 1) || it.kt == p.n_ktiles - 1;
-    return it;
+CSA_DEVINL Cursor cursor_at(const IndexTcParams &p, long long w) {
+    Cursor c;
+    c.w = w;
+    const long long grp = w / p.n_ktiles;
+    c.kt = (int)(w - grp * p.n_ktiles);
+    c.b = (int)(grp / p.groups_per_batch);
+    c.g = (int)(grp - (long long)c.b * p.groups_per_batch);
+    return c;
 }
+
+CSA_DEVINL void advance(const IndexTcParams &p, Cursor &c) {
+    ++c.w;
+    if (++c.kt == p.n_ktiles) {
+        c.kt = 0;
+        if (++c.g == p.groups_per_batch) {
+            c.g = 0;
+            ++c.b;
+        }
+    }
+}
+
+// Named barrier of one epilogue group (128 threads).
+CSA_DEVINL void group_bar(int eg) {
+    if (eg == 0)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    else
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+// Slot and phase of a ring of n barriers.
+struct Ring {
+    int idx = 0;
+    uint32_t phase = 0;
+    CSA_DEVINL void next(int n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -69,13 +104,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *k_smem = base;
     uint8_t *q_smem = k_smem + (size_t)p.stages * p.stage_bytes;
-    float *w_s = reinterpret_cast<float *>(q_smem + p.q_bytes);          // [NQ][H_pad]
-    int *nvis_s = reinterpret_cast<int *>(w_s + p.NQ * p.H_pad);         // [NQ]
+    float *w_s = reinterpret_cast<float *>(q_smem + p.q_bytes);          // [2 groups][NQ][H_pad]
+    int *nvis_s = reinterpret_cast<int *>(w_s + 2 * p.NQ * p.H_pad);     // [2 groups][NQ]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
-        (reinterpret_cast<uintptr_t>(nvis_s + p.NQ) + 7) & ~uintptr_t(7));
+        (reinterpret_cast<uintptr_t>(nvis_s + 2 * p.NQ) + 7) & ~uintptr_t(7));
     uint64_t *full = bars, *empty = bars + kMaxStages;
-    uint64_t *tfull = bars + 2 * kMaxStages, *tempty = tfull + 2;
-    uint64_t *qfull = tempty + 2, *qempty = qfull + 1;
+    uint64_t *tfull = bars + 2 * kMaxStages, *tempty = tfull + kMaxAcc;
+    uint64_t *qfull = tempty + kMaxAcc, *qempty = qfull + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -88,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < p.n_acc; ++a) {
             mbar_init(tfull + a, 1);
             mbar_init(tempty + a, 4);
         }
@@ -109,39 +144,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     // The single-thread roles keep their whole warp in the loop: every lane
-    // polls the barriers (votes keep the warp converged), lane 0 issues.
+    // polls the barriers (votes keep the warp converged) and lane 0 issues
+    // through guarded instructions, never a branch.
     const auto wait_all = [&](uint64_t *bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, p.ctx, abort_flag));
     };
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         long long it = 0, gi = 0;
-        for (long long w = w0; w < w1; ++w) {
-            const WorkItem wi = work_item(p, w, w0, w1);
-            const int b = (int)(wi.grp / p.groups_per_batch);
-            const int g = (int)(wi.grp - (long long)b * p.groups_per_batch);
-            if (wi.first_of_group) {
+        Ring kr;
+        for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
+            if (cu.w == w0 || cu.kt == 0) {
                 if (!wait_all(qempty, (uint32_t)((gi & 1) ^ 1))) break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(smem_u32(qfull), p.q_bytes);
-                    for (int c = 0; c < p.nchunk; ++c)
-                        tc::tma_load_4d(smem_u32(q_smem + (size_t)c * p.n_cols * p.row_bytes), &qmap,
-                                        smem_u32(qfull), c * p.chunk_elems, 0, g * p.NQ, b);
-                }
-                __syncwarp();
+                mbar_arrive_expect_tx(smem_u32(qfull), p.q_bytes, lane == 0);
+                for (int c = 0; c < p.nchunk; ++c)
+                    tc::tma_load_4d(smem_u32(q_smem + (size_t)c * p.n_cols * p.row_bytes), &qmap, smem_u32(qfull),
+                                    c * p.chunk_elems, 0, cu.g * p.NQ, cu.b, lane == 0);
                 ++gi;
             }
-            const int st = (int)(it % p.stages);
-            const uint32_t ph = (uint32_t)((it / p.stages) & 1);
-            if (!wait_all(empty + st, ph ^ 1u)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes);
-                uint8_t *dst = k_smem + (size_t)st * p.stage_bytes;
-                for (int c = 0; c < p.nchunk; ++c)
-                    tc::tma_load_3d(smem_u32(dst + (size_t)c * kTileKeys * p.row_bytes), &kmap, smem_u32(full + st),
-                                    c * p.chunk_elems, wi.kt * kTileKeys, b);
-            }
-            __syncwarp();
+            const int st = kr.idx;
+            if (!wait_all(empty + st, kr.phase ^ 1u)) break;
+            mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes, lane == 0);
+            uint8_t *dst = k_smem + (size_t)st * p.stage_bytes;
+            for (int c = 0; c < p.nchunk; ++c)
+                tc::tma_load_3d(smem_u32(dst + (size_t)c * kTileKeys * p.row_bytes), &kmap, smem_u32(full + st),
+                                c * p.chunk_elems, cu.kt * kTileKeys, cu.b, lane == 0);
+            kr.next(p.stages);
             ++it;
         }
         // drain: wait (bounded) for the copies this warp issued last into each stage
@@ -151,77 +179,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        long long it = 0, gi = 0;
+        long long gi = 0;
+        Ring kr, ar;
         const uint32_t sbo = 8u * p.row_bytes;
-        for (long long w = w0; w < w1; ++w) {
-            const WorkItem wi = work_item(p, w, w0, w1);
-            if (wi.first_of_group) {
+        // descriptors built once, advanced by constant offsets (16-byte units)
+        const uint64_t kdesc0 = tc::smem_desc(smem_u32(k_smem), sbo, p.layout);
+        const uint64_t qdesc0 = tc::smem_desc(smem_u32(q_smem), sbo, p.layout);
+        const bool issuer = lane == 0;
+        for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
+            if (cu.w == w0 || cu.kt == 0) {
                 if (!wait_all(qfull, (uint32_t)(gi & 1))) break;
                 ++gi;
             }
-            const int acc = (int)(it & 1);
-            const uint32_t aph = (uint32_t)((it >> 1) & 1);
-            if (!wait_all(tempty + acc, aph ^ 1u)) break;
-            const int st = (int)(it % p.stages);
-            const uint32_t ph = (uint32_t)((it / p.stages) & 1);
-            if (!wait_all(full + st, ph)) break;
+            const int acc = ar.idx;
+            if (!wait_all(tempty + acc, ar.phase ^ 1u)) break;
+            const int st = kr.idx;
+            if (!wait_all(full + st, kr.phase)) break;
             tc::fence_after_sync();
             const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols);
-            const uint32_t a0 = smem_u32(k_smem + (size_t)st * p.stage_bytes);
-            const uint32_t b0 = smem_u32(q_smem);
-            if (lane == 0) {
-                uint32_t accumulate = 0;
-                for (int c = 0; c < p.nchunk; ++c) {
-                    for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
-                        const uint64_t ad = tc::smem_desc(a0 + c * kTileKeys * p.row_bytes + kk * 32, sbo, p.layout);
-                        const uint64_t bd = tc::smem_desc(b0 + c * p.n_cols * p.row_bytes + kk * 32, sbo, p.layout);
-                        tc::mma_f16(d_tmem, ad, bd, p.idesc, accumulate);
-                        accumulate = 1;
-                    }
+            const uint64_t kd = kdesc0 + ((uint64_t)(st * p.stage_bytes) >> 4);
+            uint32_t accumulate = 0;
+            for (int c = 0; c < p.nchunk; ++c) {
+                for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
+                    tc::mma_f16(d_tmem, kd + ((uint32_t)(c * kTileKeys * p.row_bytes + kk * 32) >> 4),
+                                qdesc0 + ((uint32_t)(c * p.n_cols * p.row_bytes + kk * 32) >> 4), p.idesc, accumulate,
+                                issuer);
+                    accumulate = 1;
                 }
-                tc::mma_commit(smem_u32(empty + st));
-                tc::mma_commit(smem_u32(tfull + acc));
-                if (wi.last_of_group) tc::mma_commit(smem_u32(qempty));
             }
-            __syncwarp();
-            ++it;
+            tc::mma_commit(smem_u32(empty + st), issuer);
+            tc::mma_commit(smem_u32(tfull + acc), issuer);
+            if (cu.w == w1 - 1 || cu.kt == p.n_ktiles - 1) tc::mma_commit(smem_u32(qempty), issuer);
+            kr.next(p.stages);
+            ar.next(p.n_acc);
         }
     } else if (warp >= 2) {
         // ------------------------------------------------------------ epilogue
+        // Two groups of four warps take alternate tiles (tile i -> group i & 1,
+        // accumulator i % n_acc), doubling the epilogue rate.
+        const int eg = (warp - 2) >> 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
-        const int et = threadIdx.x - 64;  // 0..127
-        long long it = 0;
-        for (long long w = w0; w < w1; ++w) {
-            const WorkItem wi = work_item(p, w, w0, w1);
-            const int b = (int)(wi.grp / p.groups_per_batch);
-            const int g = (int)(wi.grp - (long long)b * p.groups_per_batch);
-            if (wi.first_of_group) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int et = (threadIdx.x - 64) & 127;
+        float *ws_g = w_s + eg * p.NQ * p.H_pad;
+        int *nv_g = nvis_s + eg * p.NQ;
+        int loaded_b = -1, loaded_g = -1;
+        for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
+            const int li = (int)(cu.w - w0);
+            if ((li & 1) != eg) continue;
+            const int b = cu.b, g = cu.g;
+            if (b != loaded_b || g != loaded_g) {
+                group_bar(eg);
                 for (int i = et; i < p.NQ * p.H_pad; i += 128) {
                     const int qi = i / p.H_pad, h = i - qi * p.H_pad;
                     const int q = g * p.NQ + qi;
-                    w_s[i] = (q < p.nq && h < p.H_I) ? __ldg(p.w + ((size_t)b * p.nq + q) * p.H_I + h) : 0.f;
+                    ws_g[i] = (q < p.nq && h < p.H_I) ? __ldg(p.w + ((size_t)b * p.nq + q) * p.H_I + h) : 0.f;
                 }
                 for (int qi = et; qi < p.NQ; qi += 128) {
                     const int q = g * p.NQ + qi;
-                    nvis_s[qi] = q < p.nq ? (int)n_visible(__ldg(p.q_pos + (size_t)b * p.nq + q), p.m, p.N) : 0;
+                    nv_g[qi] = q < p.nq ? (int)n_visible(__ldg(p.q_pos + (size_t)b * p.nq + q), p.m, p.N) : 0;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                group_bar(eg);
+                loaded_b = b;
+                loaded_g = g;
             }
-            const int acc = (int)(it & 1);
-            const uint32_t aph = (uint32_t)((it >> 1) & 1);
+            const int acc = li & (p.n_acc - 1);
+            const uint32_t aph = (uint32_t)((li / p.n_acc) & 1);
             // every lane polls and the warp votes (tcgen05.ld below is warp-collective;
             // a single polling lane leaves the warp's following code much slower)
             const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag));
             if (!ok) break;
             tc::fence_after_sync();
-            const long long s = (long long)wi.kt * kTileKeys + row;
+            const long long s = (long long)cu.kt * kTileKeys + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.n_cols);
             for (int qi = 0; qi < p.NQ; ++qi) {
                 const int q = g * p.NQ + qi;
                 if (q >= p.nq) break;
-                float score = 0.f;
+                // four independent partial sums (one per 16-column load) keep the
+                // FMA chains short
+                float part[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int hc = 0; hc < p.H_pad; hc += 64) {
                     // up to four 16-column loads in flight per wait
                     float v[64];
@@ -230,22 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int u = 0; u < 4; ++u)
                         if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
                     tc::tmem_wait_ld();
-                    const float *ws = w_s + qi * p.H_pad + hc;
+                    const float *ws = ws_g + qi * p.H_pad + hc;
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         if (u < nl) {
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
-                                score = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), score);
+                                part[u] = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), part[u]);
                         }
                 }
-                if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nvis_s[qi] ? score : -INFINITY;
+                const float score = (part[0] + part[1]) + (part[2] + part[3]);
+                if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nv_g[qi] ? score : -INFINITY;
             }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
-            __syncwarp();
-            ++it;
+            mbar_arrive(smem_u32(tempty + acc), lane == 0);
         }
     }
     tc::fence_before_sync();
@@ -285,8 +320,9 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
     p.stages = (int)std::min<size_t>(kMaxStages, (smem_cap - p.q_bytes) / p.stage_bytes);
     if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
     p.idesc = tc::idesc_f16(p.n_cols, true);
+    p.n_acc = p.n_cols <= 128 ? 4 : 2;
     uint32_t cols = 32;
-    while (cols < 2u * (uint32_t)p.n_cols) cols *= 2;
+    while (cols < (uint32_t)(p.n_acc * p.n_cols)) cols *= 2;
     p.tmem_cols = cols;
     p.groups_per_batch = (nq + NQ - 1) / NQ;
     p.n_ktiles = (int)((N + kTileKeys - 1) / kTileKeys);
@@ -308,8 +344,8 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
         if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q_idx, dims, strides, box, sw))
             return CSA_ERR_CUDA;
     }
-    const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + p.q_bytes + (size_t)NQ * p.H_pad * 4 + NQ * 4 +
-                        8 + (2 * kMaxStages + 6) * 8 + 16;
+    const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + p.q_bytes + 2 * ((size_t)NQ * p.H_pad * 4 + NQ * 4) +
+                        8 + (2 * kMaxStages + 2 * kMaxAcc + 2) * 8 + 16;
     if (cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
     const int grid = (int)std::min<long long>(p.total_work, num_sms());
