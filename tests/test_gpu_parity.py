@@ -314,6 +314,9 @@ def test_quantize_fp4_bit_exact(cuda):
 @pytest.mark.parametrize("batch,nq,H_I,d_I,N,m,ts", [
     (1, 1, 64, 128, 4096, 4, [16383]),
     (2, 2, 16, 64, 777, 4, [3107, 50, 3000, 7]),
+    (1, 40, 64, 128, 2048, 4, [8191 - 197 * i for i in range(40)]),   # several query groups per sequence
+    (2, 1, 32, 256, 1500, 4, [5999, 2001]),                              # d_I = 256, ragged last tile
+    (1, 1, 4, 32, 300, 4, [1199]),                                       # d_I = 32: CUDA-core path
 ])
 def test_index_fp4_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
     qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts, seed=80)
