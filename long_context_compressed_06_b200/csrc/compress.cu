@@ -135,7 +135,10 @@ __global__ void __launch_bounds__(256) compress_small_kernel(
 // `rank` owns channels [rank*dc, (rank+1)*dc).  The 256 threads are RG row
 // groups x (dc/8) channel chunks while pooling (thread sums rows rg, rg+RG, ..)
 // and E entries x dc channels (one output each) while reducing/normalising.
-template <int E>
+// A thread issues the 16-byte loads of NR of its rows of every entry of the
+// group before the first FMA, so E*NR loads per thread are in flight (the op
+// is bound by HBM latency x bytes in flight); larger m takes several batches.
+template <int E, int NR>
 __global__ void __launch_bounds__(256, 1) compress_cluster_kernel(
     const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, const float *__restrict__ logits,
     int batch, long long T, int d, int m, int apply_rms, const float *__restrict__ gain, float eps,
@@ -164,30 +167,50 @@ __global__ void __launch_bounds__(256, 1) compress_cluster_kernel(
         const long long b = it / groups, i0 = (it - b * groups) * E;
         const uint16_t *Ab = A + (size_t)b * T * d + c_base + chunk * 8;
         const uint16_t *Bb = B + (size_t)b * T * d + c_base + chunk * 8;
+        float acc[E][8];
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            float acc[8];
+        for (int e = 0; e < E; ++e)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-            const long long i = i0 + e;
-            if (i < N) {
-                for (int r = rg; r < 2 * m; r += RG) {
-                    if (i == 0) {
+            for (int q = 0; q < 8; ++q) acc[e][q] = 0.f;
+        for (int r0 = rg; r0 < 2 * m; r0 += RG * NR) {
+            // all loads of this batch first (rows past 2m or N, and entry 0's missing B half, read nothing)
+            uint4 x[E][NR];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const long long i = i0 + e;
+#pragma unroll
+                for (int k = 0; k < NR; ++k) {
+                    const int r = r0 + RG * k;
+                    const uint16_t *src = nullptr;
+                    if (i < N && r < 2 * m) {
                         if (r >= m)
-                            fma8(acc, w_first + (size_t)(r - m) * dc + chunk * 8,
-                                 ldg_stream(Ab + (size_t)(r - m) * d));
-                    } else if (r < m) {
-                        fma8(acc, w_full + (size_t)r * dc + chunk * 8,
-                             ldg_stream(Bb + (size_t)((i - 1) * m + r) * d));
+                            src = Ab + (size_t)(i * m + r - m) * d;
+                        else if (i > 0)
+                            src = Bb + (size_t)((i - 1) * m + r) * d;
+                    }
+                    x[e][k] = src ? ldg_stream(src) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const long long i = i0 + e;
+#pragma unroll
+                for (int k = 0; k < NR; ++k) {
+                    const int r = r0 + RG * k;
+                    if (r >= 2 * m) continue;
+                    if (i == 0) {
+                        if (r >= m) fma8(acc[e], w_first + (size_t)(r - m) * dc + chunk * 8, x[e][k]);
                     } else {
-                        fma8(acc, w_full + (size_t)r * dc + chunk * 8,
-                             ldg_stream(Ab + (size_t)(i * m + r - m) * d));
+                        fma8(acc[e], w_full + (size_t)r * dc + chunk * 8, x[e][k]);
                     }
                 }
             }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
             float4 *dst = reinterpret_cast<float4 *>(red + ((size_t)rg * E + e) * dc + chunk * 8);
-            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            dst[0] = make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
+            dst[1] = make_float4(acc[e][4], acc[e][5], acc[e][6], acc[e][7]);
         }
         __syncthreads();
         float v = 0.f;
@@ -266,7 +289,19 @@ int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, i
     const int RG = 256 / (dc / 8);
     const size_t smem = ((size_t)3 * m * dc + (size_t)RG * E * dc + 2 * E + 8) * sizeof(float);
     if (smem > 220 * 1024) return CSA_ERR_UNSUPPORTED;
-    auto k = E == 4 ? compress_cluster_kernel<4> : (E == 2 ? compress_cluster_kernel<2> : compress_cluster_kernel<1>);
+    // loads in flight per thread: E entries x NR rows (32 registers of uint4 at most)
+    const int rows_per_thread = (2 * m + RG - 1) / RG;
+    int NR = 32 / E;
+    while (NR > 1 && NR / 2 >= rows_per_thread) NR /= 2;
+    void (*k)(const uint16_t *, const uint16_t *, const float *, int, long long, int, int, int, const float *,
+              float, uint16_t *, long long, int) = nullptr;
+#define CSA_CK(e_, nr_) \
+    if (E == e_ && NR == nr_) k = compress_cluster_kernel<e_, nr_>;
+    CSA_CK(4, 1) CSA_CK(4, 2) CSA_CK(4, 4) CSA_CK(4, 8)
+    CSA_CK(2, 1) CSA_CK(2, 2) CSA_CK(2, 4) CSA_CK(2, 8) CSA_CK(2, 16)
+    CSA_CK(1, 1) CSA_CK(1, 2) CSA_CK(1, 4) CSA_CK(1, 8) CSA_CK(1, 16) CSA_CK(1, 32)
+#undef CSA_CK
+    if (!k) return CSA_ERR_UNSUPPORTED;
     err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return CSA_ERR_CUDA;
     const long long items = (long long)batch * ((N + E - 1) / E);

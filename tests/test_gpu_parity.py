@@ -54,6 +54,8 @@ def positions(batch, nq, ts):
     (2, 300, 256, 16, True, True),
     (3, 5, 64, 4, True, False),         # N = 1
     (1, 1000, 1024, 64, True, False),   # cluster kernel, dc = 128
+    (1, 1000, 256, 20, True, True),     # cluster kernel, m not a multiple of the row groups
+    (1, 3 * 160 + 50, 128, 160, True, False),   # cluster kernel, two row batches per entry
 ])
 def test_compress_parity(cuda, batch, T, d, m, rms, use_gain):
     A = seeded((batch, T, d), 11)
