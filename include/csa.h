@@ -147,6 +147,33 @@ int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long
              void *stream);
 
 /*
+ * csa_rescore_topk -- re-ranks FP4-indexer candidates with the bf16 index keys.
+ * The FP4 page ("DeepSeek V4 paper full version is out, FP4 QAT details")
+ * reports 99.7 % recall of the full-precision selection for FP4 activations in
+ * the indexer QK path (on real activations).  On i.i.d. synthetic data a
+ * single FP4 selection recalls ~86 % of the bf16-operand top-k; this call is
+ * the second stage of an over-select-and-re-score reading of that passage:
+ * csa_index_fp4 + csa_topk pick kc > k candidates, then for each candidate
+ *   S_c[j] = sum_h w[h] * max(0, q_idx[h] . k_idx[cand[j]])   (bf16 operands,
+ *            fp32 arithmetic -- exactly the csa_index score; -1 or out-of-range
+ *            candidates score -inf)
+ * and idx = the k best candidates (ties towards the lower candidate slot, i.e.
+ * the lower entry index when cand is ascending), written in candidate order
+ * (ascending entries for ascending cand), -1 padded.
+ *   q_idx [batch][nq][H_I][d_I] bf16   w [batch][nq][H_I] fp32
+ *   k_idx [batch][N][d_I] bf16         cand [batch][nq][kc] int32 (from csa_topk)
+ *   idx   [batch][nq][k] int32
+ * Requirements: k <= 8192; kc <= 2^19; H_I * d_I * 4 <= 200 KiB.  Workspace:
+ * csa_rescore_workspace_bytes, 256-byte aligned (CSA_ERR_WORKSPACE otherwise).
+ * Causality is the candidates' (they come from a causal csa_topk).
+ */
+size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k);
+int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx,
+                     const int *cand, int kc, int batch, int nq, long long N, int H_I,
+                     int d_I, int k, int *idx, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/*
  * csa_attend -- core attention of CSA: multi-query attention with H query
  * heads sharing one KV head (K = V) over the selected compressed entries plus
  * a sliding window of raw stream-A rows (techniques map rows "Grouped-query

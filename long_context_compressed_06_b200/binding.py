@@ -46,6 +46,8 @@ def load() -> ctypes.CDLL:
         "csa_index_fp4": ([P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
         "csa_topk_workspace_bytes": ([i32, i32, i64, i32], sz),
         "csa_topk": ([P, P, i32, i32, i64, i32, i32, P, P, sz, P], i32),
+        "csa_rescore_workspace_bytes": ([i32, i32, i32, i32], sz),
+        "csa_rescore_topk": ([P, P, P, P, i32, i32, i32, i64, i32, i32, i32, P, P, sz, P], i32),
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
         "csa_attend": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
         "hca_attend": ([P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
@@ -165,6 +167,31 @@ def csa_topk(scores, q_pos, m: int, k: int, idx=None):
     if idx is None:
         idx = torch.empty((batch, nq, k), dtype=torch.int32, device=scores.device)
     _check(L.csa_topk(_p(scores), _p(q_pos), batch, nq, N, m, k, _p(idx), None, 0, _stream()), "csa_topk")
+    return idx
+
+
+def rescore_workspace_bytes(batch: int, nq: int, kc: int, k: int) -> int:
+    return int(load().csa_rescore_workspace_bytes(batch, nq, kc, k))
+
+
+def csa_rescore_topk(q_idx, w, k_idx, cand, k: int, idx=None, workspace=None):
+    """Re-rank FP4 candidates cand [b][nq][kc] with the bf16 index keys; -> idx [b][nq][k]."""
+    L = load()
+    _need(q_idx, torch.bfloat16, "q_idx", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(k_idx, torch.bfloat16, "k_idx", 3)
+    _need(cand, torch.int32, "cand", 3)
+    batch, nq, H_I, d_I = q_idx.shape
+    N = k_idx.shape[1]
+    kc = cand.shape[2]
+    if idx is None:
+        idx = torch.empty((batch, nq, k), dtype=torch.int32, device=q_idx.device)
+    nbytes = rescore_workspace_bytes(batch, nq, kc, k)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q_idx.device)
+    _check(L.csa_rescore_topk(_p(q_idx), _p(w), _p(k_idx), _p(cand), kc, batch, nq, N, H_I, d_I, k, _p(idx),
+                              _p(workspace), workspace.numel() * workspace.element_size(), _stream()),
+           "csa_rescore_topk")
     return idx
 
 

@@ -154,6 +154,26 @@ int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long
     return csa::launch_topk(scores, q_pos, batch, nq, N, m, k, idx, S(stream));
 }
 
+size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k) {
+    if (batch < 1 || nq < 1 || kc < 1 || k < 1) return 0;
+    return csa::rescore_workspace_bytes(batch, nq, kc, k);
+}
+
+int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
+                     int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+    if (!al16(q_idx) || !al4(w) || !al16(k_idx) || !al4(cand) || !al4(idx)) return CSA_ERR_INVALID;
+    if (batch < 1 || nq < 1 || N < 1 || kc < 1 || k < 1 || H_I < 1 || d_I < 16 || d_I % 16 != 0)
+        return CSA_ERR_INVALID;
+    if (k > 8192 || kc > (1 << 19) || N > (1LL << 31) - 1 || !csa::rescore_supported(H_I, d_I))
+        return CSA_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < csa::rescore_workspace_bytes(batch, nq, kc, k))
+        return CSA_ERR_WORKSPACE;
+    return csa::launch_rescore_topk(q_idx, w, k_idx, cand, kc, batch, nq, N, H_I, d_I, k, idx, workspace,
+                                    S(stream));
+}
+
 size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys) {
     if (batch < 1 || nq < 1 || H < 1 || D < 1 || max_keys < 1) return 0;
     return csa::attend_workspace_bytes(batch, nq, H, D, max_keys);

@@ -26,8 +26,15 @@ int launch_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, cons
                      int d_I, int m, float *scores, const DevCtx &ctx, cudaStream_t st);
 
 size_t topk_workspace_bytes(int batch, int nq, long long N, int k);
+// q_pos may be null inside the library: every entry is then eligible.
 int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k,
                 int *idx, cudaStream_t st);
+
+size_t rescore_workspace_bytes(int batch, int nq, int kc, int k);
+bool rescore_supported(int H_I, int d_I);
+int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
+                        int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *ws,
+                        cudaStream_t st);
 
 // Attention: dense selects the HCA key set of the first n_vis(t) entries;
 // otherwise the k selected entries idx (may be null when k == 0).

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
 
     for (int i = threadIdx.x; i < 2 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
 
-    const long long nv = n_visible(q_pos[bq], m, N);
+    const long long nv = q_pos ? n_visible(q_pos[bq], m, N) : N;  // no q_pos: every entry is eligible
     const long long kk = nv < k ? nv : k;
     const long long seg0 = ((long long)rank * kTopkThreads + threadIdx.x) * R;
     const int nloc = (int)(nv - seg0 <= 0 ? 0 : (nv - seg0 >= R ? R : nv - seg0));

@@ -91,6 +91,22 @@ def test_topk_validation(lib):
     assert lib.csa_topk_workspace_bytes(8, 1, 32768, 1024) == 0
 
 
+def test_rescore_validation_and_workspace(lib):
+    f = lib.csa_rescore_topk
+    ws = ctypes.c_void_p(0x40000)          # 256-byte aligned
+    need = lib.csa_rescore_workspace_bytes(4, 1, 4096, 1024)
+    assert need >= 4 * 4096 * 4 + 4 * 1024 * 4
+    args = (A16, A16, A16, A16, 4096, 4, 1, 262144, 64, 128, 1024, A16b)
+    assert f(NULL, *args[1:], ws, need, NULL) == csa.CSA_ERR_INVALID                    # q_idx
+    assert f(*args[:3], NULL, *args[4:], ws, need, NULL) == csa.CSA_ERR_INVALID        # cand
+    assert f(*args[:10], 0, A16b, ws, need, NULL) == csa.CSA_ERR_INVALID               # k
+    assert f(*args[:10], 9000, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED
+    assert f(*args[:8], 256, 256, 1024, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED  # query too big
+    assert f(*args, ws, need - 1, NULL) == csa.CSA_ERR_WORKSPACE
+    assert f(*args, ctypes.c_void_p(0x40010), need, NULL) == csa.CSA_ERR_WORKSPACE     # misaligned workspace
+    assert f(*args, NULL, need, NULL) == csa.CSA_ERR_WORKSPACE
+
+
 def test_attend_validation_and_workspace(lib):
     f = lib.csa_attend
     args = dict(q=A16, g=NULL, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048, W=16, pos=A16, b=1, nq=1, H=8,

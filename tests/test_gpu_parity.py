@@ -331,6 +331,51 @@ def test_index_fp4_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
     _check_scores(got, ref, 1e-5)
 
 
+@pytest.mark.parametrize("batch,nq,H_I,d_I,N,kc,k", [
+    (2, 1, 64, 128, 8192, 2048, 512),      # decode shape, over-select 4x
+    (1, 3, 16, 64, 1000, 300, 100),        # several queries, small
+])
+def test_rescore_topk_matches_oracle(cuda, batch, nq, H_I, d_I, N, kc, k):
+    """FP4 over-selection re-ranked with the bf16 keys.  The candidates are the
+    oracle's own FP4 selection; the expected result is the oracle's exact
+    bf16-operand scores restricted to those candidates."""
+    m = 4
+    ts = [N * m - 1 - 5 * i for i in range(batch * nq)]
+    qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts, seed=90)
+    wn, qpn = w.cpu().numpy(), qp.cpu().numpy()
+    rq4, rq4s = oracle.quantize_fp4(bits(qI))
+    rk4, rk4s = oracle.quantize_fp4(bits(kI))
+    cand = oracle.topk(oracle.index_fp4(rq4, rq4s, wn, rk4, rk4s, qpn, m), qpn, m, kc)
+    # ascending entries, -1 slots last (the order csa_topk writes)
+    cand = np.where(cand < 0, np.iinfo(np.int32).max, cand)
+    cand.sort(axis=-1)
+    cand = np.where(cand == np.iinfo(np.int32).max, -1, cand).astype(np.int32)
+    got = cuda.csa_rescore_topk(qI, w, kI, torch.from_numpy(cand).to(DEV), k).cpu().numpy()
+    S16 = oracle.index(bits(qI), wn, bits(kI), qpn, m)
+    masked = np.full_like(S16, -np.inf)
+    for q in np.ndindex(cand.shape[:-1]):
+        c = cand[q][cand[q] >= 0]
+        masked[q][c] = S16[q][c]
+    _check_topk_band(got, masked, qpn, m, k, N)
+    # every returned entry is one of the candidates, in ascending order
+    for q in np.ndindex(cand.shape[:-1]):
+        g = got[q][got[q] >= 0]
+        assert set(g.tolist()) <= set(cand[q].tolist())
+        assert np.all(np.diff(g) > 0)
+
+
+def test_rescore_topk_with_every_entry_is_plain_topk(cuda):
+    """With every entry as a candidate (and -1 slots mixed in) the re-ranking is
+    the plain top-k of the bf16-operand scores."""
+    batch, nq, H_I, d_I, N, m, k = 2, 1, 64, 128, 3000, 4, 256
+    qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, [N * m - 1] * batch, seed=95)
+    cand = np.tile(np.arange(N, dtype=np.int32), (batch, nq, 1))
+    cand = np.concatenate([cand, np.full((batch, nq, 77), -1, np.int32)], axis=2)
+    got = cuda.csa_rescore_topk(qI, w, kI, torch.from_numpy(cand).to(DEV), k).cpu().numpy()
+    ref = oracle.index(bits(qI), w.cpu().numpy(), bits(kI), qp.cpu().numpy(), m)
+    _check_topk_band(got, ref, qp.cpu().numpy(), m, k, N)
+
+
 # ----------------------------------------------------------------------------- failure path
 def test_bounded_wait_times_out_and_context_survives(cuda):
     assert cuda.csa_sync_status() == 0
