@@ -615,6 +615,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress"],
+                    help="run one of the other workloads alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -627,6 +629,19 @@ def main():
     import long_context_compressed_06_b200 as csa
     csa.load()
     peaks, peak_kind = load_peaks()
+    if args.only:
+        run_one = {"prefill": lambda: bench_prefill(csa, args, device, peaks),
+                   "hca": lambda: bench_hca(csa, args, device, peaks),
+                   "fp4": lambda: bench_fp4(csa, args, device, peaks),
+                   "compress": lambda: bench_compress(csa, args, device, peaks, W.HCA_DECODE)}[args.only]
+        res = run_one()
+        rc = csa.csa_sync_status()
+        if rc != 0:
+            raise RuntimeError("device status: %s" % csa.strerror(rc))
+        if rank == 0:
+            print(json.dumps(res))
+        barrier(world)
+        return 0
 
     head, _ = bench_csa_decode(csa, args, device, world, rank, peaks)
     rc = csa.csa_sync_status()
