@@ -20,14 +20,18 @@
 // no exchange; each streams the gathered rows itself (the second read of a
 // row is an L2 hit).
 //
-// Warp roles (256 threads): warp 0 TMEM owner + MMA issuer (lane 0 issues);
-// warps 1..3 gather the key rows with 16-byte cp.async into the 128-byte
-// swizzled layout (one 512-byte coalesced row segment per warp instruction);
-// warps 4..7 softmax and output, two threads per head (keys 0-31 / 32-63,
-// D/2 output columns each); all eight warps build Q_hat for each query.  Work
-// items are (query, key split, head half); splits write fp32 partials +
-// (max, sum) that attend_combine merges in a fixed order.  Every wait is
-// bounded.
+// Warp roles (256 threads): warp 0 TMEM owner, TMA loader of each work
+// item's raw query rows and MMA issuer (lane 0 issues through guarded
+// instructions); warps 1..3 gather the key rows with 16-byte cp.async into
+// the 128-byte swizzled layout (one 512-byte coalesced row segment per warp
+// instruction) from kernel entry on, each tile's key-validity mask travelling
+// with it; warps 4..7 normalise Q_hat in place, then run the softmax, two
+// threads per head (keys 0-31 / 32-63, D/2 output columns each), and stage
+// the output through shared memory for coalesced stores.  The roles only
+// meet at mbarriers, so the gathers of the next work item overlap the output
+// of the current one.  Work items are (query, key split, head half); splits
+// write fp32 partials + (max, sum) that attend_combine merges in a fixed
+// order.  Every wait is bounded and every role warp stays converged.
 #include <algorithm>
 
 #include "attend_common.cuh"
