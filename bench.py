@@ -498,7 +498,7 @@ def bench_fp4(csa, args, device, peaks):
 
     KC = 4 * wl.k  # FP4 over-selection before the bf16 re-ranking
     cand = torch.empty((wl.batch, 1, KC), dtype=torch.int32, device=device)
-    rws = torch.empty(csa.rescore_workspace_bytes(wl.batch, 1, KC, wl.k), dtype=torch.uint8, device=device)
+    rws = torch.empty(csa.rescore_workspace_bytes(wl.batch, 1, KC, wl.k, wl.d_I), dtype=torch.uint8, device=device)
 
     def step(mark):
         csa.csa_quantize_fp4(qI, packed=q4, scales=q4s)

@@ -164,10 +164,12 @@ int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long
  *   k_idx [batch][N][d_I] bf16         cand [batch][nq][kc] int32 (from csa_topk)
  *   idx   [batch][nq][k] int32
  * Requirements: k <= 8192; kc <= 2^19; H_I * d_I * 4 <= 200 KiB.  Workspace:
- * csa_rescore_workspace_bytes, 256-byte aligned (CSA_ERR_WORKSPACE otherwise).
+ * csa_rescore_workspace_bytes(batch, nq, kc, k, d_I) bytes, 256-byte aligned
+ * (CSA_ERR_WORKSPACE otherwise): candidate scores, chosen positions and a copy
+ * of the candidates' key rows (scored by the tensor-core indexer).
  * Causality is the candidates' (they come from a causal csa_topk).
  */
-size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k);
+size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I);
 int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx,
                      const int *cand, int kc, int batch, int nq, long long N, int H_I,
                      int d_I, int k, int *idx, void *workspace, size_t workspace_bytes,

@@ -46,7 +46,7 @@ def load() -> ctypes.CDLL:
         "csa_index_fp4": ([P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
         "csa_topk_workspace_bytes": ([i32, i32, i64, i32], sz),
         "csa_topk": ([P, P, i32, i32, i64, i32, i32, P, P, sz, P], i32),
-        "csa_rescore_workspace_bytes": ([i32, i32, i32, i32], sz),
+        "csa_rescore_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "csa_rescore_topk": ([P, P, P, P, i32, i32, i32, i64, i32, i32, i32, P, P, sz, P], i32),
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
         "csa_attend": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
@@ -170,8 +170,8 @@ def csa_topk(scores, q_pos, m: int, k: int, idx=None):
     return idx
 
 
-def rescore_workspace_bytes(batch: int, nq: int, kc: int, k: int) -> int:
-    return int(load().csa_rescore_workspace_bytes(batch, nq, kc, k))
+def rescore_workspace_bytes(batch: int, nq: int, kc: int, k: int, d_I: int) -> int:
+    return int(load().csa_rescore_workspace_bytes(batch, nq, kc, k, d_I))
 
 
 def csa_rescore_topk(q_idx, w, k_idx, cand, k: int, idx=None, workspace=None):
@@ -186,7 +186,7 @@ def csa_rescore_topk(q_idx, w, k_idx, cand, k: int, idx=None, workspace=None):
     kc = cand.shape[2]
     if idx is None:
         idx = torch.empty((batch, nq, k), dtype=torch.int32, device=q_idx.device)
-    nbytes = rescore_workspace_bytes(batch, nq, kc, k)
+    nbytes = rescore_workspace_bytes(batch, nq, kc, k, d_I)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q_idx.device)
     _check(L.csa_rescore_topk(_p(q_idx), _p(w), _p(k_idx), _p(cand), kc, batch, nq, N, H_I, d_I, k, _p(idx),

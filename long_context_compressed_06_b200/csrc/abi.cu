@@ -154,9 +154,9 @@ int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long
     return csa::launch_topk(scores, q_pos, batch, nq, N, m, k, idx, S(stream));
 }
 
-size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k) {
-    if (batch < 1 || nq < 1 || kc < 1 || k < 1) return 0;
-    return csa::rescore_workspace_bytes(batch, nq, kc, k);
+size_t csa_rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I) {
+    if (batch < 1 || nq < 1 || kc < 1 || k < 1 || d_I < 1) return 0;
+    return csa::rescore_workspace_bytes(batch, nq, kc, k, d_I);
 }
 
 int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
@@ -168,9 +168,11 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
     if (k > 8192 || kc > (1 << 19) || N > (1LL << 31) - 1 || !csa::rescore_supported(H_I, d_I))
         return CSA_ERR_UNSUPPORTED;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-        workspace_bytes < csa::rescore_workspace_bytes(batch, nq, kc, k))
+        workspace_bytes < csa::rescore_workspace_bytes(batch, nq, kc, k, d_I))
         return CSA_ERR_WORKSPACE;
-    return csa::launch_rescore_topk(q_idx, w, k_idx, cand, kc, batch, nq, N, H_I, d_I, k, idx, workspace,
+    csa::DevCtx ctx;
+    if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
+    return csa::launch_rescore_topk(q_idx, w, k_idx, cand, kc, batch, nq, N, H_I, d_I, k, idx, workspace, ctx,
                                     S(stream));
 }
 

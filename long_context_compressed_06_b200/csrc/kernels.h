@@ -30,11 +30,16 @@ size_t topk_workspace_bytes(int batch, int nq, long long N, int k);
 int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k,
                 int *idx, cudaStream_t st);
 
-size_t rescore_workspace_bytes(int batch, int nq, int kc, int k);
+size_t rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I);
 bool rescore_supported(int H_I, int d_I);
 int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
                         int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *ws,
-                        cudaStream_t st);
+                        const DevCtx &ctx, cudaStream_t st);
+
+bool index_tc_supported(int H_I, int d_I);
+int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
+                    int nq, long long N, int H_I, int d_I, int m, float *scores, const DevCtx &ctx,
+                    cudaStream_t st);
 
 // Attention: dense selects the HCA key set of the first n_vis(t) entries;
 // otherwise the k selected entries idx (may be null when k == 0).

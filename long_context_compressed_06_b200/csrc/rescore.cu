@@ -10,9 +10,12 @@
 // operands, fp32 arithmetic), and the k best candidates are kept:
 //   S_c[j] = sum_h w_h * max(0, q_I[h] . K_I[cand[j]])    (cand[j] < 0 -> -inf)
 //   idx    = cand[ top-k of S_c ]   (ascending entry order, -1 padded)
-// Three launches: candidate scoring (thread per candidate, query in shared
-// memory), the top-k selector over the kc candidate scores, and the map from
-// candidate positions back to entry indices.
+// When the tensor-core indexer takes the shape, the candidate key rows are
+// gathered into a contiguous buffer and scored by it (each query is its own
+// sequence of kc entries, all visible), invalid slots are set to -inf, the
+// top-k selector runs over the kc scores and the chosen positions are mapped
+// back to entry indices.  Otherwise a CUDA-core kernel scores the candidates
+// in place (thread per candidate, query in shared memory).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -83,23 +86,72 @@ __global__ void remap_kernel(const int *__restrict__ cand, const int *__restrict
     idx[t] = (l >= 0 && l < kc) ? cand[bq * kc + l] : -1;
 }
 
+// gathered[bq][j][:] = k_idx[b][cand[bq][j]][:] (zeros for invalid slots); pos[bq] = kc - 1
+__global__ void gather_kernel(const uint16_t *__restrict__ k_idx, const int *__restrict__ cand, int kc, int nq,
+                              long long N, int d_I, long long n16, uint16_t *__restrict__ gathered,
+                              int *__restrict__ pos) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // 16-byte unit
+    if (t >= n16) return;
+    const int upr = d_I / 8;  // 16-byte units per row
+    const long long row = t / upr;  // bq * kc + j
+    const int u = (int)(t - row * upr);
+    const long long bq = row / kc;
+    const int c = cand[row];
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (c >= 0 && c < N) v = ldg16(k_idx + ((size_t)(bq / nq) * N + c) * d_I + u * 8);
+    *reinterpret_cast<uint4 *>(gathered + (size_t)row * d_I + u * 8) = v;
+    if (row - bq * kc == 0 && u == 0) pos[bq] = kc - 1;
+}
+
+// scores of invalid candidate slots -> -inf
+__global__ void mask_kernel(const int *__restrict__ cand, long long n, long long N, float *__restrict__ sc) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n) return;
+    const int c = cand[t];
+    if (c < 0 || c >= N) sc[t] = -INFINITY;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-size_t rescore_workspace_bytes(int batch, int nq, int kc, int k) {
+// [scores fp32 nbq x kc][chosen positions int nbq x k][gathered keys bf16 nbq x kc x d_I][positions int nbq]
+size_t rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I) {
     const size_t nbq = (size_t)batch * nq;
-    return align256(nbq * kc * sizeof(float)) + align256(nbq * k * sizeof(int));
+    return align256(nbq * kc * sizeof(float)) + align256(nbq * k * sizeof(int)) +
+           align256(nbq * kc * (size_t)d_I * 2) + align256(nbq * sizeof(int));
 }
 
 bool rescore_supported(int H_I, int d_I) { return (size_t)H_I * d_I * 4 + (size_t)H_I * 4 <= 200 * 1024; }
 
 int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
                         int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *ws,
-                        cudaStream_t st) {
+                        const DevCtx &ctx, cudaStream_t st) {
     const long long nbq = (long long)batch * nq;
-    float *sc = reinterpret_cast<float *>(ws);
-    int *local = reinterpret_cast<int *>(reinterpret_cast<char *>(ws) + align256((size_t)nbq * kc * sizeof(float)));
+    char *wsb = reinterpret_cast<char *>(ws);
+    float *sc = reinterpret_cast<float *>(wsb);
+    wsb += align256((size_t)nbq * kc * sizeof(float));
+    int *local = reinterpret_cast<int *>(wsb);
+    wsb += align256((size_t)nbq * k * sizeof(int));
+    uint16_t *gathered = reinterpret_cast<uint16_t *>(wsb);
+    wsb += align256((size_t)nbq * kc * (size_t)d_I * 2);
+    int *pos = reinterpret_cast<int *>(wsb);
+    if (index_tc_supported(H_I, d_I)) {
+        const long long n16 = nbq * kc * (d_I / 8);
+        gather_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(k_idx, cand, kc, nq, N, d_I, n16, gathered, pos);
+        if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+        // every (sequence, query) is one sequence of kc entries with its query at position kc - 1 (m = 1)
+        int rc = launch_index_tc(q_idx, w, gathered, pos, (int)nbq, 1, kc, H_I, d_I, 1, sc, ctx, st);
+        if (rc != CSA_OK) return rc;
+        const long long n = nbq * kc;
+        mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cand, n, N, sc);
+        if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+        rc = launch_topk(sc, nullptr, batch, nq, kc, 1, k, local, st);
+        if (rc != CSA_OK) return rc;
+        const long long nk = nbq * k;
+        remap_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, st>>>(cand, local, kc, k, nk, idx);
+        return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    }
     const size_t smem = ((size_t)H_I * d_I + H_I) * sizeof(float);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -94,8 +94,8 @@ def test_topk_validation(lib):
 def test_rescore_validation_and_workspace(lib):
     f = lib.csa_rescore_topk
     ws = ctypes.c_void_p(0x40000)          # 256-byte aligned
-    need = lib.csa_rescore_workspace_bytes(4, 1, 4096, 1024)
-    assert need >= 4 * 4096 * 4 + 4 * 1024 * 4
+    need = lib.csa_rescore_workspace_bytes(4, 1, 4096, 1024, 128)
+    assert need >= 4 * 4096 * 4 + 4 * 1024 * 4 + 4 * 4096 * 128 * 2
     args = (A16, A16, A16, A16, 4096, 4, 1, 262144, 64, 128, 1024, A16b)
     assert f(NULL, *args[1:], ws, need, NULL) == csa.CSA_ERR_INVALID                    # q_idx
     assert f(*args[:3], NULL, *args[4:], ws, need, NULL) == csa.CSA_ERR_INVALID        # cand
