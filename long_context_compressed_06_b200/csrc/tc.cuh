@@ -136,87 +136,7 @@ CSA_DEVINL void tmem_ld16(uint32_t taddr, float v[16]) {
 
 CSA_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-CSA_DEVINL void tmem_st16(uint32_t taddr, const float v[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-          "r"(__float_as_uint(v[15]))
-        : "memory");
-}
-
 CSA_DEVINL void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// ---------------------------------------------------------------- gathered rows
-// Four rows (y0..y3) x one 128-byte box column (x) of a 2D tensor map into
-// four consecutive 128-byte rows of shared memory (box height 1).
-CSA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y0, int y1, int y2,
-                            int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
-}
-
-// ---------------------------------------------------------------- cluster (DSMEM)
-CSA_DEVINL uint32_t map_peer(uint32_t local_smem, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
-    return r;
-}
-
-CSA_DEVINL void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-
-// arrive (release, cluster scope) on an mbarrier of another CTA of the cluster
-CSA_DEVINL void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-// Non-blocking probe (test_wait): the phases polled here are completed by
-// arrivals from the peer CTA, so the waiter spins instead of parking in
-// try_wait's suspended state.
-CSA_DEVINL bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// bounded wait with cluster-scope acquire (for data a peer CTA wrote)
-CSA_DEVINL bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const DevCtx &ctx, volatile int *abort) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (abort && *abort) return false;
-        if (global_timer_ns() - t0 > ctx.budget_ns) {
-            record_status(ctx.status, CSA_ERR_TIMEOUT);
-            if (abort) *abort = 1;
-            return false;
-        }
-    }
-}
-
-CSA_DEVINL void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Instruction descriptor for P.V: A = P (K-major), B = V read MN-major.
-__host__ __device__ constexpr uint32_t idesc_f16_bmn(int n, bool bf16) {
-    return idesc_f16(n, bf16) | (1u << 16);
-}
 
 }  // namespace tc
 
