@@ -181,6 +181,9 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  * a sliding window of raw stream-A rows (techniques map rows "Grouped-query
  * attention" and "Sliding-window attention"; "DeepSeek v4" Figure 3 text).
  *   q_hat_h = RMSNorm(q_h) (eps, q_gain [D] or NULL = unit gain)
+ *   sinks   [H] fp32 or NULL: a learnable per-head sink logit that joins each
+ *             head's softmax denominator with no value row (techniques map,
+ *             "Learnable attention sink"); NULL = no sink
  *   J       = { kv[b][j] : j in idx[b][q], 0 <= j < N }
  *             U { stream-A row of position u : max(0, t-W+1) <= u <= t }
  *   out_h   = sum_{x in J} softmax(scale * q_hat_h . x) * x
@@ -196,7 +199,7 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, k + W).
  */
 size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
-int csa_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                long long win_rows, int W,
                const int *q_pos, int batch, int nq, int H, int D, float scale, float eps,
@@ -209,7 +212,7 @@ int csa_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long 
  * compresses every m' >> m tokens and keeps attention dense).
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, N + W).
  */
-int hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
+int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
                const int *q_pos,
                int batch, int nq, int H, int D, float scale, float eps,
@@ -240,7 +243,7 @@ int hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long 
  * race on it, so serialise them.
  */
 #define CSA_ATTEND_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
-int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                        const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                        long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
                        float scale, float eps, uint16_t *out, void *stream);

@@ -49,9 +49,10 @@ def load() -> ctypes.CDLL:
         "csa_rescore_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "csa_rescore_topk": ([P, P, P, P, i32, i32, i32, i64, i32, i32, i32, P, P, sz, P], i32),
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
-        "csa_attend": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
-        "hca_attend": ([P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
-        "csa_attend_noalloc": ([P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
+        "csa_attend": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
+                       i32),
+        "hca_attend": ([P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_attend_noalloc": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
                                i32),
         "csa_sync_status": ([P], i32),
         "csa_set_wait_budget_ns": ([ctypes.c_ulonglong], None),
@@ -207,10 +208,18 @@ def _workspace(nbytes: int, device, workspace):
     return workspace, workspace.numel() * workspace.element_size()
 
 
+def _sinks(sinks, H):
+    if sinks is not None:
+        _need(sinks, torch.float32, "sinks", 1)
+        if sinks.shape[0] != H:
+            raise ValueError("sinks must hold one logit per head (%d), got %d" % (H, sinks.shape[0]))
+    return _p(sinks)
+
+
 def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0):
+               workspace=None, win_pos0: int = 0, sinks=None):
     """q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] (bf16, stream-A rows of positions
-    win_pos0..) -> out [b][nq][H][D] bf16."""
+    win_pos0..) -> out [b][nq][H][D] bf16.  sinks: optional per-head sink logits [H] fp32."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
     _need(kv, torch.bfloat16, "kv", 3)
@@ -222,13 +231,14 @@ def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, 
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
-    _check(L.csa_attend(_p(q), _p(q_gain), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W, _p(q_pos),
+    _check(L.csa_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
+                        _p(q_pos),
                         batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend")
     return out
 
 
 def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0):
+               workspace=None, win_pos0: int = 0, sinks=None):
     """Dense attention over every visible entry of kv [b][N][D] plus the window."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
@@ -240,13 +250,14 @@ def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
-    _check(L.hca_attend(_p(q), _p(q_gain), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos), batch, nq, H,
+    _check(L.hca_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos),
+                        batch, nq, H,
                         D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend")
     return out
 
 
 def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-                       win_pos0: int = 0):
+                       win_pos0: int = 0, sinks=None):
     """csa_attend without a caller workspace: the library's own fixed device
     scratch is used (for callers that cannot allocate; see include/csa.h)."""
     L = load()
@@ -259,7 +270,8 @@ def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float 
     N, rows, k = kv.shape[1], win.shape[1], idx.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
+    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0),
+                                rows, W,
                                 _p(q_pos), batch, nq, H, D, float(scale), float(eps), _p(out), _stream()),
            "csa_attend_noalloc")
     return out

@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(AttendArgs a) {
         acc.z = fmaf(w, o.z, acc.z);
         acc.w = fmaf(w, o.w, acc.w);
     }
+    // the head's sink logit (natural units; the partials are in log2 units)
+    if (a.sinks) L += exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - M);
     const float inv = L > 0.f ? 1.0f / L : 0.f;
     uint16_t *dst = a.out + ((size_t)bq * a.H + h) * a.D + i;
     *reinterpret_cast<uint2 *>(dst) =
@@ -77,13 +79,13 @@ size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_key
     return ws_bytes_for(n_bq, H, D, splits);
 }
 
-int launch_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N, int m,
+int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
                   size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
     AttendArgs a = {};
-    a.q = q; a.q_gain = q_gain; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
+    a.q = q; a.q_gain = q_gain; a.sinks = sinks; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
     a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
     a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
     if (a.n_bq == 0) return CSA_OK;

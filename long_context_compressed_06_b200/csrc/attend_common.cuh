@@ -9,6 +9,7 @@ namespace csa {
 struct AttendArgs {
     const uint16_t *q;      // [n_bq][H][D]
     const float *q_gain;    // [D] or null
+    const float *sinks;     // [H] per-head sink logits (natural units) or null
     const uint16_t *kv;     // [batch][N][D]
     long long N;
     int m;                  // compression ratio (dense key set only)

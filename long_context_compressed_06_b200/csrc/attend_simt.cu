@@ -104,7 +104,9 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendArgs a) {
         const int h = head[hh];
         if (h >= a.H) continue;
         if (a.splits == 1) {
-            const float inv = l[hh] > 0.f ? 1.0f / l[hh] : 0.f;
+            // the head's sink logit joins the denominator (natural units -> log2 units)
+            const float L = l[hh] + (a.sinks ? exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - mrun[hh]) : 0.f);
+            const float inv = L > 0.f ? 1.0f / L : 0.f;
             float f[DPL];
 #pragma unroll
             for (int i = 0; i < DPL; ++i) f[i] = o[hh][i] * inv;

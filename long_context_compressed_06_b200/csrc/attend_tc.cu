@@ -583,7 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!warp_wait(smem_u32(s.oready + (gl & 1)), (uint32_t)((gl >> 1) & 1), p.ctx, s.abort_flag)) break;
                 tc::fence_after_sync();
             }
-            const float inv = a.splits == 1 ? (l > 0.f ? 1.0f / l : 0.f) : 1.0f;
+            // one split: normalise here, the head's sink logit (natural units ->
+            // log2 units) joining the denominator; several: the merge does it
+            const float L = l + ((a.sinks && h < a.H) ? exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - m_run) : 0.f);
+            const float inv = a.splits == 1 ? (L > 0.f ? 1.0f / L : 0.f) : 1.0f;
             uint8_t *stg = s.p;
             for (int c = 0; c < D; c += 64) {
                 float v[32];

@@ -36,9 +36,9 @@ def lib():
         L.orc_n_visible.restype = i64
         L.orc_index.argtypes = [P, P, P, P, i32, i32, i64, i32, i32, i32, P]
         L.orc_topk.argtypes = [P, P, i32, i32, i64, i32, i32, P]
-        L.orc_attend.argtypes = [P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
+        L.orc_attend.argtypes = [P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
                                  f64, f64, P]
-        L.orc_hca_attend.argtypes = [P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
+        L.orc_hca_attend.argtypes = [P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
                                      f64, f64, P]
         L.orc_e2m1_decode.argtypes = [ctypes.c_uint]
         L.orc_e2m1_decode.restype = f64
@@ -132,7 +132,7 @@ def topk(scores, q_pos, m, k):
     return out
 
 
-def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0):
+def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None):
     """CSA attention: q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] holding stream-A
     positions win_pos0.. -> float64 [b][nq][H][D]."""
     q, pq = _c(q, np.uint16)
@@ -146,12 +146,13 @@ def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0):
     k = idx.shape[2]
     rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
-    lib().orc_attend(pq, pg, pkv, N, pidx, k, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
+    s_, ps_ = _opt(sinks, np.float32)
+    lib().orc_attend(pq, pg, ps_, pkv, N, pidx, k, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
                      float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 
-def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0):
+def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None):
     """HCA attention over all visible entries + window -> float64 [b][nq][H][D]."""
     q, pq = _c(q, np.uint16)
     kv, pkv = _c(kv, np.uint16)
@@ -162,7 +163,8 @@ def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0
     N = kv.shape[1]
     rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
-    lib().orc_hca_attend(pq, pg, pkv, N, m, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
+    s_, ps_ = _opt(sinks, np.float32)
+    lib().orc_hca_attend(pq, pg, ps_, pkv, N, m, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
                          float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
     return out
 

@@ -290,8 +290,8 @@ void orc_topk(const double *scores, const int *q_pos, int batch, int nq, long lo
  * Keys and values are the same rows (one KV head).  Window rows are raw
  * stream-A rows (no RMSNorm); overlap with compressed entries is kept.
  */
-static void attend_one(const uint16_t *q, const float *q_gain, int H, int D, double scale,
-                       double eps, const uint16_t *const *rows, long long nrows, double *out)
+static void attend_one(const uint16_t *q, const float *q_gain, const float *sinks, int H, int D,
+                       double scale, double eps, const uint16_t *const *rows, long long nrows, double *out)
 {
     double *qh = (double *)malloc(sizeof(double) * (size_t)D);
     double *z = (double *)malloc(sizeof(double) * (size_t)(nrows > 0 ? nrows : 1));
@@ -313,14 +313,18 @@ static void attend_one(const uint16_t *q, const float *q_gain, int H, int D, dou
             z[j] = scale * dot;
             if (z[j] > mx) mx = z[j];
         }
-        double den = 0.0;
+        /* learnable sink ([DSv4-MAP] "Learnable attention sink"): one more
+         * logit per head in the softmax denominator, with no value row */
+        const double sink = sinks ? (double)sinks[h] : -INFINITY;
+        if (sink > mx) mx = sink;
+        double den = sinks && isfinite(mx) ? exp(sink - mx) : 0.0;
         for (long long j = 0; j < nrows; ++j) {
             z[j] = exp(z[j] - mx);
             den += z[j];
         }
         double *o = out + (size_t)h * D;
         for (int c = 0; c < D; ++c) o[c] = 0.0;
-        for (long long j = 0; j < nrows; ++j) {
+        for (long long j = 0; j < nrows && den > 0.0; ++j) {
             const double p = z[j] / den;
             for (int c = 0; c < D; ++c) o[c] += p * bf16_bits_to_double(rows[j][c]);
         }
@@ -347,7 +351,7 @@ static long long window_rows(const uint16_t *win, long long win_pos0, long long 
 /* CSA: key list = selected compressed entries (idx != -1 and 0 <= idx < N)
  * plus the sliding window.  q [batch][nq][H][D], kv [batch][N][D],
  * idx [batch][nq][k], win [batch][win_rows][D], out [batch][nq][H][D]. */
-void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+void orc_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                 const int *idx, int k, const uint16_t *win, long long win_pos0, long long win_rows, int W,
                 const int *q_pos, int batch, int nq, int H, int D, double scale, double eps,
                 double *out)
@@ -365,7 +369,7 @@ void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long
             rows[n++] = kv + ((size_t)b * N + j) * D;
         }
         n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
-        attend_one(q + (size_t)bq * H * D, q_gain, H, D, scale, eps, rows, n,
+        attend_one(q + (size_t)bq * H * D, q_gain, sinks, H, D, scale, eps, rows, n,
                    out + (size_t)bq * H * D);
         free(rows);
     }
@@ -374,7 +378,7 @@ void orc_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long
 /* HCA: dense attention over every visible compressed entry (j < n_vis(t))
  * plus the sliding window; no indexer ([DSv4-KR] hybrid-attention section:
  * HCA compresses every m' >> m tokens and keeps attention dense). */
-void orc_hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, long long N,
+void orc_hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                     int m, const uint16_t *win, long long win_pos0, long long win_rows, int W,
                     const int *q_pos,
                     int batch, int nq, int H, int D, double scale, double eps, double *out)
@@ -389,7 +393,7 @@ void orc_hca_attend(const uint16_t *q, const float *q_gain, const uint16_t *kv, 
         long long n = 0;
         for (long long j = 0; j < nv; ++j) rows[n++] = kv + ((size_t)b * N + j) * D;
         n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
-        attend_one(q + (size_t)bq * H * D, q_gain, H, D, scale, eps, rows, n,
+        attend_one(q + (size_t)bq * H * D, q_gain, sinks, H, D, scale, eps, rows, n,
                    out + (size_t)bq * H * D);
         free(rows);
     }

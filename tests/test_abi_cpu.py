@@ -109,15 +109,16 @@ def test_rescore_validation_and_workspace(lib):
 
 def test_attend_validation_and_workspace(lib):
     f = lib.csa_attend
-    args = dict(q=A16, g=NULL, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048, W=16, pos=A16, b=1, nq=1, H=8,
+    args = dict(q=A16, g=NULL, sk=NULL, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048, W=16, pos=A16, b=1, nq=1, H=8,
                 D=64, scale=0.125, eps=1e-6, out=A16b)
 
     def call(ws=NULL, wsb=0, **kw):
         a = dict(args, **kw)
-        return f(a["q"], a["g"], a["kv"], a["N"], a["idx"], a["k"], a["win"], a["p0"], a["T"], a["W"], a["pos"],
+        return f(a["q"], a["g"], a["sk"], a["kv"], a["N"], a["idx"], a["k"], a["win"], a["p0"], a["T"], a["W"], a["pos"],
                  a["b"], a["nq"], a["H"], a["D"], a["scale"], a["eps"], a["out"], ws, wsb, NULL)
 
     assert call(q=NULL) == csa.CSA_ERR_INVALID
+    assert call(sk=ctypes.c_void_p(0x10002)) == csa.CSA_ERR_INVALID    # sinks not 4-byte aligned
     assert call(W=0) == csa.CSA_ERR_INVALID
     assert call(p0=-1) == csa.CSA_ERR_INVALID
     assert call(T=0) == csa.CSA_ERR_INVALID
@@ -128,7 +129,7 @@ def test_attend_validation_and_workspace(lib):
     assert call(ws=A16, wsb=need - 1, k=1024) == csa.CSA_ERR_WORKSPACE
     assert call(ws=MIS, wsb=need, k=1024) == csa.CSA_ERR_WORKSPACE
     h = lib.hca_attend
-    assert h(A16, NULL, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b, NULL, 0,
+    assert h(A16, NULL, NULL, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b, NULL, 0,
              NULL) == csa.CSA_ERR_INVALID    # m
     # workspace sizing is monotone in the key count and batch
     assert lib.csa_attend_workspace_bytes(8, 1, 128, 512, 1152) >= lib.csa_attend_workspace_bytes(1, 1, 128, 512, 1152)

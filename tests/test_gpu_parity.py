@@ -213,6 +213,48 @@ def test_csa_attend_parity_large(cuda, batch, nq, H, D, N, T, k, Wn, m):
     assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
 
 
+@pytest.mark.parametrize("batch,nq,H,D,N,T,k,Wn,m,ts", [
+    (8, 1, 128, 512, 4096, 16384, 1024, 128, 4, [16383] * 8),      # key splits + merge
+    (1, 3, 128, 256, 300, 1200, 64, 16, 4, [1199, 700, 5]),        # one split per query
+    (2, 1, 40, 128, 97, 400, 33, 7, 4, [399, 13]),                 # ragged heads
+])
+def test_csa_attend_sinks_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts):
+    """Per-head sink logits in the softmax denominator (techniques map,
+    "Learnable attention sink"), against the oracle on the same selection."""
+    q = seeded((batch, nq, H, D), 64)
+    kv = seeded((batch, N, D), 65)
+    win = seeded((batch, T, D), 66)
+    qp = positions(batch, nq, ts)
+    idx = _random_selection(batch, nq, k, ts, m, N, 67)
+    sinks = (seeded((H,), 68, "uniform") * 6.0 - 3.0).contiguous()
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale, sinks=sinks)
+    ref = oracle.attend(bits(q), bits(kv), idx, bits(win), qp.cpu().numpy(), Wn, scale,
+                        sinks=sinks.cpu().numpy())
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+    # a sink of -inf is no sink at all
+    plain = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale)
+    none = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale,
+                           sinks=torch.full((H,), float("-inf"), device=DEV))
+    assert torch.equal(plain, none)
+
+
+def test_hca_attend_sinks_parity(cuda):
+    batch, H, D, N, m, Wn = 4, 128, 512, 700, 128, 128
+    T = N * m
+    q = seeded((batch, 1, H, D), 71)
+    kv = seeded((batch, N, D), 72)
+    win = seeded((batch, Wn, D), 73)
+    qp = positions(batch, 1, [T - 1, T - 1, 300 * 128 + 5, 64])
+    sinks = (seeded((H,), 74, "uniform") * 6.0 - 3.0).contiguous()
+    out = cuda.hca_attend(q, kv, m, win, qp, Wn, D ** -0.5, win_pos0=T - Wn, sinks=sinks)
+    ref = oracle.hca_attend(bits(q), bits(kv), m, bits(win), qp.cpu().numpy(), Wn, D ** -0.5, win_pos0=T - Wn,
+                            sinks=sinks.cpu().numpy())
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
 def test_attend_running_max_rescale(cuda):
     """Entries whose norms grow along the key order (logit scale 0.01 -> 5) push
     the running max up by more than 2^8 after the first tiles (the O rescale

@@ -312,6 +312,35 @@ def test_attend_query_rmsnorm_makes_query_scale_irrelevant():
     np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
 
 
+def test_attend_sink_single_key_is_a_sigmoid():
+    """One all-ones key and an all-ones query: the key's logit is
+    a = scale * D / sqrt(1 + eps), and with a sink logit c the key keeps the
+    weight e^a / (e^a + e^c) = sigmoid(a - c) -- a closed form."""
+    H, D, eps = 3, 16, 1e-6
+    q = bf16_bits(np.ones((1, 1, H, D)))
+    win = bf16_bits(np.ones((1, 8, D)))
+    idx = np.full((1, 1, 2), -1, np.int32)
+    scale = 1.0 / D
+    a = scale * D / math.sqrt(1.0 + eps)
+    sinks = np.array([-2.0, 0.5, 3.0], np.float32)
+    out = oracle.attend(q, win, idx, win, np.array([[5]], np.int32), W=1, scale=scale, eps=eps, sinks=sinks)
+    for h in range(H):
+        want = 1.0 / (1.0 + math.exp(float(sinks[h]) - a))
+        np.testing.assert_allclose(out[0, 0, h], np.full(D, want), rtol=1e-12)
+
+
+def test_attend_sink_at_minus_infinity_is_no_sink_and_a_huge_sink_silences():
+    r = rng(16)
+    q, kv, win = _attn_inputs(r)
+    idx = np.array([[[2, 7, -1, 11]]], np.int32)
+    pos = np.array([[33]], np.int32)
+    base = oracle.attend(q, kv, idx, win, pos, W=6, scale=0.2)
+    none = oracle.attend(q, kv, idx, win, pos, W=6, scale=0.2, sinks=np.full(4, -np.inf, np.float32))
+    assert np.array_equal(base, none)
+    loud = oracle.attend(q, kv, idx, win, pos, W=6, scale=0.2, sinks=np.full(4, 1e4, np.float32))
+    assert np.abs(loud).max() == 0.0
+
+
 def test_hca_equals_csa_with_every_visible_entry():
     r = rng(15)
     m, N, T, W = 4, 12, 48, 5
