@@ -79,7 +79,9 @@ int csa_version(void);
  *   gain    [d] fp32 or NULL
  *   out     [batch][floor(T/m)][d] bf16
  * Requirements: batch >= 1, T >= m >= 1, d % 8 == 0, 8 <= d <= 1024, m <= 256
- * (m > 16 or 24*m*d > 96 KiB additionally needs d % 64 == 0).
+ * (m > 16 or 24*m*d > 96 KiB additionally needs d % 64 == 0, and the pooling
+ * weights of one channel slice must fit in shared memory -- e.g. m <= 128 at
+ * d = 512; CSA_ERR_UNSUPPORTED otherwise).
  */
 int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
                  int batch, long long T, int d, int m,
@@ -91,13 +93,14 @@ int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
  * Lightning Indexer": per-head weight times ReLU(q . K), summed over heads).
  *   S[b][q][s] = sum_h w[b][q][h] * max(0, q_idx[b][q][h] . k_idx[b][s])   for s < n_vis(q_pos[b][q])
  *   S[b][q][s] = -inf                                                      otherwise
- * bf16 operands on the tensor cores, fp32 accumulation and epilogue.
+ * bf16 operands on the tensor cores (d_I in {32, 64, 128, 256}; other sizes on
+ * CUDA cores), fp32 accumulation and epilogue.
  *
  *   q_idx  [batch][nq][H_I][d_I] bf16     w [batch][nq][H_I] fp32
  *   k_idx  [batch][N][d_I] bf16           q_pos [batch][nq] int32 (0 <= t)
  *   scores [batch][nq][N] fp32 (output)
- * Requirements: d_I in {16, 32, 64, 128, 256}; 1 <= H_I <= 256 and
- * H_I % 16 == 0 or H_I < 16 (padded internally); m >= 1; N >= 1.
+ * Requirements: d_I % 16 == 0, 16 <= d_I <= 256; 1 <= H_I <= 256 (padded to a
+ * multiple of 16 internally); m >= 1; N >= 1.
  */
 int csa_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx,
               const int *q_pos, int batch, int nq, long long N, int H_I, int d_I,
@@ -121,10 +124,12 @@ int csa_quantize_fp4(const uint16_t *x, long long rows, int d,
 /*
  * csa_index_fp4 -- csa_index on FP4 operands (layouts of csa_quantize_fp4):
  * the score is the same formula on the dequantised values e2m1 * e4m3, with
- * exact products and fp32 accumulation.
+ * exact products and fp32 accumulation.  d_I in {64, 128, 256} with k4s
+ * aligned to d_I/16 bytes runs on the tensor cores (exact f16 dequantisation);
+ * other shapes on CUDA cores.
  *   q4 [batch][nq][H_I][d_I/2]   q4s [batch][nq][H_I][d_I/16]   w [batch][nq][H_I] fp32
  *   k4 [batch][N][d_I/2]         k4s [batch][N][d_I/16]         scores [batch][nq][N] fp32
- * Requirements: as csa_index (d_I % 64 == 0 for the packed path).
+ * Requirements: as csa_index.
  */
 int csa_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w,
                   const uint8_t *k4, const uint8_t *k4s, const int *q_pos,
