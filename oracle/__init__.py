@@ -31,6 +31,7 @@ def lib():
         L.orc_num_threads.restype = i32
         L.orc_set_num_threads.argtypes = [i32]
         L.orc_compress.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, f64, i64, i64, P]
+        L.orc_compress_dynamic.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, f64, i64, i64, P]
         L.orc_rmsnorm_bf16.argtypes = [P, i64, i32, f64, P, P]
         L.orc_n_visible.argtypes = [i64, i32, i64]
         L.orc_n_visible.restype = i64
@@ -95,6 +96,30 @@ def compress(A, B, logits, m, apply_rmsnorm=True, gain=None, eps=1e-6, i0=0, ni=
     out = np.empty((batch, ni, d), np.float64)
     lib().orc_compress(pA, pB, pL, batch, T, d, m, int(bool(apply_rmsnorm)), pg, float(eps),
                        int(i0), int(ni), out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def compress_dynamic(A, B, Za, Zb, bias, m, apply_rmsnorm=True, gain=None, eps=1e-6, i0=0, ni=None):
+    """Compressed entries [i0, i0+ni) with input-dependent weights: A, B, Za, Zb [batch][T][d] bf16 bits
+    (Za / Zb may be None = 0), bias [2m][d] -> float64 [batch][ni][d]."""
+    A, pA = _c(A, np.uint16)
+    B, pB = _c(B, np.uint16)
+    batch, T, d = A.shape
+    assert B.shape == A.shape
+    za, pza = _opt(Za, np.uint16)
+    zb, pzb = _opt(Zb, np.uint16)
+    assert za is None or za.shape == A.shape
+    assert zb is None or zb.shape == A.shape
+    L, pL = _c(bias, np.float32)
+    assert L.shape == (2 * m, d)
+    g, pg = _opt(gain, np.float32)
+    N = T // m
+    if ni is None:
+        ni = N - i0
+    assert 0 <= i0 and i0 + ni <= N
+    out = np.empty((batch, ni, d), np.float64)
+    lib().orc_compress_dynamic(pA, pB, pza, pzb, pL, batch, T, d, m, int(bool(apply_rmsnorm)), pg, float(eps),
+                               int(i0), int(ni), out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 

@@ -163,6 +163,79 @@ void orc_compress(const uint16_t *A, const uint16_t *B, const float *logits,
     free(w_first);
 }
 
+/*
+ * Compressed entries with input-dependent compression weights
+ * [DSv4-KR "압축된 Key-Value entry"]: from the hidden states come, per token,
+ * the two KV streams C_a (here A), C_b (here B) and two compression-weight
+ * rows Z_a, Z_b; entry i combines its 2m rows with the weights plus the
+ * learnable positional biases B_a, B_b under a per-channel softmax over the
+ * 2m elements, and for i = 0 the previous block is padded with Z_b = -inf,
+ * C_b = 0.  For channel c:
+ *   l_j = Zb[(i-1)m + j][c] + bias[j][c]      (j = 0..m-1, previous block, i >= 1)
+ *   l_j = Za[i*m + j-m][c]  + bias[j][c]      (j = m..2m-1, own block)
+ *   C_i[c] = sum_j softmax_j(l)[j] * x_j[c]   (x_j the matching B or A row)
+ * then the optional RMSNorm of orc_compress.
+ * Readings: bias rows 0..m-1 are B_b and rows m..2m-1 are B_a (the order
+ * orc_compress uses); Z_a and Z_b are bf16 like the streams; a NULL Za or Zb
+ * contributes 0, so with both NULL this is orc_compress.
+ *
+ * Computes entries [i0, i0 + ni) of every sequence; out is [batch][ni][d].
+ */
+void orc_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Za, const uint16_t *Zb,
+                          const float *bias, int batch, long long T, int d, int m,
+                          int apply_rmsnorm, const float *gain, double eps,
+                          long long i0, long long ni, double *out)
+{
+    const long long total = (long long)batch * ni;
+#pragma omp parallel for schedule(static)
+    for (long long job = 0; job < total; ++job) {
+        const long long b = job / ni;
+        const long long i = i0 + job % ni;
+        const size_t seq = (size_t)b * T * d;
+        double *o = out + (size_t)job * d;
+        double *l = (double *)malloc(sizeof(double) * 2 * (size_t)m);
+        double *x = (double *)malloc(sizeof(double) * 2 * (size_t)m);
+
+        for (int c = 0; c < d; ++c) {
+            /* the 2m (logit, value) pairs of this channel; entry 0 has only its own block */
+            int n = 0;
+            if (i > 0) {
+                for (int j = 0; j < m; ++j) {
+                    const size_t row = seq + (size_t)((i - 1) * m + j) * d + c;
+                    l[n] = (Zb ? bf16_bits_to_double(Zb[row]) : 0.0) + (double)bias[(size_t)j * d + c];
+                    x[n] = bf16_bits_to_double(B[row]);
+                    ++n;
+                }
+            }
+            for (int j = 0; j < m; ++j) {
+                const size_t row = seq + (size_t)(i * m + j) * d + c;
+                l[n] = (Za ? bf16_bits_to_double(Za[row]) : 0.0) + (double)bias[(size_t)(m + j) * d + c];
+                x[n] = bf16_bits_to_double(A[row]);
+                ++n;
+            }
+            double mx = -INFINITY;
+            for (int j = 0; j < n; ++j)
+                if (l[j] > mx) mx = l[j];
+            double den = 0.0, acc = 0.0;
+            for (int j = 0; j < n; ++j) {
+                const double e = exp(l[j] - mx);
+                den += e;
+                acc += e * x[j];
+            }
+            o[c] = acc / den;
+        }
+        if (apply_rmsnorm) {
+            double ms = 0.0;
+            for (int c = 0; c < d; ++c) ms += o[c] * o[c];
+            ms /= d;
+            const double r = 1.0 / sqrt(ms + eps);
+            for (int c = 0; c < d; ++c) o[c] = o[c] * r * (gain ? (double)gain[c] : 1.0);
+        }
+        free(l);
+        free(x);
+    }
+}
+
 /* RMSNorm of `rows` vectors of length d (used for the query heads).
  * [DSv4-AN]: an RMSNorm is applied to each query head before core attention. */
 void orc_rmsnorm_bf16(const uint16_t *x, long long rows, int d, double eps,

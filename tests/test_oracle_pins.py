@@ -128,6 +128,99 @@ def test_compress_entry_range_matches_full():
     np.testing.assert_array_equal(part, full[:, 7:12])
 
 
+# input-dependent compression weights Z_a, Z_b ("DeepSeek v4", compressed Key-Value entry)
+def test_compress_dynamic_m1_is_a_sigmoid_blend():
+    """m = 1: entry i >= 1 pools B[i-1] and A[i] with weight sigma(l_A - l_B) on A,
+    l_A = Za[i] + bias[1], l_B = Zb[i-1] + bias[0]; entry 0 is A[0]."""
+    r = rng(40)
+    T, d = 9, 16
+    A, B, Za, Zb = (bf16_bits(r.standard_normal((2, T, d))) for _ in range(4))
+    bias = r.standard_normal((2, d)).astype(np.float32)
+    out = oracle.compress_dynamic(A, B, Za, Zb, bias, 1, apply_rmsnorm=False)
+    Av, Bv, Zav, Zbv = bf16_val(A), bf16_val(B), bf16_val(Za), bf16_val(Zb)
+    bb = bias.astype(np.float64)
+    np.testing.assert_array_equal(out[:, 0], Av[:, 0])
+    for i in range(1, T):
+        s = 1.0 / (1.0 + np.exp(-((Zav[:, i] + bb[1]) - (Zbv[:, i - 1] + bb[0]))))
+        np.testing.assert_allclose(out[:, i], s * Av[:, i] + (1 - s) * Bv[:, i - 1], rtol=1e-12, atol=1e-14)
+
+
+def test_compress_dynamic_one_hot_z_selects_the_named_token():
+    """Channel c of entry i puts Z = +80 on row j = (i + c) mod 2m and 0 elsewhere:
+    the output is that row's token, B[(i-1)m + j] for j < m, A[im + j - m] otherwise
+    (entry 0 takes j in the A half)."""
+    r = rng(41)
+    m, T, d = 4, 42, 24
+    A = bf16_bits(r.standard_normal((1, T, d)))
+    B = bf16_bits(r.standard_normal((1, T, d)))
+    Za = np.zeros((1, T, d), np.float32)
+    Zb = np.zeros((1, T, d), np.float32)
+    N = T // m
+    want = np.empty((N, d))
+    Av, Bv = bf16_val(A)[0], bf16_val(B)[0]
+    for i in range(N):
+        for c in range(d):
+            j = (i + c) % (2 * m)
+            if i == 0 and j < m:
+                j += m
+            if j < m:
+                Zb[0, (i - 1) * m + j, c] = 80.0
+                want[i, c] = Bv[(i - 1) * m + j, c]
+            else:
+                Za[0, i * m + j - m, c] = 80.0
+                want[i, c] = Av[i * m + j - m, c]
+    bias = np.zeros((2 * m, d), np.float32)
+    out = oracle.compress_dynamic(A, B, bf16_bits(Za), bf16_bits(Zb), bias, m, apply_rmsnorm=False)[0]
+    np.testing.assert_allclose(out, want, rtol=1e-13, atol=1e-30)
+
+
+def test_compress_dynamic_entry0_ignores_the_previous_block():
+    """Z_b = +80 on every token: entry 0 (no previous block) is the mean of its A
+    rows; every later entry is the mean of its m previous-block B rows."""
+    r = rng(42)
+    m, T, d = 3, 21, 16
+    A = bf16_bits(r.standard_normal((2, T, d)))
+    B = bf16_bits(r.standard_normal((2, T, d)))
+    Zb = bf16_bits(np.full((2, T, d), 80.0))
+    bias = np.zeros((2 * m, d), np.float32)
+    out = oracle.compress_dynamic(A, B, None, Zb, bias, m, apply_rmsnorm=False)
+    Av, Bv = bf16_val(A), bf16_val(B)
+    np.testing.assert_allclose(out[:, 0], Av[:, 0:m].mean(1), rtol=1e-13, atol=1e-15)
+    for i in range(1, T // m):
+        np.testing.assert_allclose(out[:, i], Bv[:, (i - 1) * m:i * m].mean(1), rtol=1e-12, atol=1e-15)
+
+
+def test_compress_dynamic_without_z_is_the_static_compress():
+    r = rng(43)
+    m, T, d = 4, 50, 32
+    A = bf16_bits(r.standard_normal((2, T, d)))
+    B = bf16_bits(r.standard_normal((2, T, d)))
+    bias = r.standard_normal((2 * m, d)).astype(np.float32)
+    g = r.uniform(0.5, 2.0, d).astype(np.float32)
+    static = oracle.compress(A, B, bias, m, apply_rmsnorm=True, gain=g)
+    zeros = np.zeros(A.shape, np.uint16)
+    np.testing.assert_allclose(oracle.compress_dynamic(A, B, None, None, bias, m, gain=g), static, rtol=1e-12)
+    np.testing.assert_allclose(oracle.compress_dynamic(A, B, zeros, zeros, bias, m, gain=g), static, rtol=1e-12)
+
+
+def test_compress_dynamic_shift_invariance_and_entry_range():
+    """A constant added to every Z value leaves the softmax unchanged; a sub-range
+    of entries equals the same rows of the full result."""
+    r = rng(44)
+    m, T, d = 4, 60, 16
+    A = bf16_bits(r.standard_normal((2, T, d)))
+    B = bf16_bits(r.standard_normal((2, T, d)))
+    # Z on a 1/8 grid in [-3, 3]: +2 stays exact in bf16
+    Za = np.clip(np.round(r.standard_normal((2, T, d)) * 8) / 8, -3, 3)
+    Zb = np.clip(np.round(r.standard_normal((2, T, d)) * 8) / 8, -3, 3)
+    bias = r.standard_normal((2 * m, d)).astype(np.float32)
+    base = oracle.compress_dynamic(A, B, bf16_bits(Za), bf16_bits(Zb), bias, m)
+    shifted = oracle.compress_dynamic(A, B, bf16_bits(Za + 2), bf16_bits(Zb + 2), bias, m)
+    np.testing.assert_allclose(shifted, base, rtol=1e-12, atol=1e-14)
+    part = oracle.compress_dynamic(A, B, bf16_bits(Za), bf16_bits(Zb), bias, m, i0=6, ni=5)
+    np.testing.assert_array_equal(part, base[:, 6:11])
+
+
 # ----------------------------------------------------------------------------
 # indexer
 # ----------------------------------------------------------------------------
