@@ -445,6 +445,24 @@ def bench_compress(csa, args, device, peaks, wl: W.Workload, seqs: int = 2):
             "hbm_gbs": round(byts / t / 1e9, 1), "frac": round(byts / t / 1e9 / peaks["hbm_gbs"], 4)}
 
 
+def bench_compress_dynamic(csa, args, device, peaks, wl: W.Workload):
+    """Cache build with input-dependent compression weights (tokens/s), one sequence of the workload's
+    length: streams A, B and weight rows Z_a, Z_b read once, entries written once."""
+    L = W.pool_logits(wl, device)
+    A, B, Za, Zb = (torch.empty((1, wl.T, wl.D), dtype=torch.bfloat16, device=device) for _ in range(4))
+    A[0] = W.stream(wl, "A", 0, device)
+    B[0] = W.stream(wl, "B", 0, device)
+    Za[0] = W.compression_weights(wl, "Za", 0, device)
+    Zb[0] = W.compression_weights(wl, "Zb", 0, device)
+    out = torch.empty((1, wl.N, wl.D), dtype=torch.bfloat16, device=device)
+    steps = max(2, min(args.steps, 5))
+    tot, _ = Timer(device).run(lambda mark: csa.csa_compress_dynamic(A, B, Za, Zb, L, wl.m, out=out), steps, 2)
+    byts = 4 * wl.T * wl.D * 2 + wl.N * wl.D * 2
+    t = tot / steps
+    return {"workload": wl.name + "_compress_dynamic", "tokens_per_s": wl.T / t, "ms": round(t * 1e3, 3),
+            "hbm_gbs": round(byts / t / 1e9, 1), "frac": round(byts / t / 1e9 / peaks["hbm_gbs"], 4)}
+
+
 def bench_hca(csa, args, device, peaks):
     wl = W.HCA_DECODE
     L = W.pool_logits(wl, device)
@@ -615,7 +633,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress"],
+    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress", "compress_dynamic"],
                     help="run one of the other workloads alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -633,7 +651,9 @@ def main():
         run_one = {"prefill": lambda: bench_prefill(csa, args, device, peaks),
                    "hca": lambda: bench_hca(csa, args, device, peaks),
                    "fp4": lambda: bench_fp4(csa, args, device, peaks),
-                   "compress": lambda: bench_compress(csa, args, device, peaks, W.HCA_DECODE)}[args.only]
+                   "compress": lambda: bench_compress(csa, args, device, peaks, W.HCA_DECODE),
+                   "compress_dynamic": lambda: bench_compress_dynamic(csa, args, device, peaks, W.CSA_DECODE),
+                   }[args.only]
         res = run_one()
         rc = csa.csa_sync_status()
         if rc != 0:
@@ -658,6 +678,9 @@ def main():
         torch.cuda.empty_cache()
         extra["compress_m4_128k"] = bench_compress(csa, args, device, peaks, W.CSA_DECODE)
         extra["compress_m128_1m"] = bench_compress(csa, args, device, peaks, W.HCA_DECODE)
+        torch.cuda.empty_cache()
+        extra["compress_dynamic_m4_128k"] = bench_compress_dynamic(csa, args, device, peaks, W.CSA_DECODE)
+        extra["compress_dynamic_m128_1m"] = bench_compress_dynamic(csa, args, device, peaks, W.HCA_DECODE)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, threads = oracle_decode_sample(W.CSA_DECODE)

@@ -89,6 +89,42 @@ int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
                  uint16_t *out, void *stream);
 
 /*
+ * csa_compress_dynamic -- compressed KV entries with input-dependent
+ * compression weights ("DeepSeek v4" -> "Compressed Sparse Attention" ->
+ * compressed Key-Value entry: from the hidden states, per token, the KV rows
+ * C_a, C_b and the compression weights Z_a, Z_b; learnable positional biases
+ * B_a, B_b; a softmax over the 2m elements of each entry; Z_b = -inf and
+ * C_b = 0 before the first block).
+ *
+ * For every sequence b, entry i in [i0, i0 + ni) and channel c:
+ *   l_j  = Zb[(i-1)m + j][c] + bias[j][c]        j = 0..m-1    (previous block, i >= 1)
+ *   l_j  = Za[im + j-m][c]   + bias[j][c]        j = m..2m-1   (own block)
+ *   C_i[c] = sum_j softmax_j(l)[j] * x_j[c]      x_j = B[(i-1)m + j][c], resp. A[im + j-m][c]
+ * Entry 0 has no previous block: its softmax runs over the A half only.  A
+ * NULL Za or Zb counts as all zeros (with both NULL the result is
+ * csa_compress's with logits = bias).  If apply_rmsnorm != 0 each entry is
+ * then y[c] = C_i[c] / sqrt(mean_c(C_i^2) + eps) * gain[c] (gain NULL -> 1).
+ * Arithmetic in fp32 (online softmax); the result is rounded to bf16 once and
+ * written to out[b][i][:].  Rows of out outside [i0, i0 + ni) are untouched, so
+ * at decode time the newest entry (i0 = N - 1, ni = 1) is appended to a cache.
+ *
+ *   A, B      [batch][T][d] bf16     stream A (own block), stream B (previous block)
+ *   Za, Zb    [batch][T][d] bf16 or NULL   compression-weight rows of A and B
+ *   bias      [2m][d] fp32           rows 0..m-1: B's positional bias, m..2m-1: A's
+ *   gain      [d] fp32 or NULL
+ *   out       [batch][n_out][d] bf16, n_out >= i0 + ni
+ * Logits must be finite or -inf (an -inf logit drops its row; a channel with
+ * every logit -inf gives 0).  Requirements: batch >= 1, T >= m >= 1,
+ * d % 8 == 0, 8 <= d, 0 <= i0, 0 <= ni, (i0 + ni) * m <= T; A, B, Za, Zb,
+ * bias and out 16-byte aligned, gain 4-byte aligned (CSA_ERR_INVALID);
+ * d <= 2048 (CSA_ERR_UNSUPPORTED).
+ */
+int csa_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Za, const uint16_t *Zb,
+                         const float *bias, int batch, long long T, int d, int m,
+                         int apply_rmsnorm, const float *gain, float eps,
+                         long long i0, long long ni, uint16_t *out, long long n_out, void *stream);
+
+/*
  * csa_index -- lightning-indexer scores ("DeepSeek v4" -> "sparse selection
  * Lightning Indexer": per-head weight times ReLU(q . K), summed over heads).
  *   S[b][q][s] = sum_h w[b][q][h] * max(0, q_idx[b][q][h] . k_idx[b][s])   for s < n_vis(q_pos[b][q])

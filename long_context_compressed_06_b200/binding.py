@@ -41,6 +41,7 @@ def load() -> ctypes.CDLL:
         "csa_strerror": ([i32], ctypes.c_char_p),
         "csa_version": ([], i32),
         "csa_compress": ([P, P, P, i32, i64, i32, i32, i32, P, f32, P, P], i32),
+        "csa_compress_dynamic": ([P, P, P, P, P, i32, i64, i32, i32, i32, P, f32, i64, i64, P, i64, P], i32),
         "csa_index": ([P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
         "csa_quantize_fp4": ([P, i64, i32, P, P, P], i32),
         "csa_index_fp4": ([P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
@@ -111,6 +112,38 @@ def csa_compress(A, B, logits, m: int, apply_rmsnorm: bool = True, gain=None, ep
         out = torch.empty((batch, T // m, d), dtype=torch.bfloat16, device=A.device)
     _check(L.csa_compress(_p(A), _p(B), _p(logits), batch, T, d, m, int(bool(apply_rmsnorm)), _p(gain),
                           float(eps), _p(out), _stream()), "csa_compress")
+    return out
+
+
+def csa_compress_dynamic(A, B, Za, Zb, bias, m: int, apply_rmsnorm: bool = True, gain=None, eps: float = 1e-6,
+                         i0: int = 0, ni=None, out=None):
+    """Compressed entries [i0, i0+ni) with input-dependent weights.  A, B, Za, Zb [batch][T][d] bf16 (Za / Zb
+    may be None), bias [2m][d] fp32 -> out [batch][n_out][d] bf16 with rows i0..i0+ni-1 written (default: all
+    T//m entries into a new tensor; pass a cache as `out` to append entries)."""
+    L = load()
+    _need(A, torch.bfloat16, "A", 3)
+    _need(B, torch.bfloat16, "B", 3)
+    for z, name in ((Za, "Za"), (Zb, "Zb")):
+        if z is not None:
+            _need(z, torch.bfloat16, name, 3)
+            if z.shape != A.shape:
+                raise ValueError("shape mismatch: %s" % name)
+    _need(bias, torch.float32, "bias", 2)
+    batch, T, d = A.shape
+    if B.shape != A.shape or bias.shape != (2 * m, d):
+        raise ValueError("shape mismatch")
+    if gain is not None:
+        _need(gain, torch.float32, "gain", 1)
+    if ni is None:
+        ni = T // m - i0
+    if out is None:
+        out = torch.zeros((batch, T // m, d), dtype=torch.bfloat16, device=A.device)
+    _need(out, torch.bfloat16, "out", 3)
+    if out.shape[0] != batch or out.shape[2] != d:
+        raise ValueError("shape mismatch: out")
+    _check(L.csa_compress_dynamic(_p(A), _p(B), _p(Za), _p(Zb), _p(bias), batch, T, d, m,
+                                  int(bool(apply_rmsnorm)), _p(gain), float(eps), int(i0), int(ni), _p(out),
+                                  out.shape[1], _stream()), "csa_compress_dynamic")
     return out
 
 

@@ -108,6 +108,19 @@ int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits, int 
     return csa::launch_compress(A, B, logits, batch, T, d, m, apply_rmsnorm, gain, eps, out, S(stream));
 }
 
+int csa_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Za, const uint16_t *Zb,
+                         const float *bias, int batch, long long T, int d, int m, int apply_rmsnorm,
+                         const float *gain, float eps, long long i0, long long ni, uint16_t *out, long long n_out,
+                         void *stream) {
+    if (!al16(A) || !al16(B) || !al16(bias) || !al16(out)) return CSA_ERR_INVALID;
+    if ((Za && !al16(Za)) || (Zb && !al16(Zb)) || (gain && !al4(gain))) return CSA_ERR_INVALID;
+    if (batch < 1 || m < 1 || T < m || d < 8 || d % 8 != 0 || !(eps >= 0.f)) return CSA_ERR_INVALID;
+    if (i0 < 0 || ni < 0 || i0 + ni > T / m || n_out < i0 + ni) return CSA_ERR_INVALID;
+    if (d > 2048) return CSA_ERR_UNSUPPORTED;
+    return csa::launch_compress_dynamic(A, B, Za, Zb, bias, batch, T, d, m, apply_rmsnorm, gain, eps, i0, ni,
+                                        n_out, out, S(stream));
+}
+
 int csa_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
               int nq, long long N, int H_I, int d_I, int m, float *scores, void *stream) {
     if (!al16(q_idx) || !al4(w) || !al16(k_idx) || !al4(q_pos) || !al16(scores)) return CSA_ERR_INVALID;

@@ -14,6 +14,11 @@ int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, i
                     int d, int m, int apply_rmsnorm, const float *gain, float eps, uint16_t *out,
                     cudaStream_t st);
 
+int launch_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Za, const uint16_t *Zb,
+                            const float *bias, int batch, long long T, int d, int m, int apply_rmsnorm,
+                            const float *gain, float eps, long long i0, long long ni, long long n_out,
+                            uint16_t *out, cudaStream_t st);
+
 int launch_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos,
                  int batch, int nq, long long N, int H_I, int d_I, int m, float *scores,
                  const DevCtx &ctx, cudaStream_t st);

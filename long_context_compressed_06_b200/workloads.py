@@ -13,7 +13,8 @@ Distributions (the recipe; every tensor has its own seed ``seed*1000 + id``
 and, for per-sequence tensors, ``+ 100000*(b+1)``):
   * streams A, B, queries q, indexer queries q_I, indexer keys K_I and the
     directly drawn compressed KV rows: bf16 from N(0,1) (fp32 draw, RNE cast);
-  * pooling logits [2m][d]: fp32 N(0,1);
+  * pooling logits [2m][d] (the positional bias): fp32 N(0,1);
+  * input-dependent compression weights Z_a, Z_b [T][d]: bf16 from N(0,1);
   * indexer head weights w: fp32 U(0,1);
   * the FP4 workload scales ``key_outliers`` fixed indexer-key channels by 8
     (ceil(1% of 128) = 2 channels, chosen by a seeded permutation).
@@ -27,7 +28,7 @@ from typing import Optional
 import torch
 
 # tensor ids for seeding
-_ID_A, _ID_B, _ID_LOGITS, _ID_Q, _ID_QI, _ID_W, _ID_KI, _ID_KV, _ID_OUTLIER = range(1, 10)
+_ID_A, _ID_B, _ID_LOGITS, _ID_Q, _ID_QI, _ID_W, _ID_KI, _ID_KV, _ID_OUTLIER, _ID_ZA, _ID_ZB = range(1, 12)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -103,6 +104,12 @@ def uniform_f32(shape, seed: int, device="cpu") -> torch.Tensor:
 def stream(wl: Workload, which: str, b: int, device="cpu", T: Optional[int] = None) -> torch.Tensor:
     """Latent KV stream 'A' or 'B' of sequence b: [T][D] bf16."""
     tid = _ID_A if which == "A" else _ID_B
+    return normal_bf16((wl.T if T is None else T, wl.D), _seed(wl, tid, b), device)
+
+
+def compression_weights(wl: Workload, which: str, b: int, device="cpu", T: Optional[int] = None) -> torch.Tensor:
+    """Compression-weight rows 'Za' or 'Zb' of sequence b: [T][D] bf16."""
+    tid = _ID_ZA if which == "Za" else _ID_ZB
     return normal_bf16((wl.T if T is None else T, wl.D), _seed(wl, tid, b), device)
 
 

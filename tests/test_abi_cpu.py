@@ -28,7 +28,7 @@ def declared_functions():
 
 def test_header_declares_the_pipeline_calls():
     names = declared_functions()
-    for n in ("csa_compress", "csa_index", "csa_index_fp4", "csa_quantize_fp4", "csa_topk", "csa_attend",
+    for n in ("csa_compress", "csa_compress_dynamic", "csa_index", "csa_index_fp4", "csa_quantize_fp4", "csa_topk", "csa_attend",
               "hca_attend", "csa_sync_status", "csa_strerror"):
         assert n in names
 
@@ -61,6 +61,34 @@ def test_compress_validation(lib):
     assert f(A16, A16, A16, 1, 64, 64, 4, 1, NULL, -1.0, A16b, NULL) == csa.CSA_ERR_INVALID   # eps
     assert f(A16, A16, A16, 1, 4096, 2048, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
     assert f(A16, A16, A16, 1, 4096, 64, 512, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
+
+
+def test_compress_dynamic_validation(lib):
+    f = lib.csa_compress_dynamic
+    # (A, B, Za, Zb, bias, batch, T, d, m, rms, gain, eps, i0, ni, out, n_out, stream)
+    ok = dict(A=A16, B=A16, Za=A16, Zb=NULL, bias=A16, batch=1, T=64, d=64, m=4, rms=1, gain=NULL, eps=1e-6,
+              i0=0, ni=16, out=A16b, n_out=16)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["A"], a["B"], a["Za"], a["Zb"], a["bias"], a["batch"], a["T"], a["d"], a["m"], a["rms"],
+                 a["gain"], a["eps"], a["i0"], a["ni"], a["out"], a["n_out"], NULL)
+
+    assert call(A=NULL) == csa.CSA_ERR_INVALID
+    assert call(bias=NULL) == csa.CSA_ERR_INVALID
+    assert call(Za=MIS) == csa.CSA_ERR_INVALID
+    assert call(Zb=MIS) == csa.CSA_ERR_INVALID
+    assert call(bias=MIS) == csa.CSA_ERR_INVALID
+    assert call(gain=ctypes.c_void_p(0x10002)) == csa.CSA_ERR_INVALID
+    assert call(d=60) == csa.CSA_ERR_INVALID                   # d % 8
+    assert call(T=3) == csa.CSA_ERR_INVALID                    # T < m
+    assert call(batch=0) == csa.CSA_ERR_INVALID
+    assert call(eps=-1.0) == csa.CSA_ERR_INVALID
+    assert call(i0=-1, ni=1) == csa.CSA_ERR_INVALID
+    assert call(ni=-1) == csa.CSA_ERR_INVALID
+    assert call(i0=10, ni=7) == csa.CSA_ERR_INVALID            # (i0 + ni) * m > T
+    assert call(i0=0, ni=16, n_out=15) == csa.CSA_ERR_INVALID  # out too short
+    assert call(T=4096, d=2056, ni=1, n_out=1) == csa.CSA_ERR_UNSUPPORTED
 
 
 def test_index_validation(lib):

@@ -71,6 +71,104 @@ def test_compress_parity(cuda, batch, T, d, m, rms, use_gain):
     assert np.all(err <= 8e-3 * np.abs(ref).max(-1)), err.max()
 
 
+# ----------------------------------------------------------------------------- compress, input-dependent weights
+def _dyn_inputs(batch, T, d, m, z_scale=1.0, seed=60):
+    A = seeded((batch, T, d), seed)
+    B = seeded((batch, T, d), seed + 1)
+    Za = (seeded((batch, T, d), seed + 2).float() * z_scale).to(torch.bfloat16)
+    Zb = (seeded((batch, T, d), seed + 3).float() * z_scale).to(torch.bfloat16)
+    bias = torch.randn((2 * m, d), generator=torch.Generator(DEV).manual_seed(seed + 4), device=DEV)
+    return A, B, Za, Zb, bias
+
+
+def _check_rows(got, ref):
+    assert got.shape == ref.shape
+    err = np.abs(got - ref).max(-1)
+    assert np.all(err <= 8e-3 * np.abs(ref).max(-1)), err.max()
+
+
+@pytest.mark.parametrize("batch,T,d,m,rms,use_gain,za,zb,z_scale", [
+    (1, 2048, 64, 4, True, False, True, True, 1.0),       # tiny workload shape
+    (2, 1037, 512, 4, True, True, True, True, 1.0),       # V4 width (warp reduction), ragged T
+    (2, 777, 64, 3, False, False, True, False, 1.0),      # odd m, no norm, Zb absent
+    (1, 4 * 128 + 77, 512, 128, True, False, True, True, 1.0),  # HCA ratio, ragged tail
+    (2, 300, 128, 16, True, True, False, True, 8.0),      # 16 threads per entry, Za absent, wide logits
+    (3, 5, 64, 4, True, False, True, True, 1.0),          # N = 1 (entry 0 only)
+    (1, 90, 48, 5, True, True, True, True, 30.0),         # 6 threads per entry (252-thread blocks), sharp softmax
+    (1, 40, 2048, 2, True, False, True, True, 1.0),       # 256 threads per entry
+    (2, 333, 8, 7, True, False, True, True, 4.0),         # one thread per entry
+])
+def test_compress_dynamic_parity(cuda, batch, T, d, m, rms, use_gain, za, zb, z_scale):
+    A, B, Za, Zb, bias = _dyn_inputs(batch, T, d, m, z_scale)
+    Za = Za if za else None
+    Zb = Zb if zb else None
+    gain = (seeded((d,), 64, "uniform") + 0.5) if use_gain else None
+    out = cuda.csa_compress_dynamic(A, B, Za, Zb, bias, m, rms, gain, 1e-6)
+    ref = oracle.compress_dynamic(bits(A), bits(B), None if Za is None else bits(Za), None if Zb is None else bits(Zb),
+                                  bias.cpu().numpy(), m, rms, None if gain is None else gain.cpu().numpy(), 1e-6)
+    _check_rows(f64(out), ref)
+    again = cuda.csa_compress_dynamic(A, B, Za, Zb, bias, m, rms, gain, 1e-6)
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))   # fixed reduction order
+
+
+def test_compress_dynamic_minus_inf_bias_rows_and_no_z(cuda):
+    """-inf bias drops a row for the channels it covers; with no Z the call is
+    csa_compress on the same logits."""
+    batch, T, d, m = 2, 203, 128, 4
+    A, B, Za, Zb, bias = _dyn_inputs(batch, T, d, m, seed=70)
+    bias[0, : d // 2] = float("-inf")
+    bias[2 * m - 1, d // 4:] = float("-inf")
+    out = cuda.csa_compress_dynamic(A, B, Za, Zb, bias, m)
+    ref = oracle.compress_dynamic(bits(A), bits(B), bits(Za), bits(Zb), bias.cpu().numpy(), m)
+    _check_rows(f64(out), ref)
+    bias2 = torch.randn((2 * m, d), generator=torch.Generator(DEV).manual_seed(71), device=DEV)
+    plain = cuda.csa_compress_dynamic(A, B, None, None, bias2, m)
+    _check_rows(f64(plain), oracle.compress(bits(A), bits(B), bias2.cpu().numpy(), m))
+
+
+def test_compress_dynamic_appends_into_a_cache(cuda):
+    """Entries [i0, i0+ni) land in rows i0.. of a longer cache; every other row
+    keeps its bits (decode-time compression, one entry every m tokens)."""
+    batch, T, d, m = 3, 96, 512, 4
+    A, B, Za, Zb, bias = _dyn_inputs(batch, T, d, m, seed=80)
+    n_out = 40
+    cache = torch.full((batch, n_out, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    before = cache.clone()
+    for i0, ni in ((0, 1), (5, 3), (T // m - 1, 1)):
+        cuda.csa_compress_dynamic(A, B, Za, Zb, bias, m, i0=i0, ni=ni, out=cache)
+        ref = oracle.compress_dynamic(bits(A), bits(B), bits(Za), bits(Zb), bias.cpu().numpy(), m, i0=i0, ni=ni)
+        _check_rows(f64(cache[:, i0:i0 + ni]), ref)
+    written = torch.zeros(n_out, dtype=torch.bool)
+    written[[0, 5, 6, 7, T // m - 1]] = True
+    assert torch.equal(cache[:, ~written].view(torch.int16), before[:, ~written].view(torch.int16))
+
+
+def test_compress_dynamic_decode_128k_cache_sampled(cuda):
+    """The 128K decode cache (8 x 131072 tokens, d = 512, m = 4) built in one
+    launch, checked on sampled entries: entry i depends only on token rows
+    (i-1)m .. (i+1)m-1, so the oracle computes it from those rows alone."""
+    wl = W.CSA_DECODE
+    bsz, T, d, m = wl.batch, wl.T, wl.D, wl.m
+    A = torch.stack([W.stream(wl, "A", b, DEV) for b in range(bsz)])
+    B = torch.stack([W.stream(wl, "B", b, DEV) for b in range(bsz)])
+    Za = torch.stack([W.compression_weights(wl, "Za", b, DEV) for b in range(bsz)])
+    Zb = torch.stack([W.compression_weights(wl, "Zb", b, DEV) for b in range(bsz)])
+    bias = W.pool_logits(wl, DEV)
+    out = cuda.csa_compress_dynamic(A, B, Za, Zb, bias, m)
+    N = T // m
+    rs = np.random.default_rng(81)
+    bn = bias.cpu().numpy()
+    for b in range(bsz):
+        ents = np.unique(np.concatenate([[0, 1, N - 1], rs.integers(2, N - 1, 29)]))
+        for i in ents:
+            lo = max(0, (i - 1) * m)
+            rows = slice(lo, (i + 1) * m)
+            sub = [bits(t[b:b + 1, rows]) for t in (A, B, Za, Zb)]
+            ref = oracle.compress_dynamic(*sub, bn, m, i0=0 if i == 0 else 1, ni=1)
+            _check_rows(f64(out[b:b + 1, i:i + 1]), ref)
+    del A, B, Za, Zb
+
+
 # ----------------------------------------------------------------------------- index
 def _index_case(batch, nq, H_I, d_I, N, m, ts, seed=20):
     qI = seeded((batch, nq, H_I, d_I), seed)
