@@ -29,7 +29,7 @@
 namespace csa {
 namespace {
 
-constexpr int kRows = 4;                         // rows whose loads are in flight together
+constexpr int kRows = 8;                         // rows whose loads are in flight together
 constexpr int kMaxThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
