@@ -38,9 +38,10 @@ def lib():
         L.orc_index.argtypes = [P, P, P, P, i32, i32, i64, i32, i32, i32, P]
         L.orc_topk.argtypes = [P, P, i32, i32, i64, i32, i32, P]
         L.orc_attend.argtypes = [P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
-                                 f64, f64, P]
+                                 f64, f64, i32, P, P, P]
         L.orc_hca_attend.argtypes = [P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
-                                     f64, f64, P]
+                                     f64, f64, i32, P, P, P]
+        L.orc_rope.argtypes = [P, i64, i32, i32, P, P, P, i32, P]
         L.orc_e2m1_decode.argtypes = [ctypes.c_uint]
         L.orc_e2m1_decode.restype = f64
         L.orc_e4m3_decode.argtypes = [ctypes.c_uint]
@@ -157,9 +158,37 @@ def topk(scores, q_pos, m, k):
     return out
 
 
-def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None):
+def _rope_tables(rope, q_pos):
+    """rope = (cos, sin) tables [positions][rope_dim/2] or None -> (rope_dim, arrays, pointers)."""
+    if rope is None:
+        return 0, (None, None), (None, None)
+    c, pc = _c(rope[0], np.float32)
+    s, ps = _c(rope[1], np.float32)
+    assert c.ndim == 2 and c.shape == s.shape
+    assert int(np.max(q_pos)) < c.shape[0] and int(np.min(q_pos)) >= 0
+    return 2 * c.shape[1], (c, s), (pc, ps)
+
+
+def rope(x, pos, cos, sin, inverse=False):
+    """Partial RoPE of float64 rows x [..., width] at integer positions pos [...] with tables
+    cos / sin [positions][rope_dim/2] (the trailing rope_dim channels rotate) -> float64."""
+    x, px = _c(x, np.float64)
+    width = x.shape[-1]
+    p, pp = _c(np.broadcast_to(pos, x.shape[:-1]), np.int32)
+    c, pc = _c(cos, np.float32)
+    s, ps = _c(sin, np.float32)
+    assert c.shape == s.shape and 2 * c.shape[1] <= width
+    assert int(p.max()) < c.shape[0] and int(p.min()) >= 0
+    out = np.empty(x.shape, np.float64)
+    lib().orc_rope(px, x.size // width, width, 2 * c.shape[1], pp, pc, ps, int(bool(inverse)),
+                   out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None, rope=None):
     """CSA attention: q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] holding stream-A
-    positions win_pos0.. -> float64 [b][nq][H][D]."""
+    positions win_pos0.. -> float64 [b][nq][H][D].  rope = (cos, sin) applies partial RoPE to the
+    query heads and its conjugate to the outputs (keys arrive rotated)."""
     q, pq = _c(q, np.uint16)
     kv, pkv = _c(kv, np.uint16)
     idx, pidx = _c(idx, np.int32)
@@ -172,12 +201,13 @@ def attend(q, kv, idx, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, 
     rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
     s_, ps_ = _opt(sinks, np.float32)
+    rd, _keep, (pc, ps) = _rope_tables(rope, qp)
     lib().orc_attend(pq, pg, ps_, pkv, N, pidx, k, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
-                     float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
+                     float(scale), float(eps), rd, pc, ps, out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 
-def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None):
+def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0, sinks=None, rope=None):
     """HCA attention over all visible entries + window -> float64 [b][nq][H][D]."""
     q, pq = _c(q, np.uint16)
     kv, pkv = _c(kv, np.uint16)
@@ -189,8 +219,9 @@ def hca_attend(q, kv, m, win, q_pos, W, scale, eps=1e-6, q_gain=None, win_pos0=0
     rows = win.shape[1]
     out = np.empty(q.shape, np.float64)
     s_, ps_ = _opt(sinks, np.float32)
+    rd, _keep, (pc, ps) = _rope_tables(rope, qp)
     lib().orc_hca_attend(pq, pg, ps_, pkv, N, m, pwin, int(win_pos0), rows, W, pqp, batch, nq, H, D,
-                         float(scale), float(eps), out.ctypes.data_as(ctypes.c_void_p))
+                         float(scale), float(eps), rd, pc, ps, out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 

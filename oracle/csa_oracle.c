@@ -363,8 +363,56 @@ void orc_topk(const double *scores, const int *q_pos, int batch, int nq, long lo
  * Keys and values are the same rows (one KV head).  Window rows are raw
  * stream-A rows (no RMSNorm); overlap with compressed entries is kept.
  */
+/*
+ * Partial rotary position embedding ([DSv4-MAP] "Partial RoPE": only the
+ * trailing qk_rope_head_dim = 64 channels of each 512-channel head are
+ * rotated, the leading "nope" channels are left as they are; the rotated
+ * slice is x*cos + rotate_half(x)*sin, rotate_half taking the slice's two
+ * halves (x1, x2) to (-x2, x1)).  For a row x of `width` channels at
+ * position p, with n = width - rope_dim, r = rope_dim / 2 and
+ * c_i = cos_t[p][i], s_i = sin_t[p][i] (i < r):
+ *   y[n + i]     = x[n + i] * c_i - x[n + r + i] * s_i
+ *   y[n + r + i] = x[n + r + i] * c_i + x[n + i] * s_i
+ * (channel n+i is paired with n+r+i).  inverse != 0 rotates by the conjugate
+ * (s_i -> -s_i), which undoes the rotation ([DSv4-MAP] "Gated attention
+ * output": the attention output goes through a rope-conjugate rotation).
+ * Reading: the cos / sin tables [positions][r] are the caller's (their
+ * frequencies, YaRN scaling included, are not part of this step).
+ */
+static void rope_rotate(double *x, int width, int rope_dim, long long p, const float *cos_t,
+                        const float *sin_t, int inverse)
+{
+    const int r = rope_dim / 2, n = width - rope_dim;
+    for (int i = 0; i < r; ++i) {
+        const double c = (double)cos_t[(size_t)p * r + i];
+        const double sn = (double)sin_t[(size_t)p * r + i];
+        const double s = inverse ? -sn : sn;
+        const double x1 = x[n + i], x2 = x[n + r + i];
+        x[n + i] = x1 * c - x2 * s;
+        x[n + r + i] = x2 * c + x1 * s;
+    }
+}
+
+/* rows x [rows][width] (float64) at positions pos[rows] -> out [rows][width] */
+void orc_rope(const double *x, long long rows, int width, int rope_dim, const int *pos,
+              const float *cos_t, const float *sin_t, int inverse, double *out)
+{
+    for (long long i = 0; i < rows; ++i) {
+        memcpy(out + (size_t)i * width, x + (size_t)i * width, sizeof(double) * (size_t)width);
+        rope_rotate(out + (size_t)i * width, width, rope_dim, pos[i], cos_t, sin_t, inverse);
+    }
+}
+
+/*
+ * One query, all H heads.  With rope_dim > 0 the RMS-normalised query head is
+ * rotated at the query position t before the dot products, and each head's
+ * output is rotated back by the conjugate at t (keys and window rows arrive
+ * already rotated at their own positions: they are values too, K = V).
+ */
 static void attend_one(const uint16_t *q, const float *q_gain, const float *sinks, int H, int D,
-                       double scale, double eps, const uint16_t *const *rows, long long nrows, double *out)
+                       double scale, double eps, const uint16_t *const *rows, long long nrows,
+                       int rope_dim, const float *rope_cos, const float *rope_sin, long long t,
+                       double *out)
 {
     double *qh = (double *)malloc(sizeof(double) * (size_t)D);
     double *z = (double *)malloc(sizeof(double) * (size_t)(nrows > 0 ? nrows : 1));
@@ -378,6 +426,7 @@ static void attend_one(const uint16_t *q, const float *q_gain, const float *sink
         const double r = 1.0 / sqrt(ms + eps);
         for (int c = 0; c < D; ++c)
             qh[c] = bf16_bits_to_double(q[(size_t)h * D + c]) * r * (q_gain ? (double)q_gain[c] : 1.0);
+        if (rope_dim > 0) rope_rotate(qh, D, rope_dim, t, rope_cos, rope_sin, 0);
 
         double mx = -INFINITY;
         for (long long j = 0; j < nrows; ++j) {
@@ -401,6 +450,7 @@ static void attend_one(const uint16_t *q, const float *q_gain, const float *sink
             const double p = z[j] / den;
             for (int c = 0; c < D; ++c) o[c] += p * bf16_bits_to_double(rows[j][c]);
         }
+        if (rope_dim > 0) rope_rotate(o, D, rope_dim, t, rope_cos, rope_sin, 1);
     }
     free(qh);
     free(z);
@@ -427,7 +477,7 @@ static long long window_rows(const uint16_t *win, long long win_pos0, long long 
 void orc_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                 const int *idx, int k, const uint16_t *win, long long win_pos0, long long win_rows, int W,
                 const int *q_pos, int batch, int nq, int H, int D, double scale, double eps,
-                double *out)
+                int rope_dim, const float *rope_cos, const float *rope_sin, double *out)
 {
     const long long total = (long long)batch * nq;
 #pragma omp parallel for schedule(dynamic)
@@ -443,7 +493,7 @@ void orc_attend(const uint16_t *q, const float *q_gain, const float *sinks, cons
         }
         n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
         attend_one(q + (size_t)bq * H * D, q_gain, sinks, H, D, scale, eps, rows, n,
-                   out + (size_t)bq * H * D);
+                   rope_dim, rope_cos, rope_sin, t, out + (size_t)bq * H * D);
         free(rows);
     }
 }
@@ -454,7 +504,8 @@ void orc_attend(const uint16_t *q, const float *q_gain, const float *sinks, cons
 void orc_hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
                     int m, const uint16_t *win, long long win_pos0, long long win_rows, int W,
                     const int *q_pos,
-                    int batch, int nq, int H, int D, double scale, double eps, double *out)
+                    int batch, int nq, int H, int D, double scale, double eps,
+                    int rope_dim, const float *rope_cos, const float *rope_sin, double *out)
 {
     const long long total = (long long)batch * nq;
 #pragma omp parallel for schedule(dynamic)
@@ -467,7 +518,7 @@ void orc_hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, 
         for (long long j = 0; j < nv; ++j) rows[n++] = kv + ((size_t)b * N + j) * D;
         n += window_rows(win, win_pos0, win_rows, W, b, t, D, rows + n);
         attend_one(q + (size_t)bq * H * D, q_gain, sinks, H, D, scale, eps, rows, n,
-                   out + (size_t)bq * H * D);
+                   rope_dim, rope_cos, rope_sin, t, out + (size_t)bq * H * D);
         free(rows);
     }
 }

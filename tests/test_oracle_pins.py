@@ -434,6 +434,111 @@ def test_attend_sink_at_minus_infinity_is_no_sink_and_a_huge_sink_silences():
     assert np.abs(loud).max() == 0.0
 
 
+# partial RoPE ("DeepSeek-V4-Pro - Model techniques map", "Partial RoPE" and the
+# rope-conjugate rotation of the attention output)
+def _rope_tables(n_pos, r, seed=0, omega=None):
+    """cos / sin of angles p * omega_i for p < n_pos (omega drawn if not given)."""
+    om = rng(seed).uniform(0.01, 1.5, r) if omega is None else np.asarray(omega, np.float64)
+    ang = np.arange(n_pos)[:, None] * om[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def test_rope_hand_worked_example():
+    """width 6 = 2 unrotated + 4 rotated channels, r = 2; at position 1 the
+    angles are (pi/2, 0): rotate_half pairs channel 2 with 4 and 3 with 5, so
+    x = [5, 6, 1, 2, 3, 4] -> [5, 6, 1*0 - 3*1, 2, 3*0 + 1*1, 4] = [5, 6, -3, 2, 1, 4]
+    and the conjugate gives [5, 6, 3, 2, -1, 4]; position 0 (angle 0) is the identity."""
+    cos = np.array([[1, 1], [0, 1]], np.float32)
+    sin = np.array([[0, 0], [1, 0]], np.float32)
+    x = np.array([5, 6, 1, 2, 3, 4], np.float64)
+    np.testing.assert_array_equal(oracle.rope(x, 1, cos, sin), [5, 6, -3, 2, 1, 4])
+    np.testing.assert_array_equal(oracle.rope(x, 1, cos, sin, inverse=True), [5, 6, 3, 2, -1, 4])
+    np.testing.assert_array_equal(oracle.rope(x, 0, cos, sin), x)
+
+
+def test_rope_is_complex_multiplication_of_half_pairs():
+    """Independent route: the rotated slice equals (x1 + i x2) * exp(i theta)
+    computed with numpy complex arithmetic; the unrotated channels are kept."""
+    r_, width = 32, 96
+    cos, sin = _rope_tables(50, r_, seed=1)
+    x = rng(2).standard_normal((7, width))
+    pos = np.array([0, 1, 7, 13, 31, 48, 49], np.int32)
+    y = oracle.rope(x, pos, cos, sin)
+    n = width - 2 * r_
+    z = (x[:, n:n + r_] + 1j * x[:, n + r_:]) * (cos[pos].astype(np.float64) + 1j * sin[pos].astype(np.float64))
+    np.testing.assert_array_equal(y[:, :n], x[:, :n])
+    np.testing.assert_allclose(y[:, n:n + r_], z.real, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(y[:, n + r_:], z.imag, rtol=1e-13, atol=1e-14)
+
+
+def test_rope_preserves_norm_inverse_undoes_and_scores_see_relative_position():
+    r_, width = 16, 64
+    cos, sin = _rope_tables(64, r_, seed=3)
+    g = rng(4)
+    q, k = g.standard_normal(width), g.standard_normal(width)
+    y = oracle.rope(q, 9, cos, sin)
+    # fp32 tables: cos^2 + sin^2 = 1 to ~1e-7, so norm and inverse hold to that
+    assert abs(np.linalg.norm(y) - np.linalg.norm(q)) < 2e-7 * np.linalg.norm(q)
+    np.testing.assert_allclose(oracle.rope(y, 9, cos, sin, inverse=True), q, rtol=0, atol=4e-7 * np.abs(q).max())
+    # (R_t q) . (R_s k) depends on t - s only (angles p * omega); fp32 tables limit the agreement
+    d1 = oracle.rope(q, 20, cos, sin) @ oracle.rope(k, 5, cos, sin)
+    d2 = oracle.rope(q, 40, cos, sin) @ oracle.rope(k, 25, cos, sin)
+    assert abs(d1 - d2) < 1e-5 * (np.linalg.norm(q) * np.linalg.norm(k))
+
+
+def test_attend_rope_identity_tables_equal_no_rope():
+    r = rng(17)
+    q, kv, win = _attn_inputs(r, H=4, D=32)
+    idx = np.array([[[2, 7, -1, 11]]], np.int32)
+    pos = np.array([[33]], np.int32)
+    cos = np.ones((40, 8), np.float32)
+    sin = np.zeros((40, 8), np.float32)
+    base = oracle.attend(q, kv, idx, win, pos, W=6, scale=0.2)
+    np.testing.assert_array_equal(oracle.attend(q, kv, idx, win, pos, W=6, scale=0.2, rope=(cos, sin)), base)
+
+
+def test_attend_rope_single_key_is_its_conjugate_rotation():
+    """One key (the window row at t): weight 1, so the output is that row
+    rotated back by the conjugate at the query position."""
+    r = rng(18)
+    q, kv, win = _attn_inputs(r, H=3, D=32)
+    cos, sin = _rope_tables(40, 8, seed=5)
+    t = 17
+    idx = np.full((1, 1, 3), -1, np.int32)
+    out = oracle.attend(q, kv, idx, win, np.array([[t]], np.int32), W=1, scale=0.3, rope=(cos, sin))
+    x = bf16_val(win)[0, t]
+    n = 32 - 16
+    z = (x[n:n + 8] + 1j * x[n + 8:]) * (cos[t].astype(np.float64) - 1j * sin[t].astype(np.float64))
+    want = np.concatenate([x[:n], z.real, z.imag])
+    np.testing.assert_allclose(out[0, 0], np.broadcast_to(want, (3, 32)), rtol=1e-13, atol=1e-14)
+
+
+def test_attend_rope_output_sees_relative_positions_only():
+    """Angles that are multiples of pi/2 keep every rotation exact in bf16.
+    Keys rotated at their positions s_j and the query at t give the same output
+    as everything shifted by one position: logits and the conjugated values
+    depend on s_j - t only.  A missing or misplaced conjugate breaks this."""
+    H, D, r_ = 2, 16, 4
+    cos, sin = _rope_tables(64, r_, omega=[np.pi / 2, np.pi, 3 * np.pi / 2, np.pi / 2])
+    cos, sin = np.round(cos), np.round(sin)
+    g = rng(19)
+    q = bf16_bits(g.standard_normal((1, 1, H, D)))
+    raw = bf16_val(bf16_bits(g.standard_normal((30, D))))
+    s_pos = np.arange(30)
+
+    def run(shift):
+        rows = oracle.rope(raw, s_pos + shift, cos, sin)       # exact: entries are permuted / negated
+        win = bf16_bits(rows)[None]
+        t = 25 + shift
+        idx = np.full((1, 1, 2), -1, np.int32)
+        return oracle.attend(q, win, idx, win, np.array([[t]], np.int32), W=8, scale=0.5, win_pos0=shift,
+                             rope=(cos, sin))
+
+    a, b = run(0), run(1)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+    assert np.abs(a[..., D - 2 * r_:]).max() > 0.1   # the rotated channels carry signal
+
+
 def test_hca_equals_csa_with_every_visible_entry():
     r = rng(15)
     m, N, T, W = 4, 12, 48, 5
@@ -452,6 +557,10 @@ def test_hca_equals_csa_with_every_visible_entry():
     idx2[0, 0, :N] = idx2[0, 0, :N][::-1]
     np.testing.assert_allclose(oracle.attend(q, kv, idx2, win, pos, W, scale=0.25), csa,
                                rtol=1e-13, atol=1e-15)
+    # and with partial RoPE on both sides
+    rope = _rope_tables(T, 8, seed=6)
+    np.testing.assert_allclose(oracle.hca_attend(q, kv, m, win, pos, W, scale=0.25, rope=rope),
+                               oracle.attend(q, kv, idx, win, pos, W, scale=0.25, rope=rope), rtol=1e-13, atol=1e-15)
 
 
 # ----------------------------------------------------------------------------
