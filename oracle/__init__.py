@@ -42,6 +42,8 @@ def lib():
         L.orc_hca_attend.argtypes = [P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32,
                                      f64, f64, i32, P, P, P]
         L.orc_rope.argtypes = [P, i64, i32, i32, P, P, P, i32, P]
+        L.orc_quantize_fp8_kv.argtypes = [P, i64, i32, i32, P, P]
+        L.orc_dequantize_fp8_kv.argtypes = [P, P, i64, i32, i32, P]
         L.orc_e2m1_decode.argtypes = [ctypes.c_uint]
         L.orc_e2m1_decode.restype = f64
         L.orc_e4m3_decode.argtypes = [ctypes.c_uint]
@@ -261,6 +263,30 @@ def dequantize_fp4(packed, scales):
     rows = p.size // (d // 2)
     out = np.empty(p.shape[:-1] + (d,), np.float64)
     lib().orc_dequantize_fp4(pp, ps, rows, d, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def quantize_fp8_kv(x, block=128):
+    """KV rows [..., d] bf16 bits -> (e4m3 codes u8 [..., d], UE8M0 block exponents u8 [..., d/block])."""
+    x, px = _c(x, np.uint16)
+    d = x.shape[-1]
+    assert d % block == 0
+    rows = x.size // d
+    codes = np.empty(x.shape, np.uint8)
+    exps = np.empty(x.shape[:-1] + (d // block,), np.uint8)
+    lib().orc_quantize_fp8_kv(px, rows, d, block, codes.ctypes.data_as(ctypes.c_void_p),
+                              exps.ctypes.data_as(ctypes.c_void_p))
+    return codes, exps
+
+
+def dequantize_fp8_kv(codes, exps, block=128):
+    """(codes [..., d], exponents [..., d/block]) -> float64 [..., d] (each value exactly a bf16 number)."""
+    c, pc = _c(codes, np.uint8)
+    e, pe = _c(exps, np.uint8)
+    d = c.shape[-1]
+    assert e.shape == c.shape[:-1] + (d // block,)
+    out = np.empty(c.shape, np.float64)
+    lib().orc_dequantize_fp8_kv(pc, pe, c.size // d, d, block, out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 

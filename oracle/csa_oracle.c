@@ -682,3 +682,57 @@ int orc_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, const u
     free(qd);
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* 6. FP8 KV cache  [DSv4-MAP] list "inference quantization"            */
+/* ------------------------------------------------------------------ */
+/*
+ * The pages list "FP8 KV-cache quantization" and give no format.  Reading:
+ * each KV row (a compressed entry or a window row, d channels) is stored as
+ * e4m3 codes with one power-of-two scale per block of `block` channels, the
+ * scale kept as an unsigned 8-bit exponent (UE8M0: s = 2^(e - 127)).  s is the
+ * smallest power of two with absmax(block) / s <= 448 (the largest finite
+ * e4m3 magnitude); the codes are e4m3_RNE(x / s), the division by a power of
+ * two being exact; an all-zero block has e = 127 and zero codes.  With s a
+ * power of two and 3 mantissa bits per code, every dequantised value
+ * code * s is a bf16 number exactly, so attention over the FP8 cache is the
+ * attention of section 4 over those bf16 rows.
+ */
+void orc_quantize_fp8_kv(const uint16_t *x, long long rows, int d, int block, uint8_t *codes,
+                         uint8_t *exps)
+{
+    const int nblk = d / block;
+    for (long long r = 0; r < rows; ++r) {
+        for (int blk = 0; blk < nblk; ++blk) {
+            const uint16_t *xs = x + (size_t)r * d + (size_t)blk * block;
+            double amax = 0.0;
+            for (int j = 0; j < block; ++j) {
+                const double a = fabs(bf16_bits_to_double(xs[j]));
+                if (a > amax) amax = a;
+            }
+            int k = 0;  /* s = 2^k */
+            if (amax > 0.0) {
+                k = (int)ceil(log2(amax / 448.0));
+                while (ldexp(amax, -k) > 448.0) ++k;          /* guard the log2 rounding */
+                while (ldexp(amax, -(k - 1)) <= 448.0) --k;   /* smallest such k */
+                if (k < -127) k = -127;
+                if (k > 127) k = 127;
+            }
+            exps[(size_t)r * nblk + blk] = (uint8_t)(k + 127);
+            for (int j = 0; j < block; ++j)
+                codes[(size_t)r * d + (size_t)blk * block + j] =
+                    (uint8_t)orc_e4m3_encode((float)ldexp(bf16_bits_to_double(xs[j]), -k));
+        }
+    }
+}
+
+/* code * 2^(e - 127) per element -> float64 [rows][d] */
+void orc_dequantize_fp8_kv(const uint8_t *codes, const uint8_t *exps, long long rows, int d, int block,
+                           double *out)
+{
+    const int nblk = d / block;
+    for (long long r = 0; r < rows; ++r)
+        for (int j = 0; j < d; ++j)
+            out[(size_t)r * d + j] = ldexp(orc_e4m3_decode(codes[(size_t)r * d + j]),
+                                           (int)exps[(size_t)r * nblk + j / block] - 127);
+}

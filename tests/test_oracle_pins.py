@@ -655,6 +655,68 @@ def test_fp4_zero_block_and_packing_order():
     assert packed[0, 8] == (0x7 | (0xD << 4))
 
 
+# FP8 KV cache ("DeepSeek-V4-Pro - Model techniques map", inference quantization)
+def _fp8_rows(seed, rows=6, d=256):
+    r = rng(seed)
+    x = r.standard_normal((rows, d)) * np.exp(r.uniform(-6, 6, (rows, 1)))   # rows of very different sizes
+    x[1, 128:] = 0.0                                                          # an all-zero block
+    x[2, :128] = 0.0
+    x[2, 5] = 2.0 ** -20                                                      # a tiny block
+    return bf16_bits(x)
+
+
+def test_fp8_kv_codes_match_torch_float8_with_the_tightest_power_of_two_scale():
+    """Independent route: the scale from frexp (smallest 2^k >= absmax/448) and
+    the codes from torch's float8_e4m3fn cast of x / 2^k (round-half-even)."""
+    x = _fp8_rows(30)
+    codes, exps = oracle.quantize_fp8_kv(x, 128)
+    xv = bf16_val(x)
+    for r_ in range(x.shape[0]):
+        for blk in range(2):
+            seg = xv[r_, blk * 128:(blk + 1) * 128]
+            amax = np.abs(seg).max()
+            if amax == 0.0:
+                assert exps[r_, blk] == 127 and not codes[r_, blk * 128:(blk + 1) * 128].any()
+                continue
+            mant, ex = np.frexp(amax / 448.0)        # amax/448 = mant * 2^ex, mant in [0.5, 1)
+            k = ex - 1 if mant == 0.5 else ex
+            assert exps[r_, blk] == k + 127
+            assert 224.0 < amax / 2.0 ** k <= 448.0
+            ref = torch.from_numpy((seg / 2.0 ** k).astype(np.float32)).to(torch.float8_e4m3fn)
+            got = codes[r_, blk * 128:(blk + 1) * 128]
+            refv = ref.to(torch.float64).numpy()
+            gotv = np.array([oracle.e4m3_decode(c) for c in got])
+            assert np.array_equal(refv, gotv), (r_, blk)
+
+
+def test_fp8_kv_dequantised_values_are_bf16_and_within_half_an_e4m3_step():
+    x = _fp8_rows(31)
+    codes, exps = oracle.quantize_fp8_kv(x, 128)
+    dq = oracle.dequantize_fp8_kv(codes, exps, 128)
+    np.testing.assert_array_equal(bf16_val(bf16_bits(dq)), dq)            # exactly representable in bf16
+    xv = bf16_val(x)
+    s = np.repeat(2.0 ** (exps.astype(np.float64) - 127), 128, axis=-1)
+    bound = np.maximum(2.0 ** -4 * np.abs(xv), 2.0 ** -10 * s)              # half a step, normal / subnormal
+    assert np.all(np.abs(dq - xv) <= bound)
+
+
+def test_fp8_kv_round_trip_of_representable_rows():
+    """Rows built from e4m3 values times a power of two whose block maximum is
+    448 * 2^k come back exactly."""
+    r = rng(32)
+    vals = np.array([oracle.e4m3_decode(c) for c in range(0x7F)])
+    rows = []
+    for k in (-9, 0, 5):
+        v = r.choice(vals, 256) * r.choice([-1.0, 1.0], 256)
+        v[0] = 448.0
+        v[128] = -448.0
+        rows.append(v * 2.0 ** k)
+    x = bf16_bits(np.array(rows))
+    codes, exps = oracle.quantize_fp8_kv(x, 128)
+    np.testing.assert_array_equal(oracle.dequantize_fp8_kv(codes, exps, 128), bf16_val(x))
+    assert list(exps[:, 0]) == [127 - 9, 127, 127 + 5]
+
+
 def test_fp4_index_equals_bf16_index_on_dequantised_operands():
     r = rng(19)
     b, nq, H_I, d_I, N, m = 2, 2, 4, 32, 16, 4
