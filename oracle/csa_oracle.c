@@ -28,14 +28,18 @@
  *              (one KV head, 128 query heads), "Sliding-window attention"
  *              (window 128, current token included), "Indexer-selected sparse
  *              attention" (top-k 1024, 64 x 128 indexer heads, invalid slots
- *              -> -1), "QK normalization"; list "inference quantization"
- *              -> "FP4 precision for the attention indexer".
+ *              -> -1), "QK normalization", "Learnable attention sink",
+ *              "Partial RoPE", "Gated attention output" (rope-conjugate
+ *              rotation of the output); list "inference quantization"
+ *              -> "FP4 precision for the attention indexer", "FP8 KV-cache
+ *              quantization".
  *   [DSv4-FP4] "DeepSeek V4 paper full version is out, FP4 QAT details and
  *              stability tricks [D]" (corsoro.com): the indexer QK path uses
  *              FP4 activations.
  * Where the pages leave a formula open the reading used here is the one
- * stated at each function (pooling logit order, causal visibility, window
- * rows, FP4 block format).
+ * stated at each function (pooling logit order, compression-weight rows,
+ * causal visibility, window rows, RoPE tables and pairing, FP4 and FP8 block
+ * formats).
  *
  * Parity pins: every function below is pinned by tests/test_oracle_pins.py
  * against closed forms, brute force or an independent library routine.
