@@ -115,7 +115,8 @@ int csa_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Z
     if (!al16(A) || !al16(B) || !al16(bias) || !al16(out)) return CSA_ERR_INVALID;
     if ((Za && !al16(Za)) || (Zb && !al16(Zb)) || (gain && !al4(gain))) return CSA_ERR_INVALID;
     if (batch < 1 || m < 1 || T < m || d < 8 || d % 8 != 0 || !(eps >= 0.f)) return CSA_ERR_INVALID;
-    if (i0 < 0 || ni < 0 || i0 + ni > T / m || n_out < i0 + ni) return CSA_ERR_INVALID;
+    // overflow-free form of 0 <= i0, 0 <= ni, i0 + ni <= floor(T / m) <= n_out
+    if (i0 < 0 || ni < 0 || ni > T / m || i0 > T / m - ni || n_out < i0 + ni) return CSA_ERR_INVALID;
     if (d > 2048) return CSA_ERR_UNSUPPORTED;
     return csa::launch_compress_dynamic(A, B, Za, Zb, bias, batch, T, d, m, apply_rmsnorm, gain, eps, i0, ni,
                                         n_out, out, S(stream));

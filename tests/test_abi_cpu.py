@@ -89,6 +89,9 @@ def test_compress_dynamic_validation(lib):
     assert call(i0=10, ni=7) == csa.CSA_ERR_INVALID            # (i0 + ni) * m > T
     assert call(i0=0, ni=16, n_out=15) == csa.CSA_ERR_INVALID  # out too short
     assert call(T=4096, d=2056, ni=1, n_out=1) == csa.CSA_ERR_UNSUPPORTED
+    big = 1 << 62                                                  # i0 + ni would overflow
+    assert call(i0=big, ni=big, n_out=big) == csa.CSA_ERR_INVALID
+    assert call(i0=big, ni=1, n_out=big) == csa.CSA_ERR_INVALID
 
 
 def test_index_validation(lib):
