@@ -225,9 +225,17 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  *   sinks   [H] fp32 or NULL: a learnable per-head sink logit that joins each
  *             head's softmax denominator with no value row (techniques map,
  *             "Learnable attention sink"); NULL = no sink
+ *   rope_cos, rope_sin [rope_positions][32] fp32 or both NULL: partial RoPE
+ *             (techniques map "Partial RoPE", "Gated attention output"): the
+ *             trailing 64 channels of q_hat_h rotate at the query position t
+ *             in the rotate-half form (channel D-64+i with D-32+i, angle of
+ *             pair i: cos/sin[t][i]) before the dot products, and out_h gets
+ *             the conjugate rotation at t.  Keys and window rows must already
+ *             be rotated at their own positions.  A query position outside
+ *             [0, rope_positions) is not rotated.
  *   J       = { kv[b][j] : j in idx[b][q], 0 <= j < N }
  *             U { stream-A row of position u : max(0, t-W+1) <= u <= t }
- *   out_h   = sum_{x in J} softmax(scale * q_hat_h . x) * x
+ *   out_h   = R_t^-1 sum_{x in J} softmax(scale * (R_t q_hat_h) . x) * x   (R = identity without RoPE)
  * bf16 operands, fp32 softmax and accumulation, bf16 output.
  *   q       [batch][nq][H][D] bf16      kv [batch][N][D] bf16
  *   idx     [batch][nq][k] int32 (-1 = invalid slot; entries outside [0, N) are skipped)
@@ -240,7 +248,8 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, k + W).
  */
 size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
-int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                long long win_rows, int W,
                const int *q_pos, int batch, int nq, int H, int D, float scale, float eps,
@@ -253,7 +262,8 @@ int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
  * compresses every m' >> m tokens and keeps attention dense).
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, N + W).
  */
-int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N, int m,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
                const int *q_pos,
                int batch, int nq, int H, int D, float scale, float eps,
@@ -284,7 +294,8 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
  * race on it, so serialise them.
  */
 #define CSA_ATTEND_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
-int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                       const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                        const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                        long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
                        float scale, float eps, uint16_t *out, void *stream);

@@ -50,10 +50,10 @@ def load() -> ctypes.CDLL:
         "csa_rescore_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "csa_rescore_topk": ([P, P, P, P, i32, i32, i32, i64, i32, i32, i32, P, P, sz, P], i32),
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
-        "csa_attend": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
+        "csa_attend": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
                        i32),
-        "hca_attend": ([P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
-        "csa_attend_noalloc": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
+        "hca_attend": ([P, P, P, P, P, i64, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_attend_noalloc": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
                                i32),
         "csa_sync_status": ([P], i32),
         "csa_set_wait_budget_ns": ([ctypes.c_ulonglong], None),
@@ -249,10 +249,23 @@ def _sinks(sinks, H):
     return _p(sinks)
 
 
+def _rope(rope, D):
+    """rope = (cos, sin) fp32 tables [positions][32] or None -> (cos ptr, sin ptr, positions)."""
+    if rope is None:
+        return None, None, 0
+    cos, sin = rope
+    _need(cos, torch.float32, "rope cos", 2)
+    _need(sin, torch.float32, "rope sin", 2)
+    if cos.shape != sin.shape or cos.shape[1] != 32 or D < 64:
+        raise ValueError("rope tables must be [positions][32] (64 rotated channels, D >= 64)")
+    return _p(cos), _p(sin), cos.shape[0]
+
+
 def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0, sinks=None):
+               workspace=None, win_pos0: int = 0, sinks=None, rope=None):
     """q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] (bf16, stream-A rows of positions
-    win_pos0..) -> out [b][nq][H][D] bf16.  sinks: optional per-head sink logits [H] fp32."""
+    win_pos0..) -> out [b][nq][H][D] bf16.  sinks: optional per-head sink logits [H] fp32.  rope: optional
+    (cos, sin) [positions][32] fp32 tables for partial RoPE (keys and window rows arrive rotated)."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
     _need(kv, torch.bfloat16, "kv", 3)
@@ -264,14 +277,14 @@ def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, 
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
-    _check(L.csa_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
+    _check(L.csa_attend(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
                         _p(q_pos),
                         batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend")
     return out
 
 
 def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0, sinks=None):
+               workspace=None, win_pos0: int = 0, sinks=None, rope=None):
     """Dense attention over every visible entry of kv [b][N][D] plus the window."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
@@ -283,14 +296,14 @@ def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
-    _check(L.hca_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos),
+    _check(L.hca_attend(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos),
                         batch, nq, H,
                         D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend")
     return out
 
 
 def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-                       win_pos0: int = 0, sinks=None):
+                       win_pos0: int = 0, sinks=None, rope=None):
     """csa_attend without a caller workspace: the library's own fixed device
     scratch is used (for callers that cannot allocate; see include/csa.h)."""
     L = load()
@@ -303,7 +316,7 @@ def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float 
     N, rows, k = kv.shape[1], win.shape[1], idx.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0),
+    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, _p(idx), k, _p(win), int(win_pos0),
                                 rows, W,
                                 _p(q_pos), batch, nq, H, D, float(scale), float(eps), _p(out), _stream()),
            "csa_attend_noalloc")

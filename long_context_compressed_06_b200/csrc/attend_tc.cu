@@ -214,9 +214,15 @@ struct QLanes {
     static constexpr int PASSES = (kHeads / 4) / RPI;
 };
 
+// With partial RoPE the row's last kRopeDim / 8 units (all in a lane's last
+// unit slot, since kRopeDim <= D) rotate after the gain: unit r0 + j pairs
+// with r0 + j + 4, held by lane ^ 4 in the same slot, so one shuffle fetches
+// the partner values.
 template <int D>
-CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8]) {
+CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8],
+                            long long t) {
     using QL = QLanes<D>;
+    static_assert(D >= kRopeDim && kRopeDim / 8 == 8, "rope units: 8 per row, partners 4 units apart");
     const int lane = threadIdx.x & 31;
     const int sub = lane / QL::LPR, ul = lane % QL::LPR;
 #pragma unroll 4
@@ -238,12 +244,28 @@ CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const fl
         for (int o = QL::LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
 #pragma unroll
-        for (int u = 0; u < QL::UPL; ++u) {
-            float y[8];
+        for (int u = 0; u < QL::UPL; ++u)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = x[u][e] * r * g[u][e];
-            *ptr[u] = pack8(y);
+            for (int e = 0; e < 8; ++e) x[u][e] = x[u][e] * r * g[u][e];
+        if (a.rope_cos) {  // uniform over the grid: every lane takes the shuffles
+            constexpr int u = QL::UPL - 1;
+            constexpr int r0 = QL::UR - kRopeDim / 8;  // first rotated unit
+            const int unit = ul + u * QL::LPR;
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, x[u][e], 4);
+            if (unit >= r0) {
+                const bool first = unit < r0 + 4;  // first half of the rotated slice
+                const int i0 = ((unit - r0) & 3) * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float2 cs = rope_cs(a, t, i0 + e);
+                    x[u][e] = first ? x[u][e] * cs.x - pv[e] * cs.y : x[u][e] * cs.x + pv[e] * cs.y;
+                }
+            }
         }
+#pragma unroll
+        for (int u = 0; u < QL::UPL; ++u) *ptr[u] = pack8(x[u]);
     }
 }
 
@@ -491,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = work_item(p, wi);
             const int h = it.head0 + hl;
             if (!warp_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag)) break;
-            normalize_q<D>(a, s, sp, qg);
+            const long long tq = __ldg(a.q_pos + it.bq);
+            normalize_q<D>(a, s, sp, qg, tq);
             tc::fence_proxy_async_smem();
             mbar_arrive(smem_u32(s.qready));
 
@@ -610,7 +633,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
                         const float4 hi =
                             *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
-                        const float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        if (a.rope_cos && c == D - kRopeDim) {
+                            // conjugate rotation of the rotated slice (this 64-column slab):
+                            // column 8*cu + e pairs with 8*(cu ^ 4) + e, held by lane ^ 4
+                            float pv[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
+                            const bool first = cu < 4;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float2 cs = rope_cs(a, tq, (cu & 3) * 8 + e);
+                                o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
+                            }
+                        }
                         if (hr < a.H)
                             *reinterpret_cast<uint4 *>(a.out + ((size_t)it.bq * a.H + hr) * D + c + 8 * cu) = pack8(o);
                     }

@@ -49,7 +49,8 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
 // Attention: dense selects the HCA key set of the first n_vis(t) entries;
 // otherwise the k selected entries idx (may be null when k == 0).
 size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
-int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                  const float *rope_sin, long long rope_npos, const uint16_t *kv, long long N, int m,
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,
