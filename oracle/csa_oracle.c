@@ -696,11 +696,14 @@ int orc_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, const u
  * e4m3 codes with one power-of-two scale per block of `block` channels, the
  * scale kept as an unsigned 8-bit exponent (UE8M0: s = 2^(e - 127)).  s is the
  * smallest power of two with absmax(block) / s <= 448 (the largest finite
- * e4m3 magnitude); the codes are e4m3_RNE(x / s), the division by a power of
- * two being exact; an all-zero block has e = 127 and zero codes.  With s a
- * power of two and 3 mantissa bits per code, every dequantised value
- * code * s is a bf16 number exactly, so attention over the FP8 cache is the
- * attention of section 4 over those bf16 rows.
+ * e4m3 magnitude), its exponent k kept in [-124, 119]; the codes are
+ * e4m3_RNE(x / s), the division by a power of two being exact; an all-zero
+ * block has e = 127 and zero codes.  With s a power of two, 3 mantissa bits
+ * per code and k in that range (the smallest code times s is at least bf16's
+ * smallest subnormal 2^-133, 448 * s stays below bf16's largest value), every
+ * dequantised value code * s is a bf16 number exactly, so attention over the
+ * FP8 cache is the attention of section 4 over those bf16 rows.  (Blocks whose
+ * absmax exceeds 448 * 2^119 saturate.)
  */
 void orc_quantize_fp8_kv(const uint16_t *x, long long rows, int d, int block, uint8_t *codes,
                          uint8_t *exps)
@@ -719,8 +722,8 @@ void orc_quantize_fp8_kv(const uint16_t *x, long long rows, int d, int block, ui
                 k = (int)ceil(log2(amax / 448.0));
                 while (ldexp(amax, -k) > 448.0) ++k;          /* guard the log2 rounding */
                 while (ldexp(amax, -(k - 1)) <= 448.0) --k;   /* smallest such k */
-                if (k < -127) k = -127;
-                if (k > 127) k = 127;
+                if (k < -124) k = -124;   /* 2^-9 * 2^k stays a bf16 number (>= 2^-133) */
+                if (k > 119) k = 119;     /* 448 * 2^k stays finite in bf16 */
             }
             exps[(size_t)r * nblk + blk] = (uint8_t)(k + 127);
             for (int j = 0; j < block; ++j)

@@ -700,6 +700,23 @@ def test_fp8_kv_dequantised_values_are_bf16_and_within_half_an_e4m3_step():
     assert np.all(np.abs(dq - xv) <= bound)
 
 
+def test_fp8_kv_extreme_blocks_keep_every_value_a_finite_bf16():
+    """A block of bf16's smallest subnormals and one near its largest value:
+    the scale exponent is clamped to [-124, 119], so the dequantised values
+    stay exact bf16 numbers and finite."""
+    tiny = np.full((1, 128), 2.0 ** -133)
+    tiny[0, 1::2] = 3 * 2.0 ** -133
+    big = np.full((1, 128), 1.9921875 * 2.0 ** 127)    # bf16's largest value: it would need k = 120
+    x = bf16_bits(np.concatenate([tiny, big], axis=1))
+    codes, exps = oracle.quantize_fp8_kv(x, 128)
+    assert list(exps[0]) == [127 - 124, 127 + 119]
+    dq = oracle.dequantize_fp8_kv(codes, exps, 128)
+    assert np.all(np.isfinite(dq))
+    np.testing.assert_array_equal(bf16_val(bf16_bits(dq)), dq)
+    np.testing.assert_array_equal(dq[0, :128], bf16_val(x)[0, :128])   # 2^-133 = code 2^-9 at s = 2^-124
+    assert np.all(dq[0, 128:] == 448.0 * 2.0 ** 119)                    # saturated
+
+
 def test_fp8_kv_round_trip_of_representable_rows():
     """Rows built from e4m3 values times a power of two whose block maximum is
     448 * 2^k come back exactly."""
