@@ -301,6 +301,41 @@ int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sink
                        float scale, float eps, uint16_t *out, void *stream);
 
 /*
+ * FP8 KV cache ("DeepSeek-V4-Pro - Model techniques map", list "inference
+ * quantization": FP8 KV-cache quantisation; the pages give no format).
+ *
+ * csa_quantize_fp8_kv -- rows x [rows][d] bf16 -> e4m3 codes [rows][d] u8 and
+ * one UE8M0 exponent byte per 128 channels, exps [rows][d/128] u8, value =
+ * code * 2^(e - 127).  Per 128-channel block: s = 2^k the smallest power of
+ * two with absmax / s <= 448, k kept in [-124, 119] (so every code times s is
+ * a finite bf16 number); codes = e4m3 round-to-nearest-even of x / s with
+ * saturation, a zero magnitude stored as +0; an all-zero block has e = 127.
+ * Requirements: d % 128 == 0, rows >= 0; x and codes 16-byte aligned, exps
+ * non-NULL (CSA_ERR_INVALID otherwise).
+ *
+ * csa_attend_fp8kv / hca_attend_fp8kv -- csa_attend / hca_attend with the
+ * compressed entries (kv8 [batch][N][D], kv8_exp [batch][N][D/128]) and the
+ * window rows (win8 [batch][win_rows][D], win8_exp [batch][win_rows][D/128])
+ * stored as above.  Each row is converted to bf16 exactly while it is
+ * gathered, so the result is that of the bf16 call on the dequantised rows.
+ * Requirements: those of csa_attend / hca_attend, D in {128, 256, 512}
+ * (CSA_ERR_UNSUPPORTED otherwise), kv8 and win8 16-byte aligned, exponent
+ * arrays non-NULL.  Workspace: as the bf16 calls.
+ */
+int csa_quantize_fp8_kv(const uint16_t *x, long long rows, int d, uint8_t *codes, uint8_t *exps, void *stream);
+int csa_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, const int *idx, int k, const uint8_t *win8, const uint8_t *win8_exp,
+                     long long win_pos0, long long win_rows, int W, const int *q_pos, int batch, int nq, int H,
+                     int D, float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes,
+                     void *stream);
+int hca_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, int m, const uint8_t *win8, const uint8_t *win8_exp, long long win_pos0,
+                     long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D, float scale,
+                     float eps, uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * csa_sync_status -- synchronise `stream`, then read and clear the device
  * status word.  Returns CSA_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call, CSA_ERR_CUDA on a CUDA error, else CSA_OK.

@@ -98,14 +98,17 @@ size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_key
 }
 
 int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
-                  const float *rope_sin, long long rope_npos, const uint16_t *kv, long long N, int m,
+                  const float *rope_sin, long long rope_npos, const Fp8Kv *fp8, const uint16_t *kv, long long N, int m,
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
                   size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
     AttendArgs a = {};
     a.q = q; a.q_gain = q_gain; a.sinks = sinks; a.rope_cos = rope_cos; a.rope_sin = rope_sin;
-    a.rope_npos = rope_npos; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
+    a.rope_npos = rope_npos; a.kv = kv;
+    if (fp8) {
+        a.kv8 = fp8->kv; a.kv8e = fp8->kv_exp; a.win8 = fp8->win; a.win8e = fp8->win_exp;
+    } a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
     a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
     a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
     if (a.n_bq == 0) return CSA_OK;
@@ -119,7 +122,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(float));
     }
     if (attend_tc_supported(H, D)) return launch_attend_tc(a, ctx, st);
-    if (rope_cos) return CSA_ERR_UNSUPPORTED;  // the CUDA-core kernel has no RoPE
+    if (rope_cos || fp8) return CSA_ERR_UNSUPPORTED;  // the CUDA-core kernel has neither RoPE nor FP8 rows
     return launch_attend_simt(a, st);
 }
 

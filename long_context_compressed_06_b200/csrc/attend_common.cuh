@@ -20,6 +20,10 @@ struct AttendArgs {
     const float *rope_sin;  // [rope_npos][kRopeDim / 2]
     long long rope_npos;
     const uint16_t *kv;     // [batch][N][D]
+    // FP8 KV cache (instead of kv / win when kv8 is set): e4m3 codes and one
+    // UE8M0 exponent byte per 128 channels, value = code * 2^(e - 127)
+    const uint8_t *kv8, *kv8e;    // [batch][N][D], [batch][N][D/128]
+    const uint8_t *win8, *win8e;  // [batch][win_rows][D], [batch][win_rows][D/128]
     long long N;
     int m;                  // compression ratio (dense key set only)
     const int *idx;         // [n_bq][k] selected entries (CSA); unused when dense

@@ -91,6 +91,33 @@ def test_compress_dynamic_validation(lib):
     assert call(T=4096, d=2056, ni=1, n_out=1) == csa.CSA_ERR_UNSUPPORTED
 
 
+def test_fp8_kv_validation(lib):
+    f = lib.csa_quantize_fp8_kv
+    assert f(NULL, 4, 512, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 512, MIS, A16, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 512, A16b, NULL, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 192, A16b, A16, NULL) == csa.CSA_ERR_INVALID     # d % 128
+    assert f(A16, -1, 512, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+    g = lib.csa_attend_fp8kv
+    # (q, g, sinks, rc, rs, rn, kv8, kv8e, N, idx, k, win8, win8e, p0, rows, W, pos, b, nq, H, D, scale, eps, out, ws, wsb, st)
+    base = [A16, NULL, NULL, NULL, NULL, 0, A16, A16, 300, A16, 64, A16, A16, 0, 2048, 16, A16, 1, 1, 8, 512, 0.125,
+            1e-6, A16b, NULL, 0, NULL]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return g(*a)
+
+    assert call(a6=MIS) == csa.CSA_ERR_INVALID          # codes misaligned
+    assert call(a7=NULL) == csa.CSA_ERR_INVALID         # exponents missing
+    assert call(a12=NULL) == csa.CSA_ERR_INVALID        # window exponents missing
+    assert call(a20=64) == csa.CSA_ERR_UNSUPPORTED      # D = 64: no whole 128-channel block
+    h = lib.hca_attend_fp8kv
+    assert h(A16, NULL, NULL, NULL, NULL, 0, A16, A16, 300, 0, A16, A16, 0, 2048, 16, A16, 1, 1, 8, 512, 0.125, 1e-6,
+             A16b, NULL, 0, NULL) == csa.CSA_ERR_INVALID    # m
+
+
 def test_index_validation(lib):
     f = lib.csa_index
     ok = (A16, A16, A16, A16)
