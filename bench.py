@@ -463,6 +463,30 @@ def bench_compress_dynamic(csa, args, device, peaks, wl: W.Workload):
             "hbm_gbs": round(byts / t / 1e9, 1), "frac": round(byts / t / 1e9 / peaks["hbm_gbs"], 4)}
 
 
+def bench_fp8kv_decode(csa, args, device, peaks):
+    """The 128K decode attention with the KV cache in FP8 (compressed entries and window rows as e4m3 codes
+    plus one exponent byte per 128 channels), timed beside the bf16 attention on the same selection."""
+    wl = W.CSA_DECODE
+    st = decode_cache_state(csa, wl, device, 0)
+    kv8, kv8e = csa.csa_quantize_fp8_kv(st["C"])
+    w8, w8e = csa.csa_quantize_fp8_kv(st["win"])
+    csa.csa_index(st["qI"], st["w"], st["kI"], st["qp"], wl.m, scores=st["S"])
+    csa.csa_topk(st["S"], st["qp"], wl.m, wl.k, idx=st["idx"])
+    args8 = (st["q"], kv8, kv8e, st["idx"], w8, w8e, st["qp"], wl.W, wl.scale, wl.eps)
+    args16 = (st["q"], st["C"], st["idx"], st["win"], st["qp"], wl.W, wl.scale, wl.eps)
+    kw = dict(out=st["out"], workspace=st["ws"], win_pos0=st["win_pos0"])
+    steps = max(3, min(args.steps, 20))
+    t8, _ = Timer(device).run(lambda mark: csa.csa_attend_fp8kv(*args8, **kw), steps, 3)
+    t16, _ = Timer(device).run(lambda mark: csa.csa_attend(*args16, **kw), steps, 3)
+    t8, t16 = t8 / steps, t16 / steps
+    rows = wl.k + wl.W
+    byts8 = wl.batch * (rows * (wl.D + wl.D // 128) + 2 * wl.H * wl.D * 2 + wl.k * 4)
+    byts16 = wl.batch * (rows * wl.D * 2 + 2 * wl.H * wl.D * 2 + wl.k * 4)
+    return {"workload": "csa_decode_128k_fp8kv_attend", "attend_ms_fp8": round(t8 * 1e3, 4),
+            "attend_ms_bf16": round(t16 * 1e3, 4), "bytes_fp8": byts8, "bytes_bf16": byts16,
+            "hbm_gbs_fp8": round(byts8 / t8 / 1e9, 1), "frac_fp8": round(byts8 / t8 / 1e9 / peaks["hbm_gbs"], 4)}
+
+
 def bench_hca(csa, args, device, peaks):
     wl = W.HCA_DECODE
     L = W.pool_logits(wl, device)
@@ -633,7 +657,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress", "compress_dynamic"],
+    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress", "compress_dynamic", "fp8kv"],
                     help="run one of the other workloads alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -653,6 +677,7 @@ def main():
                    "fp4": lambda: bench_fp4(csa, args, device, peaks),
                    "compress": lambda: bench_compress(csa, args, device, peaks, W.HCA_DECODE),
                    "compress_dynamic": lambda: bench_compress_dynamic(csa, args, device, peaks, W.CSA_DECODE),
+                   "fp8kv": lambda: bench_fp8kv_decode(csa, args, device, peaks),
                    }[args.only]
         res = run_one()
         rc = csa.csa_sync_status()
@@ -675,6 +700,8 @@ def main():
         extra["hca_decode_1m"] = bench_hca(csa, args, device, peaks)
         torch.cuda.empty_cache()
         extra["fp4_index_decode_1m"] = bench_fp4(csa, args, device, peaks)
+        torch.cuda.empty_cache()
+        extra["fp8kv_decode_128k"] = bench_fp8kv_decode(csa, args, device, peaks)
         torch.cuda.empty_cache()
         extra["compress_m4_128k"] = bench_compress(csa, args, device, peaks, W.CSA_DECODE)
         extra["compress_m128_1m"] = bench_compress(csa, args, device, peaks, W.HCA_DECODE)

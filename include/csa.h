@@ -225,9 +225,17 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  *   sinks   [H] fp32 or NULL: a learnable per-head sink logit that joins each
  *             head's softmax denominator with no value row (techniques map,
  *             "Learnable attention sink"); NULL = no sink
+ *   rope_cos, rope_sin [rope_positions][32] fp32 or both NULL: partial RoPE
+ *             (techniques map "Partial RoPE", "Gated attention output"): the
+ *             trailing 64 channels of q_hat_h rotate at the query position t
+ *             in the rotate-half form (channel D-64+i with D-32+i, angle of
+ *             pair i: cos/sin[t][i]) before the dot products, and out_h gets
+ *             the conjugate rotation at t.  Keys and window rows must already
+ *             be rotated at their own positions.  A query position outside
+ *             [0, rope_positions) is not rotated.
  *   J       = { kv[b][j] : j in idx[b][q], 0 <= j < N }
  *             U { stream-A row of position u : max(0, t-W+1) <= u <= t }
- *   out_h   = sum_{x in J} softmax(scale * q_hat_h . x) * x
+ *   out_h   = R_t^-1 sum_{x in J} softmax(scale * (R_t q_hat_h) . x) * x   (R = identity without RoPE)
  * bf16 operands, fp32 softmax and accumulation, bf16 output.
  *   q       [batch][nq][H][D] bf16      kv [batch][N][D] bf16
  *   idx     [batch][nq][k] int32 (-1 = invalid slot; entries outside [0, N) are skipped)
@@ -240,7 +248,8 @@ int csa_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_id
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, k + W).
  */
 size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
-int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                long long win_rows, int W,
                const int *q_pos, int batch, int nq, int H, int D, float scale, float eps,
@@ -253,7 +262,8 @@ int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
  * compresses every m' >> m tokens and keeps attention dense).
  * Workspace: csa_attend_workspace_bytes(batch, nq, H, D, N + W).
  */
-int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N, int m,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
                const int *q_pos,
                int batch, int nq, int H, int D, float scale, float eps,
@@ -284,10 +294,46 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
  * race on it, so serialise them.
  */
 #define CSA_ATTEND_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
-int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                       const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                        const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                        long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
                        float scale, float eps, uint16_t *out, void *stream);
+
+/*
+ * FP8 KV cache ("DeepSeek-V4-Pro - Model techniques map", list "inference
+ * quantization": FP8 KV-cache quantisation; the pages give no format).
+ *
+ * csa_quantize_fp8_kv -- rows x [rows][d] bf16 -> e4m3 codes [rows][d] u8 and
+ * one UE8M0 exponent byte per 128 channels, exps [rows][d/128] u8, value =
+ * code * 2^(e - 127).  Per 128-channel block: s = 2^k the smallest power of
+ * two with absmax / s <= 448, k kept in [-124, 119] (so every code times s is
+ * a finite bf16 number); codes = e4m3 round-to-nearest-even of x / s with
+ * saturation, a zero magnitude stored as +0; an all-zero block has e = 127.
+ * Requirements: d % 128 == 0, rows >= 0; x and codes 16-byte aligned, exps
+ * non-NULL (CSA_ERR_INVALID otherwise).
+ *
+ * csa_attend_fp8kv / hca_attend_fp8kv -- csa_attend / hca_attend with the
+ * compressed entries (kv8 [batch][N][D], kv8_exp [batch][N][D/128]) and the
+ * window rows (win8 [batch][win_rows][D], win8_exp [batch][win_rows][D/128])
+ * stored as above.  Each row is converted to bf16 exactly while it is
+ * gathered, so the result is that of the bf16 call on the dequantised rows.
+ * Requirements: those of csa_attend / hca_attend, D in {128, 256, 512}
+ * (CSA_ERR_UNSUPPORTED otherwise), kv8 and win8 16-byte aligned, exponent
+ * arrays non-NULL.  Workspace: as the bf16 calls.
+ */
+int csa_quantize_fp8_kv(const uint16_t *x, long long rows, int d, uint8_t *codes, uint8_t *exps, void *stream);
+int csa_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, const int *idx, int k, const uint8_t *win8, const uint8_t *win8_exp,
+                     long long win_pos0, long long win_rows, int W, const int *q_pos, int batch, int nq, int H,
+                     int D, float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes,
+                     void *stream);
+int hca_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, int m, const uint8_t *win8, const uint8_t *win8_exp, long long win_pos0,
+                     long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D, float scale,
+                     float eps, uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * csa_sync_status -- synchronise `stream`, then read and clear the device

@@ -41,6 +41,11 @@ def load() -> ctypes.CDLL:
         "csa_strerror": ([i32], ctypes.c_char_p),
         "csa_version": ([], i32),
         "csa_compress": ([P, P, P, i32, i64, i32, i32, i32, P, f32, P, P], i32),
+        "csa_quantize_fp8_kv": ([P, i64, i32, P, P, P], i32),
+        "csa_attend_fp8kv": ([P, P, P, P, P, i64, P, P, i64, P, i32, P, P, i64, i64, i32, P, i32, i32, i32, i32, f32,
+                              f32, P, P, sz, P], i32),
+        "hca_attend_fp8kv": ([P, P, P, P, P, i64, P, P, i64, i32, P, P, i64, i64, i32, P, i32, i32, i32, i32, f32,
+                              f32, P, P, sz, P], i32),
         "csa_compress_dynamic": ([P, P, P, P, P, i32, i64, i32, i32, i32, P, f32, i64, i64, P, i64, P], i32),
         "csa_index": ([P, P, P, P, i32, i32, i64, i32, i32, i32, P, P], i32),
         "csa_quantize_fp4": ([P, i64, i32, P, P, P], i32),
@@ -50,10 +55,10 @@ def load() -> ctypes.CDLL:
         "csa_rescore_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "csa_rescore_topk": ([P, P, P, P, i32, i32, i32, i64, i32, i32, i32, P, P, sz, P], i32),
         "csa_attend_workspace_bytes": ([i32, i32, i32, i32, i64], sz),
-        "csa_attend": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
+        "csa_attend": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
                        i32),
-        "hca_attend": ([P, P, P, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
-        "csa_attend_noalloc": ([P, P, P, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
+        "hca_attend": ([P, P, P, P, P, i64, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_attend_noalloc": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
                                i32),
         "csa_sync_status": ([P], i32),
         "csa_set_wait_budget_ns": ([ctypes.c_ulonglong], None),
@@ -249,10 +254,23 @@ def _sinks(sinks, H):
     return _p(sinks)
 
 
+def _rope(rope, D):
+    """rope = (cos, sin) fp32 tables [positions][32] or None -> (cos ptr, sin ptr, positions)."""
+    if rope is None:
+        return None, None, 0
+    cos, sin = rope
+    _need(cos, torch.float32, "rope cos", 2)
+    _need(sin, torch.float32, "rope sin", 2)
+    if cos.shape != sin.shape or cos.shape[1] != 32 or D < 64:
+        raise ValueError("rope tables must be [positions][32] (64 rotated channels, D >= 64)")
+    return _p(cos), _p(sin), cos.shape[0]
+
+
 def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0, sinks=None):
+               workspace=None, win_pos0: int = 0, sinks=None, rope=None):
     """q [b][nq][H][D], kv [b][N][D], idx [b][nq][k], win [b][rows][D] (bf16, stream-A rows of positions
-    win_pos0..) -> out [b][nq][H][D] bf16.  sinks: optional per-head sink logits [H] fp32."""
+    win_pos0..) -> out [b][nq][H][D] bf16.  sinks: optional per-head sink logits [H] fp32.  rope: optional
+    (cos, sin) [positions][32] fp32 tables for partial RoPE (keys and window rows arrive rotated)."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
     _need(kv, torch.bfloat16, "kv", 3)
@@ -264,14 +282,14 @@ def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, 
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
-    _check(L.csa_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
+    _check(L.csa_attend(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, _p(idx), k, _p(win), int(win_pos0), rows, W,
                         _p(q_pos),
                         batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend")
     return out
 
 
 def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-               workspace=None, win_pos0: int = 0, sinks=None):
+               workspace=None, win_pos0: int = 0, sinks=None, rope=None):
     """Dense attention over every visible entry of kv [b][N][D] plus the window."""
     L = load()
     _need(q, torch.bfloat16, "q", 4)
@@ -283,14 +301,79 @@ def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-
     if out is None:
         out = torch.empty_like(q)
     ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
-    _check(L.hca_attend(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos),
+    _check(L.hca_attend(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, m, _p(win), int(win_pos0), rows, W, _p(q_pos),
                         batch, nq, H,
                         D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend")
     return out
 
 
+def csa_quantize_fp8_kv(x, codes=None, exps=None):
+    """KV rows x [..., d] bf16 (d % 128 == 0) -> (e4m3 codes [..., d] u8, UE8M0 exponents [..., d/128] u8)."""
+    L = load()
+    _need(x, torch.bfloat16, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if exps is None:
+        exps = torch.empty(x.shape[:-1] + (d // 128,), dtype=torch.uint8, device=x.device)
+    _need(codes, torch.uint8, "codes")
+    _need(exps, torch.uint8, "exps")
+    if codes.shape != x.shape or exps.numel() != rows * (d // 128):
+        raise ValueError("shape mismatch")
+    _check(L.csa_quantize_fp8_kv(_p(x), rows, d, _p(codes), _p(exps), _stream()), "csa_quantize_fp8_kv")
+    return codes, exps
+
+
+def _fp8_rows(codes, exps, name):
+    _need(codes, torch.uint8, name, 3)
+    _need(exps, torch.uint8, name + " exponents", 3)
+    if exps.shape != codes.shape[:2] + (codes.shape[2] // 128,):
+        raise ValueError("%s exponents must be [..][..][D/128]" % name)
+
+
+def csa_attend_fp8kv(q, kv8, kv8_exp, idx, win8, win8_exp, q_pos, W: int, scale: float, eps: float = 1e-6,
+                     q_gain=None, out=None, workspace=None, win_pos0: int = 0, sinks=None, rope=None):
+    """csa_attend over an FP8 KV cache: kv8 [b][N][D] / win8 [b][rows][D] e4m3 codes with UE8M0 exponents
+    [..][D/128] (from csa_quantize_fp8_kv)."""
+    L = load()
+    _need(q, torch.bfloat16, "q", 4)
+    _fp8_rows(kv8, kv8_exp, "kv8")
+    _fp8_rows(win8, win8_exp, "win8")
+    _need(idx, torch.int32, "idx", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H, D = q.shape
+    N, rows, k = kv8.shape[1], win8.shape[1], idx.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
+    _check(L.csa_attend_fp8kv(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv8), _p(kv8_exp), N, _p(idx),
+                              k, _p(win8), _p(win8_exp), int(win_pos0), rows, W, _p(q_pos), batch, nq, H, D,
+                              float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend_fp8kv")
+    return out
+
+
+def hca_attend_fp8kv(q, kv8, kv8_exp, m: int, win8, win8_exp, q_pos, W: int, scale: float, eps: float = 1e-6,
+                     q_gain=None, out=None, workspace=None, win_pos0: int = 0, sinks=None, rope=None):
+    """hca_attend over an FP8 KV cache."""
+    L = load()
+    _need(q, torch.bfloat16, "q", 4)
+    _fp8_rows(kv8, kv8_exp, "kv8")
+    _fp8_rows(win8, win8_exp, "win8")
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H, D = q.shape
+    N, rows = kv8.shape[1], win8.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, N + W), q.device, workspace)
+    _check(L.hca_attend_fp8kv(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv8), _p(kv8_exp), N, m,
+                              _p(win8), _p(win8_exp), int(win_pos0), rows, W, _p(q_pos), batch, nq, H, D,
+                              float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "hca_attend_fp8kv")
+    return out
+
+
 def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,
-                       win_pos0: int = 0, sinks=None):
+                       win_pos0: int = 0, sinks=None, rope=None):
     """csa_attend without a caller workspace: the library's own fixed device
     scratch is used (for callers that cannot allocate; see include/csa.h)."""
     L = load()
@@ -303,7 +386,7 @@ def csa_attend_noalloc(q, kv, idx, win, q_pos, W: int, scale: float, eps: float 
     N, rows, k = kv.shape[1], win.shape[1], idx.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _sinks(sinks, H), _p(kv), N, _p(idx), k, _p(win), int(win_pos0),
+    _check(L.csa_attend_noalloc(_p(q), _p(q_gain), _sinks(sinks, H), *_rope(rope, D), _p(kv), N, _p(idx), k, _p(win), int(win_pos0),
                                 rows, W,
                                 _p(q_pos), batch, nq, H, D, float(scale), float(eps), _p(out), _stream()),
            "csa_attend_noalloc")

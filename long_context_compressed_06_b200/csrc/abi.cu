@@ -195,24 +195,28 @@ size_t csa_attend_workspace_bytes(int batch, int nq, int H, int D, long long max
     return csa::attend_workspace_bytes(batch, nq, H, D, max_keys);
 }
 
-static int validate_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+static int validate_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                           const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                            const uint16_t *win, long long win_pos0, long long win_rows, int W, const int *q_pos,
                            int batch, int nq, int H, int D, float eps, const void *out) {
     if (!al16(q) || !al16(kv) || !al16(win) || !al4(q_pos) || !al16(out)) return CSA_ERR_INVALID;
     if ((q_gain && !al4(q_gain)) || (sinks && !al4(sinks))) return CSA_ERR_INVALID;
+    if ((rope_cos == nullptr) != (rope_sin == nullptr)) return CSA_ERR_INVALID;
+    if (rope_cos && (!al4(rope_cos) || !al4(rope_sin) || rope_positions < 1)) return CSA_ERR_INVALID;
     if (batch < 1 || nq < 1 || N < 1 || win_pos0 < 0 || win_rows < 1 || W < 1 || H < 1 || D < 1 || !(eps >= 0.f))
         return CSA_ERR_INVALID;
     if (H > 128 || !(D == 64 || D == 128 || D == 256 || D == 512)) return CSA_ERR_UNSUPPORTED;
     return CSA_OK;
 }
 
-int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N,
+int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                const int *idx, int k,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W, const int *q_pos, int batch,
                int nq, int H, int D, float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes,
                void *stream) {
-    int rc = validate_attend(q, q_gain, sinks, kv, N, win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps,
-                             out);
+    int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, win_src, win_pos0,
+                             win_rows, W, q_pos, batch, nq, H, D, eps, out);
     if (rc != CSA_OK) return rc;
     if (k < 0 || (k > 0 && !al4(idx))) return CSA_ERR_INVALID;
     if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, (long long)k + W) ||
@@ -220,17 +224,18 @@ int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
         return CSA_ERR_WORKSPACE;
     csa::DevCtx ctx;
     if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
-    return csa::launch_attend(q, q_gain, sinks, kv, N, 1, k > 0 ? idx : nullptr, k, false, win_src, win_pos0,
+    return csa::launch_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, nullptr, kv, N, 1, k > 0 ? idx : nullptr, k, false, win_src, win_pos0,
                               win_rows, W,
                               q_pos, batch, nq, H, D, scale, eps, out, workspace, workspace_bytes, ctx, S(stream));
 }
 
-int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+               const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N, int m,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W, const int *q_pos, int batch,
                int nq, int H, int D, float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes,
                void *stream) {
-    int rc = validate_attend(q, q_gain, sinks, kv, N, win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps,
-                             out);
+    int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, win_src, win_pos0,
+                             win_rows, W, q_pos, batch, nq, H, D, eps, out);
     if (rc != CSA_OK) return rc;
     if (m < 1) return CSA_ERR_INVALID;
     if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, N + W) ||
@@ -238,9 +243,68 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
         return CSA_ERR_WORKSPACE;
     csa::DevCtx ctx;
     if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
-    return csa::launch_attend(q, q_gain, sinks, kv, N, m, nullptr, 0, true, win_src, win_pos0, win_rows, W, q_pos,
+    return csa::launch_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, nullptr, kv, N, m, nullptr, 0, true, win_src, win_pos0, win_rows, W, q_pos,
                               batch,
                               nq, H, D, scale, eps, out, workspace, workspace_bytes, ctx, S(stream));
+}
+
+int csa_quantize_fp8_kv(const uint16_t *x, long long rows, int d, uint8_t *codes, uint8_t *exps, void *stream) {
+    if (!al16(x) || !al16(codes) || !exps) return CSA_ERR_INVALID;
+    if (rows < 0 || d < 128 || d % 128 != 0) return CSA_ERR_INVALID;
+    return csa::launch_quantize_fp8_kv(x, rows, d, codes, exps, S(stream));
+}
+
+static int validate_fp8kv(const uint8_t *kv8, const uint8_t *kv8_exp, const uint8_t *win8, const uint8_t *win8_exp,
+                          int D) {
+    if (!al16(kv8) || !al16(win8) || !kv8_exp || !win8_exp) return CSA_ERR_INVALID;
+    if (D % 128 != 0) return CSA_ERR_UNSUPPORTED;
+    return CSA_OK;
+}
+
+int csa_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, const int *idx, int k, const uint8_t *win8, const uint8_t *win8_exp,
+                     long long win_pos0, long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
+                     float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions,
+                             reinterpret_cast<const uint16_t *>(kv8), N, reinterpret_cast<const uint16_t *>(win8),
+                             win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    if (rc != CSA_OK) return rc;
+    rc = validate_fp8kv(kv8, kv8_exp, win8, win8_exp, D);
+    if (rc != CSA_OK) return rc;
+    if (k < 0 || (k > 0 && !al4(idx))) return CSA_ERR_INVALID;
+    if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, (long long)k + W) ||
+        (workspace_bytes > 0 && !al16(workspace)))
+        return CSA_ERR_WORKSPACE;
+    csa::DevCtx ctx;
+    if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
+    const csa::Fp8Kv f8 = {kv8, kv8_exp, win8, win8_exp};
+    return csa::launch_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, &f8, nullptr, N, 1,
+                              k > 0 ? idx : nullptr, k, false, nullptr, win_pos0, win_rows, W, q_pos, batch, nq, H, D,
+                              scale, eps, out, workspace, workspace_bytes, ctx, S(stream));
+}
+
+int hca_attend_fp8kv(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                     const float *rope_sin, long long rope_positions, const uint8_t *kv8, const uint8_t *kv8_exp,
+                     long long N, int m, const uint8_t *win8, const uint8_t *win8_exp, long long win_pos0,
+                     long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D, float scale,
+                     float eps, uint16_t *out, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions,
+                             reinterpret_cast<const uint16_t *>(kv8), N, reinterpret_cast<const uint16_t *>(win8),
+                             win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    if (rc != CSA_OK) return rc;
+    rc = validate_fp8kv(kv8, kv8_exp, win8, win8_exp, D);
+    if (rc != CSA_OK) return rc;
+    if (m < 1) return CSA_ERR_INVALID;
+    if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, N + W) ||
+        (workspace_bytes > 0 && !al16(workspace)))
+        return CSA_ERR_WORKSPACE;
+    csa::DevCtx ctx;
+    if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
+    const csa::Fp8Kv f8 = {kv8, kv8_exp, win8, win8_exp};
+    return csa::launch_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, &f8, nullptr, N, m, nullptr, 0,
+                              true, nullptr, win_pos0, win_rows, W, q_pos, batch, nq, H, D, scale, eps, out,
+                              workspace, workspace_bytes, ctx, S(stream));
 }
 
 }  // extern "C"

@@ -19,12 +19,12 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(AttendArgs a) {
     const long long bq = blockIdx.x;
     const int h = blockIdx.y;
     const int i = threadIdx.x * 4;
-    if (i >= a.D) return;
+    const bool active = i < a.D;  // no early exit: the RoPE shuffles need whole warps
     float M = -INFINITY;
     for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((size_t)s * a.n_bq + bq) * a.H + h].x);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < a.splits; ++s) {
+    for (int s = 0; s < a.splits && active; ++s) {
         const size_t off = ((size_t)s * a.n_bq + bq) * a.H + h;
         const float2 ml = a.part_ml[off];
         const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
@@ -38,9 +38,27 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(AttendArgs a) {
     // the head's sink logit (natural units; the partials are in log2 units)
     if (a.sinks) L += exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - M);
     const float inv = L > 0.f ? 1.0f / L : 0.f;
+    float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    if (a.rope_cos) {
+        // conjugate rotation of the trailing kRopeDim channels: channel D-64+j pairs
+        // with D-32+j, 8 threads (32 channels) away in the same warp
+        float pv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 8);
+        if (active && i >= a.D - kRopeDim) {
+            const long long t = __ldg(a.q_pos + bq);
+            const bool first = i < a.D - kRopeDim / 2;
+            const int i0 = (i - (a.D - kRopeDim)) & (kRopeDim / 2 - 1);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 cs = rope_cs(a, t, i0 + e);
+                o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
+            }
+        }
+    }
+    if (!active) return;
     uint16_t *dst = a.out + ((size_t)bq * a.H + h) * a.D + i;
-    *reinterpret_cast<uint2 *>(dst) =
-        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
 }
 
 size_t ws_bytes_for(long long n_bq, int H, int D, int splits) {
@@ -79,13 +97,18 @@ size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_key
     return ws_bytes_for(n_bq, H, D, splits);
 }
 
-int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                  const float *rope_sin, long long rope_npos, const Fp8Kv *fp8, const uint16_t *kv, long long N, int m,
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
                   size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
     AttendArgs a = {};
-    a.q = q; a.q_gain = q_gain; a.sinks = sinks; a.kv = kv; a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
+    a.q = q; a.q_gain = q_gain; a.sinks = sinks; a.rope_cos = rope_cos; a.rope_sin = rope_sin;
+    a.rope_npos = rope_npos; a.kv = kv;
+    if (fp8) {
+        a.kv8 = fp8->kv; a.kv8e = fp8->kv_exp; a.win8 = fp8->win; a.win8e = fp8->win_exp;
+    } a.N = N; a.m = m; a.idx = idx; a.k = k; a.dense = dense;
     a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
     a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
     if (a.n_bq == 0) return CSA_OK;
@@ -99,6 +122,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(float));
     }
     if (attend_tc_supported(H, D)) return launch_attend_tc(a, ctx, st);
+    if (rope_cos || fp8) return CSA_ERR_UNSUPPORTED;  // the CUDA-core kernel has neither RoPE nor FP8 rows
     return launch_attend_simt(a, st);
 }
 

@@ -40,8 +40,9 @@ void *scratch_on_current_device() {
 
 }  // namespace
 
-extern "C" int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv,
-                                  long long N,
+extern "C" int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const float *sinks,
+                                  const float *rope_cos, const float *rope_sin, long long rope_positions,
+                                  const uint16_t *kv, long long N,
                                   const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                                   long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
                                   float scale, float eps, uint16_t *out, void *stream) {
@@ -50,6 +51,6 @@ extern "C" int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const 
     if (need > (size_t)CSA_ATTEND_NOALLOC_MAX_BYTES) return CSA_ERR_WORKSPACE;
     void *scratch = scratch_on_current_device();
     if (!scratch) return CSA_ERR_CUDA;
-    return csa_attend(q, q_gain, sinks, kv, N, idx, k, win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, scale, eps,
+    return csa_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, idx, k, win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, scale, eps,
                       out, scratch, (size_t)CSA_ATTEND_NOALLOC_MAX_BYTES, stream);
 }

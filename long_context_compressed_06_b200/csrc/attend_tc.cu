@@ -164,10 +164,12 @@ CSA_DEVINL Keys query_keys(const AttendArgs &a, long long t) {
     return k;
 }
 
-// Row of key e and whether it takes part (keys past e_end, selection padding
-// and out-of-range indices read a valid row; their scores are masked).
-CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
-                                    long long e_end, bool &valid) {
+// Row of key e -- its index in kv (win == false) or in the window buffer --
+// and whether it takes part (keys past e_end, selection padding and
+// out-of-range indices read a valid row; their scores are masked).
+CSA_DEVINL size_t key_row_index(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
+                                long long e_end, bool &valid, bool &win) {
+    win = false;
     valid = e < e_end;
     if (!valid) e = e_end - 1;  // e_end >= 1 whenever a tile exists
     if (e < ks.nsel4) {
@@ -181,13 +183,48 @@ CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long lo
         } else {
             valid = false;
         }
-        return a.kv + ((size_t)b * a.N + j) * a.D;
+        return (size_t)b * a.N + j;
     }
     long long w = e - ks.nsel4;
     if (w >= ks.nwin) valid = false;
     w = w < ks.nwin ? w : ks.nwin - 1;
     w = w < 0 ? 0 : w;
-    return a.win + ((size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + w) * a.D;
+    win = true;
+    return (size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + w;
+}
+
+CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
+                                    long long e_end, bool &valid) {
+    bool win;
+    const size_t r = key_row_index(a, ks, b, bq, e, e_end, valid, win);
+    return (win ? a.win : a.kv) + r * a.D;
+}
+
+// FP8 rows: the codes of key e (the row's exponent bytes follow from the same index)
+CSA_DEVINL const uint8_t *key_slot8(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
+                                    long long e_end, bool &valid, const uint8_t *&exps) {
+    bool win;
+    const size_t r = key_row_index(a, ks, b, bq, e, e_end, valid, win);
+    exps = (win ? a.win8e : a.kv8e) + r * (a.D / 128);
+    return (win ? a.win8 : a.kv8) + r * a.D;
+}
+
+// 8 e4m3 codes times 2^(e - 127) -> 8 bf16, exactly: e4m3 -> f16 is exact, the
+// power-of-two scale is exact in fp32, and the product has at most 4
+// significant bits inside bf16's range (the quantiser keeps e in [3, 246]).
+CSA_DEVINL uint4 e4m3x8_bf16x8(uint2 raw, uint32_t e) {
+    const float sc = __uint_as_float(e << 23);
+    const uint32_t w[2] = {raw.x, raw.y};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)(w[i >> 1] >> (16 * (i & 1)))));
+        const float lo = __half2float(__ushort_as_half((unsigned short)(h & 0xffffu))) * sc;
+        const float hi = __half2float(__ushort_as_half((unsigned short)(h >> 16))) * sc;
+        o[i] = pack_bf16x2(lo, hi);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Warp-uniform bounded wait.  Every lane polls and the outcome is voted: a
@@ -214,9 +251,15 @@ struct QLanes {
     static constexpr int PASSES = (kHeads / 4) / RPI;
 };
 
+// With partial RoPE the row's last kRopeDim / 8 units (all in a lane's last
+// unit slot, since kRopeDim <= D) rotate after the gain: unit r0 + j pairs
+// with r0 + j + 4, held by lane ^ 4 in the same slot, so one shuffle fetches
+// the partner values.
 template <int D>
-CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8]) {
+CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8],
+                            long long t) {
     using QL = QLanes<D>;
+    static_assert(D >= kRopeDim && kRopeDim / 8 == 8, "rope units: 8 per row, partners 4 units apart");
     const int lane = threadIdx.x & 31;
     const int sub = lane / QL::LPR, ul = lane % QL::LPR;
 #pragma unroll 4
@@ -238,12 +281,28 @@ CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const fl
         for (int o = QL::LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
 #pragma unroll
-        for (int u = 0; u < QL::UPL; ++u) {
-            float y[8];
+        for (int u = 0; u < QL::UPL; ++u)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = x[u][e] * r * g[u][e];
-            *ptr[u] = pack8(y);
+            for (int e = 0; e < 8; ++e) x[u][e] = x[u][e] * r * g[u][e];
+        if (a.rope_cos) {  // uniform over the grid: every lane takes the shuffles
+            constexpr int u = QL::UPL - 1;
+            constexpr int r0 = QL::UR - kRopeDim / 8;  // first rotated unit
+            const int unit = ul + u * QL::LPR;
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, x[u][e], 4);
+            if (unit >= r0) {
+                const bool first = unit < r0 + 4;  // first half of the rotated slice
+                const int i0 = ((unit - r0) & 3) * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float2 cs = rope_cs(a, t, i0 + e);
+                    x[u][e] = first ? x[u][e] * cs.x - pv[e] * cs.y : x[u][e] * cs.x + pv[e] * cs.y;
+                }
+            }
         }
+#pragma unroll
+        for (int u = 0; u < QL::UPL; ++u) *ptr[u] = pack8(x[u]);
     }
 }
 
@@ -273,7 +332,7 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
     return it;
 }
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const AttTcParams p) {
     using Lt = Layout<D>;
@@ -347,28 +406,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = (int)(g % p.stages);
                 const long long ebase = it.e0 + (long long)j * kTileKeys;
                 bool v0, v1;
-                const uint16_t *r0 = key_slot(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0);
-                const uint16_t *r1 = key_slot(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1);
+                const uint16_t *r0 = nullptr, *r1 = nullptr;
+                const uint8_t *c0 = nullptr, *c1 = nullptr, *x0 = nullptr, *x1 = nullptr;
+                if constexpr (FP8) {
+                    c0 = key_slot8(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0, x0);
+                    c1 = key_slot8(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1, x1);
+                } else {
+                    r0 = key_slot(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0);
+                    r1 = key_slot(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1);
+                }
                 const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
                 if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag)) {
                     ok = false;
                     break;
                 }
                 const uint32_t stage = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+                if constexpr (FP8) {
+                    // FP8 rows: lane l converts the 8 codes of each of its 16-byte output units
+                    // (8 bytes in, 8 bf16 out) and stores them where cp.async would have put the
+                    // bf16 row; the async-proxy fence orders the stores before the MMA reads them.
 #pragma unroll 2
-                for (int key = pw; key < kTileKeys; key += kProducerWarps) {
-                    const uint16_t *row = reinterpret_cast<const uint16_t *>(
-                        __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? r0 : r1), key & 31));
-                    const uint32_t krow = stage + key * 128;
+                    for (int key = pw; key < kTileKeys; key += kProducerWarps) {
+                        const uint8_t *crow = reinterpret_cast<const uint8_t *>(
+                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? c0 : c1), key & 31));
+                        const uint8_t *xrow = reinterpret_cast<const uint8_t *>(
+                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? x0 : x1), key & 31));
+                        const uint32_t krow = stage + key * 128;
 #pragma unroll
-                    for (int u = lane; u < D / 8; u += 32) {  // 16-byte units of the row
-                        const uint32_t dst = krow + (u >> 3) * (kTileKeys * 128) + (((u & 7) ^ (key & 7)) << 4);
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(row + u * 8)
-                                     : "memory");
+                        for (int u = lane; u < D / 8; u += 32) {
+                            const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(crow + u * 8));
+                            const uint4 v = e4m3x8_bf16x8(raw, __ldg(xrow + (u >> 4)));
+                            const uint32_t dst = krow + (u >> 3) * (kTileKeys * 128) + (((u & 7) ^ (key & 7)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
+                                         "r"(v.z), "r"(v.w)
+                                         : "memory");
+                        }
                     }
+                    tc::fence_proxy_async_smem();
+                    mbar_arrive(smem_u32(s.kfull + st));
+                } else {
+#pragma unroll 2
+                    for (int key = pw; key < kTileKeys; key += kProducerWarps) {
+                        const uint16_t *row = reinterpret_cast<const uint16_t *>(
+                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? r0 : r1), key & 31));
+                        const uint32_t krow = stage + key * 128;
+#pragma unroll
+                        for (int u = lane; u < D / 8; u += 32) {  // 16-byte units of the row
+                            const uint32_t dst = krow + (u >> 3) * (kTileKeys * 128) + (((u & 7) ^ (key & 7)) << 4);
+                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(row + u * 8)
+                                         : "memory");
+                        }
+                    }
+                    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
+                                 : "memory");
                 }
-                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
-                             : "memory");
                 if (pw == 0) {  // the mask travels with the tile (release by lane 0's arrive)
                     if (lane == 0) s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
                     mbar_arrive(smem_u32(s.kfull + st), lane == 0);
@@ -491,7 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = work_item(p, wi);
             const int h = it.head0 + hl;
             if (!warp_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag)) break;
-            normalize_q<D>(a, s, sp, qg);
+            const long long tq = __ldg(a.q_pos + it.bq);
+            normalize_q<D>(a, s, sp, qg, tq);
             tc::fence_proxy_async_smem();
             mbar_arrive(smem_u32(s.qready));
 
@@ -610,7 +702,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
                         const float4 hi =
                             *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
-                        const float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        if (a.rope_cos && c == D - kRopeDim) {
+                            // conjugate rotation of the rotated slice (this 64-column slab):
+                            // column 8*cu + e pairs with 8*(cu ^ 4) + e, held by lane ^ 4
+                            float pv[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
+                            const bool first = cu < 4;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float2 cs = rope_cs(a, tq, (cu & 3) * 8 + e);
+                                o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
+                            }
+                        }
                         if (hr < a.H)
                             *reinterpret_cast<uint4 *>(a.out + ((size_t)it.bq * a.H + hr) * D + c + 8 * cu) = pack8(o);
                     }
@@ -647,7 +752,7 @@ constexpr uint32_t idesc_m64(int n, bool b_mn) {
            ((uint32_t)(64 >> 4) << 24);
 }
 
-template <int D>
+template <int D, bool FP8>
 int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
     AttTcParams p = {};
     p.a = a;
@@ -661,7 +766,7 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
     p.stages = stages;
     // at least 120 KiB so that one CTA owns an SM (it allocates all 512 TMEM columns)
     const size_t smem = std::max<size_t>(smem_bytes<D>(stages), 120 * 1024);
-    auto kern = attend_tc_kernel<D>;
+    auto kern = attend_tc_kernel<D, FP8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
     CUtensorMap qmap;
@@ -709,11 +814,19 @@ void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long
 }
 
 int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st) {
+    if (a.kv8) {  // FP8 rows: 128-channel scale blocks
+        switch (a.D) {
+            case 128: return launch_d<128, true>(a, ctx, st);
+            case 256: return launch_d<256, true>(a, ctx, st);
+            case 512: return launch_d<512, true>(a, ctx, st);
+            default: return CSA_ERR_UNSUPPORTED;
+        }
+    }
     switch (a.D) {
-        case 64: return launch_d<64>(a, ctx, st);
-        case 128: return launch_d<128>(a, ctx, st);
-        case 256: return launch_d<256>(a, ctx, st);
-        case 512: return launch_d<512>(a, ctx, st);
+        case 64: return launch_d<64, false>(a, ctx, st);
+        case 128: return launch_d<128, false>(a, ctx, st);
+        case 256: return launch_d<256, false>(a, ctx, st);
+        case 512: return launch_d<512, false>(a, ctx, st);
         default: return CSA_ERR_UNSUPPORTED;
     }
 }

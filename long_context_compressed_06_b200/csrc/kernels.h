@@ -19,6 +19,8 @@ int launch_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t
                             const float *gain, float eps, long long i0, long long ni, long long n_out,
                             uint16_t *out, cudaStream_t st);
 
+int launch_quantize_fp8_kv(const uint16_t *x, long long rows, int d, uint8_t *codes, uint8_t *exps, cudaStream_t st);
+
 int launch_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos,
                  int batch, int nq, long long N, int H_I, int d_I, int m, float *scores,
                  const DevCtx &ctx, cudaStream_t st);
@@ -49,7 +51,14 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
 // Attention: dense selects the HCA key set of the first n_vis(t) entries;
 // otherwise the k selected entries idx (may be null when k == 0).
 size_t attend_workspace_bytes(int batch, int nq, int H, int D, long long max_keys);
-int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const uint16_t *kv, long long N, int m,
+// The FP8 KV cache of one attention call: e4m3 codes and UE8M0 exponent
+// bytes of the compressed entries and of the window rows.
+struct Fp8Kv {
+    const uint8_t *kv, *kv_exp, *win, *win_exp;
+};
+
+int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                  const float *rope_sin, long long rope_npos, const Fp8Kv *fp8, const uint16_t *kv, long long N, int m,
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,

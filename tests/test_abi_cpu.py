@@ -94,6 +94,33 @@ def test_compress_dynamic_validation(lib):
     assert call(i0=big, ni=1, n_out=big) == csa.CSA_ERR_INVALID
 
 
+def test_fp8_kv_validation(lib):
+    f = lib.csa_quantize_fp8_kv
+    assert f(NULL, 4, 512, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 512, MIS, A16, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 512, A16b, NULL, NULL) == csa.CSA_ERR_INVALID
+    assert f(A16, 4, 192, A16b, A16, NULL) == csa.CSA_ERR_INVALID     # d % 128
+    assert f(A16, -1, 512, A16b, A16, NULL) == csa.CSA_ERR_INVALID
+    g = lib.csa_attend_fp8kv
+    # (q, g, sinks, rc, rs, rn, kv8, kv8e, N, idx, k, win8, win8e, p0, rows, W, pos, b, nq, H, D, scale, eps, out, ws, wsb, st)
+    base = [A16, NULL, NULL, NULL, NULL, 0, A16, A16, 300, A16, 64, A16, A16, 0, 2048, 16, A16, 1, 1, 8, 512, 0.125,
+            1e-6, A16b, NULL, 0, NULL]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return g(*a)
+
+    assert call(a6=MIS) == csa.CSA_ERR_INVALID          # codes misaligned
+    assert call(a7=NULL) == csa.CSA_ERR_INVALID         # exponents missing
+    assert call(a12=NULL) == csa.CSA_ERR_INVALID        # window exponents missing
+    assert call(a20=64) == csa.CSA_ERR_UNSUPPORTED      # D = 64: no whole 128-channel block
+    h = lib.hca_attend_fp8kv
+    assert h(A16, NULL, NULL, NULL, NULL, 0, A16, A16, 300, 0, A16, A16, 0, 2048, 16, A16, 1, 1, 8, 512, 0.125, 1e-6,
+             A16b, NULL, 0, NULL) == csa.CSA_ERR_INVALID    # m
+
+
 def test_index_validation(lib):
     f = lib.csa_index
     ok = (A16, A16, A16, A16)
@@ -140,16 +167,21 @@ def test_rescore_validation_and_workspace(lib):
 
 def test_attend_validation_and_workspace(lib):
     f = lib.csa_attend
-    args = dict(q=A16, g=NULL, sk=NULL, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048, W=16, pos=A16, b=1, nq=1, H=8,
-                D=64, scale=0.125, eps=1e-6, out=A16b)
+    args = dict(q=A16, g=NULL, sk=NULL, rc=NULL, rs=NULL, rn=0, kv=A16, N=300, idx=A16, k=64, win=A16, p0=0, T=2048,
+                W=16, pos=A16, b=1, nq=1, H=8, D=64, scale=0.125, eps=1e-6, out=A16b)
 
     def call(ws=NULL, wsb=0, **kw):
         a = dict(args, **kw)
-        return f(a["q"], a["g"], a["sk"], a["kv"], a["N"], a["idx"], a["k"], a["win"], a["p0"], a["T"], a["W"], a["pos"],
-                 a["b"], a["nq"], a["H"], a["D"], a["scale"], a["eps"], a["out"], ws, wsb, NULL)
+        return f(a["q"], a["g"], a["sk"], a["rc"], a["rs"], a["rn"], a["kv"], a["N"], a["idx"], a["k"], a["win"],
+                 a["p0"], a["T"], a["W"], a["pos"], a["b"], a["nq"], a["H"], a["D"], a["scale"], a["eps"], a["out"],
+                 ws, wsb, NULL)
 
     assert call(q=NULL) == csa.CSA_ERR_INVALID
     assert call(sk=ctypes.c_void_p(0x10002)) == csa.CSA_ERR_INVALID    # sinks not 4-byte aligned
+    assert call(rc=A16, rn=100) == csa.CSA_ERR_INVALID                 # rope cos without sin
+    assert call(rs=A16, rn=100) == csa.CSA_ERR_INVALID                 # rope sin without cos
+    assert call(rc=A16, rs=ctypes.c_void_p(0x10002), rn=100) == csa.CSA_ERR_INVALID
+    assert call(rc=A16, rs=A16b, rn=0) == csa.CSA_ERR_INVALID          # empty tables
     assert call(W=0) == csa.CSA_ERR_INVALID
     assert call(p0=-1) == csa.CSA_ERR_INVALID
     assert call(T=0) == csa.CSA_ERR_INVALID
@@ -160,8 +192,8 @@ def test_attend_validation_and_workspace(lib):
     assert call(ws=A16, wsb=need - 1, k=1024) == csa.CSA_ERR_WORKSPACE
     assert call(ws=MIS, wsb=need, k=1024) == csa.CSA_ERR_WORKSPACE
     h = lib.hca_attend
-    assert h(A16, NULL, NULL, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b, NULL, 0,
-             NULL) == csa.CSA_ERR_INVALID    # m
+    assert h(A16, NULL, NULL, NULL, NULL, 0, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b,
+             NULL, 0, NULL) == csa.CSA_ERR_INVALID    # m
     # workspace sizing is monotone in the key count and batch
     assert lib.csa_attend_workspace_bytes(8, 1, 128, 512, 1152) >= lib.csa_attend_workspace_bytes(1, 1, 128, 512, 1152)
 

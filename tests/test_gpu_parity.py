@@ -353,6 +353,157 @@ def test_hca_attend_sinks_parity(cuda):
     assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
 
 
+def _rope_tables(n_pos, base=10000.0):
+    """cos / sin [n_pos][32] of angles p * base^(-i/32) (the 64 rotated channels' 32 pairs)."""
+    om = base ** (-np.arange(32) / 32.0)
+    ang = np.arange(n_pos)[:, None] * om[None, :]
+    c = torch.from_numpy(np.cos(ang).astype(np.float32)).to(DEV)
+    s = torch.from_numpy(np.sin(ang).astype(np.float32)).to(DEV)
+    return c, s
+
+
+@pytest.mark.parametrize("batch,nq,H,D,N,T,k,Wn,m,ts,sinks", [
+    (8, 1, 128, 512, 4096, 16384, 1024, 128, 4, [16383] * 8, False),     # key splits + merge
+    (1, 3, 128, 256, 300, 1200, 64, 16, 4, [1199, 700, 5], True),        # one split per query, with sinks
+    (2, 1, 40, 128, 97, 400, 33, 7, 4, [399, 13], False),                # ragged heads
+    (1, 2, 8, 64, 512, 2048, 64, 16, 4, [2047, 1000], False),            # D = 64: every channel rotates
+    (1, 64, 128, 512, 1024, 4096, 64, 32, 4, [4095 - 5 * i for i in range(64)], False),   # single split, bf16 epilogue
+])
+def test_csa_attend_rope_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts, sinks):
+    """Partial RoPE (techniques map "Partial RoPE", rope-conjugate output):
+    the 64 trailing channels of the normalised query rotate at its position,
+    the output gets the conjugate rotation; keys are inputs as they stand."""
+    q = seeded((batch, nq, H, D), 90)
+    kv = seeded((batch, N, D), 91)
+    win = seeded((batch, T, D), 92)
+    qp = positions(batch, nq, ts)
+    idx = _random_selection(batch, nq, k, ts, m, N, 93)
+    sk = (seeded((H,), 94, "uniform") * 6.0 - 3.0).contiguous() if sinks else None
+    cos, sin = _rope_tables(T)
+    scale = 1.0 / np.sqrt(D)
+    out = cuda.csa_attend(q, kv, torch.from_numpy(idx).to(DEV), win, qp, Wn, scale, sinks=sk, rope=(cos, sin))
+    ref = oracle.attend(bits(q), bits(kv), idx, bits(win), qp.cpu().numpy(), Wn, scale,
+                        sinks=None if sk is None else sk.cpu().numpy(), rope=(cos.cpu().numpy(), sin.cpu().numpy()))
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+    # the rotation is not a no-op on these inputs
+    plain = oracle.attend(bits(q), bits(kv), idx, bits(win), qp.cpu().numpy(), Wn, scale,
+                          sinks=None if sk is None else sk.cpu().numpy())
+    assert np.abs(plain - ref).max() > 0.05 * np.abs(ref).max()
+
+
+def test_attend_rope_paths_cover_split_and_single(cuda):
+    """The two output paths the rotation lives in: the merge kernel (several key
+    splits) and the attention kernel's own bf16 epilogue (one split)."""
+    assert cuda.attend_workspace_bytes(8, 1, 128, 512, 1024 + 128) > 0
+    assert cuda.attend_workspace_bytes(1, 64, 128, 512, 64 + 32) == 0
+
+
+def test_attend_rope_outside_the_table_is_unrotated_and_noalloc_agrees(cuda):
+    batch, nq, H, D, N, T, k, Wn, m = 2, 1, 128, 512, 600, 2400, 128, 64, 4
+    q = seeded((batch, nq, H, D), 95)
+    kv = seeded((batch, N, D), 96)
+    win = seeded((batch, T, D), 97)
+    qp = positions(batch, nq, [2399, 1500])
+    idx = torch.from_numpy(_random_selection(batch, nq, k, [2399, 1500], m, N, 98)).to(DEV)
+    cos, sin = _rope_tables(2000)            # position 2399 lies outside, 1500 inside
+    out = cuda.csa_attend(q, kv, idx, win, qp, Wn, D ** -0.5, rope=(cos, sin))
+    plain = cuda.csa_attend(q, kv, idx, win, qp, Wn, D ** -0.5)
+    assert torch.equal(out[0], plain[0])
+    assert not torch.equal(out[1], plain[1])
+    na = cuda.csa_attend_noalloc(q, kv, idx, win, qp, Wn, D ** -0.5, rope=(cos, sin))
+    assert torch.equal(na, out)
+
+
+def test_hca_attend_rope_parity(cuda):
+    batch, H, D, N, m, Wn = 4, 128, 512, 700, 128, 128
+    T = N * m
+    q = seeded((batch, 1, H, D), 99)
+    kv = seeded((batch, N, D), 100)
+    win = seeded((batch, Wn, D), 101)
+    qp = positions(batch, 1, [T - 1, T - 1, 300 * 128 + 5, T - 2])
+    cos, sin = _rope_tables(T)
+    out = cuda.hca_attend(q, kv, m, win, qp, Wn, D ** -0.5, win_pos0=T - Wn, rope=(cos, sin))
+    ref = oracle.hca_attend(bits(q), bits(kv), m, bits(win), qp.cpu().numpy(), Wn, D ** -0.5, win_pos0=T - Wn,
+                            rope=(cos.cpu().numpy(), sin.cpu().numpy()))
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
+# FP8 KV cache (techniques map, inference quantization): e4m3 codes, power-of-two block scales
+def _fp8_inputs(shape, seed):
+    x = seeded(shape, seed).float()
+    x = x * torch.exp(torch.linspace(-3, 3, shape[-2], device=DEV))[:, None]    # rows of different sizes
+    return x.to(torch.bfloat16)
+
+
+def test_quantize_fp8_kv_bit_exact(cuda):
+    x = _fp8_inputs((3, 77, 512), 110)
+    x[0, 5, 128:256] = 0.0                                   # an all-zero block
+    x[1, 9, :128] = 2.0 ** -30                               # a tiny block
+    x[2, 3, 256:384] = -(2.0 ** 100)                         # a huge block
+    x[2, 4, 384:] = 1.9921875 * 2.0 ** 127                   # saturates at the exponent ceiling
+    codes, exps = cuda.csa_quantize_fp8_kv(x)
+    rc, re_ = oracle.quantize_fp8_kv(bits(x), 128)
+    assert np.array_equal(exps.cpu().numpy(), re_)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+def _oracle_fp8(x):
+    """oracle codes / exponents of bf16 rows, and the dequantised rows as bf16 bits (exact)."""
+    c, e = oracle.quantize_fp8_kv(bits(x), 128)
+    dq = oracle.dequantize_fp8_kv(c, e, 128)
+    dq_bits = W.bits(torch.from_numpy(dq).to(torch.bfloat16))
+    return c, e, dq_bits
+
+
+def _dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    return t if dtype is None else t.view(dtype)
+
+
+@pytest.mark.parametrize("batch,nq,H,D,N,T,k,Wn,m,ts", [
+    (8, 1, 128, 512, 4096, 16384, 1024, 128, 4, [16383] * 8),          # key splits + merge
+    (1, 64, 128, 512, 1024, 4096, 64, 32, 4, [4095 - 5 * i for i in range(64)]),   # one split
+    (2, 1, 40, 128, 97, 400, 33, 7, 4, [399, 13]),                     # ragged heads, D = 128
+    (1, 3, 128, 256, 300, 1200, 64, 16, 4, [1199, 700, 5]),
+])
+def test_csa_attend_fp8kv_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts):
+    """The FP8 cache (quantised by the oracle) against the oracle's attention on
+    its dequantised rows, and bit for bit against the bf16 kernel on those rows
+    (the conversion in the gather is exact, so the MMA operands are the same)."""
+    q = seeded((batch, nq, H, D), 111)
+    kv = _fp8_inputs((batch, N, D), 112)
+    win = _fp8_inputs((batch, T, D), 113)
+    qp = positions(batch, nq, ts)
+    idx = _random_selection(batch, nq, k, ts, m, N, 114)
+    kc, ke, kdq = _oracle_fp8(kv)
+    wc, we, wdq = _oracle_fp8(win)
+    scale = 1.0 / np.sqrt(D)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    out = cuda.csa_attend_fp8kv(q, _dev(kc), _dev(ke), idx_d, _dev(wc), _dev(we), qp, Wn, scale)
+    ref = oracle.attend(bits(q), kdq, idx, wdq, qp.cpu().numpy(), Wn, scale)
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+    bf = cuda.csa_attend(q, _dev(kdq, torch.bfloat16), idx_d, _dev(wdq, torch.bfloat16), qp, Wn, scale)
+    assert torch.equal(out.view(torch.int16), bf.view(torch.int16))
+
+
+def test_hca_attend_fp8kv_parity(cuda):
+    batch, H, D, N, m, Wn = 4, 128, 512, 700, 128, 128
+    T = N * m
+    q = seeded((batch, 1, H, D), 115)
+    kv = _fp8_inputs((batch, N, D), 116)
+    win = _fp8_inputs((batch, Wn, D), 117)
+    qp = positions(batch, 1, [T - 1, T - 1, 300 * 128 + 5, 64])
+    kc, ke, kdq = _oracle_fp8(kv)
+    wc, we, wdq = _oracle_fp8(win)
+    out = cuda.hca_attend_fp8kv(q, _dev(kc), _dev(ke), m, _dev(wc), _dev(we), qp, Wn, D ** -0.5, win_pos0=T - Wn)
+    ref = oracle.hca_attend(bits(q), kdq, m, wdq, qp.cpu().numpy(), Wn, D ** -0.5, win_pos0=T - Wn)
+    got = f64(out)
+    assert np.abs(got - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
 def test_attend_running_max_rescale(cuda):
     """Entries whose norms grow along the key order (logit scale 0.01 -> 5) push
     the running max up by more than 2^8 after the first tiles (the O rescale
