@@ -161,3 +161,28 @@ def test_attend_validation_and_workspace(lib):
              NULL) == csa.CSA_ERR_INVALID    # m
     # workspace sizing is monotone in the key count and batch
     assert lib.csa_attend_workspace_bytes(8, 1, 128, 512, 1152) >= lib.csa_attend_workspace_bytes(1, 1, 128, 512, 1152)
+
+
+def test_binding_refuses_host_tensors_and_has_no_fallback():
+    """Every call takes CUDA tensors only: host tensors raise before anything is
+    computed, so no step can silently run on the CPU."""
+    import torch
+    x = torch.zeros((1, 64, 64), dtype=torch.bfloat16)
+    L = torch.zeros((8, 64), dtype=torch.float32)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        csa.csa_compress(x, x, L, 4)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        csa.csa_compress_dynamic(x, x, None, None, L, 4)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        csa.csa_index(torch.zeros((1, 1, 4, 32), dtype=torch.bfloat16), torch.zeros((1, 1, 4)),
+                      torch.zeros((1, 16, 32), dtype=torch.bfloat16), torch.zeros((1, 1), dtype=torch.int32), 4)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        csa.csa_quantize_fp4(torch.zeros((4, 64), dtype=torch.bfloat16))
+
+
+def test_missing_library_raises(monkeypatch, tmp_path):
+    from long_context_compressed_06_b200 import binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.load()
