@@ -129,14 +129,14 @@ int csa_compress_dynamic(const uint16_t *A, const uint16_t *B, const uint16_t *Z
  * Lightning Indexer": per-head weight times ReLU(q . K), summed over heads).
  *   S[b][q][s] = sum_h w[b][q][h] * max(0, q_idx[b][q][h] . k_idx[b][s])   for s < n_vis(q_pos[b][q])
  *   S[b][q][s] = -inf                                                      otherwise
- * bf16 operands on the tensor cores (d_I in {32, 64, 128, 256}; other sizes on
- * CUDA cores), fp32 accumulation and epilogue.
+ * bf16 operands on the tensor cores, fp32 accumulation and epilogue.
  *
  *   q_idx  [batch][nq][H_I][d_I] bf16     w [batch][nq][H_I] fp32
  *   k_idx  [batch][N][d_I] bf16           q_pos [batch][nq] int32 (0 <= t)
  *   scores [batch][nq][N] fp32 (output)
- * Requirements: d_I % 16 == 0, 16 <= d_I <= 256; 1 <= H_I <= 256 (padded to a
- * multiple of 16 internally); m >= 1; N >= 1.
+ * Requirements: d_I % 16 == 0, 16 <= d_I (else CSA_ERR_INVALID); d_I in
+ * {32, 64, 128, 256} and 1 <= H_I <= 256 (padded to a multiple of 16
+ * internally), else CSA_ERR_UNSUPPORTED; m >= 1; 1 <= N < 2^31.
  */
 int csa_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx,
               const int *q_pos, int batch, int nq, long long N, int H_I, int d_I,
@@ -160,9 +160,9 @@ int csa_quantize_fp4(const uint16_t *x, long long rows, int d,
 /*
  * csa_index_fp4 -- csa_index on FP4 operands (layouts of csa_quantize_fp4):
  * the score is the same formula on the dequantised values e2m1 * e4m3, with
- * exact products and fp32 accumulation.  d_I in {64, 128, 256} with k4s
- * aligned to d_I/16 bytes runs on the tensor cores (exact f16 dequantisation);
- * other shapes on CUDA cores.
+ * exact products and fp32 accumulation, on the tensor cores.  d_I in
+ * {64, 128, 256} (else CSA_ERR_UNSUPPORTED); k4s aligned to d_I/16 bytes and
+ * q4s to 2 bytes (else CSA_ERR_INVALID).
  *   q4 [batch][nq][H_I][d_I/2]   q4s [batch][nq][H_I][d_I/16]   w [batch][nq][H_I] fp32
  *   k4 [batch][N][d_I/2]         k4s [batch][N][d_I/16]         scores [batch][nq][N] fp32
  * Requirements: as csa_index.
@@ -204,7 +204,9 @@ int csa_topk(const float *scores, const int *q_pos, int batch, int nq, long long
  *   q_idx [batch][nq][H_I][d_I] bf16   w [batch][nq][H_I] fp32
  *   k_idx [batch][N][d_I] bf16         cand [batch][nq][kc] int32 (from csa_topk)
  *   idx   [batch][nq][k] int32
- * Requirements: k <= 8192; kc <= 2^19; H_I * d_I * 4 <= 200 KiB.  Workspace:
+ * Requirements: k <= 8192; kc <= 2^19; H_I and d_I as csa_index (the
+ * tensor-core indexer scores the candidates; other shapes return
+ * CSA_ERR_UNSUPPORTED).  Workspace:
  * csa_rescore_workspace_bytes(batch, nq, kc, k, d_I) bytes, 256-byte aligned
  * (CSA_ERR_WORKSPACE otherwise): candidate scores, chosen positions and a copy
  * of the candidates' key rows (scored by the tensor-core indexer).
@@ -288,7 +290,11 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
  * a caller workspace then).  Nothing is allocated or freed.
  * The first call on a device looks up the array's device address on that
  * device (cudaGetSymbolAddress); make that first call before any stream
- * capture.  All calls share the array and it keeps the last call's contents
+ * capture.  That address is kept for the life of the process: after a
+ * cudaDeviceReset of a device, do not call this entry point on it again (the
+ * device status word of csa_sync_status has the same limit).  Bad arguments
+ * are reported as csa_attend reports them, before the size check.
+ * All calls share the array and it keeps the last call's contents
  * (nothing in it needs clearing: every slot read is written by the same
  * call); calls that overlap on the GPU -- different streams or host threads --
  * race on it, so serialise them.

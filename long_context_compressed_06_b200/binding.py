@@ -92,6 +92,11 @@ def _stream():
 def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> torch.Tensor:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError("%s must be a CUDA tensor" % name)
+    # every call launches on the current device: a tensor on another GPU would be
+    # read through the wrong context
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError("%s is on %s but the current device is cuda:%d (use torch.cuda.device(...))"
+                         % (name, t.device, torch.cuda.current_device()))
     if t.dtype != dtype:
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
     if not t.is_contiguous():

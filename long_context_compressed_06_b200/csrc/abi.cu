@@ -127,7 +127,7 @@ int csa_index(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, cons
     if (!al16(q_idx) || !al4(w) || !al16(k_idx) || !al4(q_pos) || !al16(scores)) return CSA_ERR_INVALID;
     if (batch < 1 || nq < 1 || N < 1 || H_I < 1 || d_I < 16 || d_I % 16 != 0 || m < 1)
         return CSA_ERR_INVALID;
-    if (H_I > 256 || d_I > 256 || N > (1LL << 31) - 1) return CSA_ERR_UNSUPPORTED;
+    if (!csa::index_tc_supported(H_I, d_I) || N > (1LL << 31) - 1) return CSA_ERR_UNSUPPORTED;
     csa::DevCtx ctx;
     if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
     return csa::launch_index(q_idx, w, k_idx, q_pos, batch, nq, N, H_I, d_I, m, scores, ctx, S(stream));
@@ -147,7 +147,10 @@ int csa_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, const u
         return CSA_ERR_INVALID;
     if (batch < 1 || nq < 1 || N < 1 || H_I < 1 || d_I < 16 || d_I % 16 != 0 || m < 1)
         return CSA_ERR_INVALID;
-    if (H_I > 256 || d_I > 256 || N > (1LL << 31) - 1) return CSA_ERR_UNSUPPORTED;
+    if (!csa::index_fp4_tc_supported(H_I, d_I) || N > (1LL << 31) - 1) return CSA_ERR_UNSUPPORTED;
+    // each key's d_I/16 scale bytes move as one copy aligned to their size
+    if (reinterpret_cast<uintptr_t>(k4s) % (uintptr_t)(d_I / 16) != 0 || reinterpret_cast<uintptr_t>(q4s) % 2 != 0)
+        return CSA_ERR_INVALID;
     csa::DevCtx ctx;
     if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
     return csa::launch_index_fp4(q4, q4s, w, k4, k4s, q_pos, batch, nq, N, H_I, d_I, m, scores, ctx,
@@ -209,16 +212,35 @@ static int validate_attend(const uint16_t *q, const float *q_gain, const float *
     return CSA_OK;
 }
 
+}  // extern "C"
+
+namespace csa {
+// The argument checks of csa_attend before its workspace check (shared with
+// csa_attend_noalloc, so that call reports a bad argument as such rather than
+// as a workspace shortfall).
+int check_attend_args(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                      const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
+                      const int *idx, int k, const uint16_t *win, long long win_pos0, long long win_rows, int W,
+                      const int *q_pos, int batch, int nq, int H, int D, float eps, const void *out) {
+    const int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, win, win_pos0,
+                                   win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    if (rc != CSA_OK) return rc;
+    if (k < 0 || (k > 0 && !al4(idx))) return CSA_ERR_INVALID;
+    return CSA_OK;
+}
+}  // namespace csa
+
+extern "C" {
+
 int csa_attend(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
                const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
                const int *idx, int k,
                const uint16_t *win_src, long long win_pos0, long long win_rows, int W, const int *q_pos, int batch,
                int nq, int H, int D, float scale, float eps, uint16_t *out, void *workspace, size_t workspace_bytes,
                void *stream) {
-    int rc = validate_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, win_src, win_pos0,
-                             win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    const int rc = csa::check_attend_args(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, idx, k,
+                                          win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps, out);
     if (rc != CSA_OK) return rc;
-    if (k < 0 || (k > 0 && !al4(idx))) return CSA_ERR_INVALID;
     if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, (long long)k + W) ||
         (workspace_bytes > 0 && !al16(workspace)))
         return CSA_ERR_WORKSPACE;

@@ -78,14 +78,15 @@ bool attend_tc_supported(int H, int D);
 void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long long *kps);
 int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st);
 
-// Split plan of the kernel that will run for these shapes (the tensor-core
-// kernel whenever it supports them).
+// Split plan of the tensor-core kernel for these shapes (one split when the
+// shapes are outside the compiled tiles: the launch then returns
+// CSA_ERR_UNSUPPORTED before using any workspace).
 static void plan_splits(long long n_bq, int H, int D, long long max_keys, int *splits, long long *kps) {
     if (attend_tc_supported(H, D)) {
         attend_tc_plan(n_bq, H, max_keys, splits, kps);
     } else {
-        *splits = attend_simt_splits(n_bq, H, max_keys);
-        *kps = (max_keys + *splits - 1) / *splits;
+        *splits = 1;
+        *kps = max_keys;
     }
 }
 
@@ -112,6 +113,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
     a.win = win; a.win_pos0 = win_pos0; a.win_rows = win_rows; a.W = W; a.q_pos = q_pos; a.nq = nq; a.n_bq = (long long)batch * nq;
     a.H = H; a.D = D; a.scale = scale; a.eps = eps; a.out = out;
     if (a.n_bq == 0) return CSA_OK;
+    if (!attend_tc_supported(H, D)) return CSA_ERR_UNSUPPORTED;
     const long long max_keys = (dense ? N : (long long)k) + W;
     plan_splits(a.n_bq, H, D, max_keys, &a.splits, &a.keys_per_split);
     const size_t need = ws_bytes_for(a.n_bq, H, D, a.splits);
@@ -121,9 +123,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
         a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(float));
     }
-    if (attend_tc_supported(H, D)) return launch_attend_tc(a, ctx, st);
-    if (rope_cos || fp8) return CSA_ERR_UNSUPPORTED;  // the CUDA-core kernel has neither RoPE nor FP8 rows
-    return launch_attend_simt(a, st);
+    return launch_attend_tc(a, ctx, st);
 }
 
 }  // namespace csa

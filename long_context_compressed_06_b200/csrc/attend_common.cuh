@@ -97,7 +97,5 @@ CSA_DEVINL void store_lane_dims(uint16_t *row, int lane, const float f[DPL]) {
 }
 
 int launch_attend_combine(const AttendArgs &a, cudaStream_t st);
-int attend_simt_splits(long long n_bq, int H, long long max_keys);
-int launch_attend_simt(const AttendArgs &a, cudaStream_t st);
 
 }  // namespace csa

@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/csa.h"
+#include "kernels.h"
 
 namespace {
 
@@ -25,7 +26,9 @@ __device__ __align__(256) unsigned char g_attend_scratch[CSA_ATTEND_NOALLOC_MAX_
 // Device address of the array on the current device.  In host code the
 // symbol is only a host-side stand-in, so the address must come from
 // cudaGetSymbolAddress; it is looked up once per device, with that device
-// current, on the first call made on it.
+// current, on the first call made on it.  The cached address outlives a
+// cudaDeviceReset of that device, after which it is stale: callers that reset
+// a device must not use this entry point on it again in the same process.
 void *scratch_on_current_device() {
     static void *cache[64] = {nullptr};
     int dev = 0;
@@ -46,7 +49,10 @@ extern "C" int csa_attend_noalloc(const uint16_t *q, const float *q_gain, const 
                                   const int *idx, int k, const uint16_t *win_src, long long win_pos0,
                                   long long win_rows, int W, const int *q_pos, int batch, int nq, int H, int D,
                                   float scale, float eps, uint16_t *out, void *stream) {
-    if (batch < 1 || nq < 1 || H < 1 || D < 1 || k < 0 || W < 1) return CSA_ERR_INVALID;
+    // the same argument checks as csa_attend first, then the array's size limit
+    const int rc = csa::check_attend_args(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, idx, k,
+                                          win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    if (rc != CSA_OK) return rc;
     const size_t need = csa_attend_workspace_bytes(batch, nq, H, D, (long long)k + W);
     if (need > (size_t)CSA_ATTEND_NOALLOC_MAX_BYTES) return CSA_ERR_WORKSPACE;
     void *scratch = scratch_on_current_device();

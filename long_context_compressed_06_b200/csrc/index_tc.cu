@@ -293,9 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// The tensor-core path takes d_I in {32, 64, 128, 256} and up to 256 heads.
+// The tensor-core path takes d_I in {32, 64, 128, 256} and up to 256 heads,
+// as long as one query's heads and two key stages fit in shared memory.
 bool index_tc_supported(int H_I, int d_I) {
-    return (d_I == 32 || d_I == 64 || d_I == 128 || d_I == 256) && H_I >= 1 && H_I <= 256;
+    if (!(d_I == 32 || d_I == 64 || d_I == 128 || d_I == 256) || H_I < 1 || H_I > 256) return false;
+    const size_t h_pad = (size_t)std::max(16, (H_I + 15) / 16 * 16);
+    return h_pad * d_I * 2 + 2 * (size_t)kTileKeys * d_I * 2 <= 200 * 1024;
 }
 
 int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,

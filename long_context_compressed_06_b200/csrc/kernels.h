@@ -43,7 +43,9 @@ int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k
                         int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *ws,
                         const DevCtx &ctx, cudaStream_t st);
 
+// Shapes the tensor-core indexers take (the only implementation).
 bool index_tc_supported(int H_I, int d_I);
+bool index_fp4_tc_supported(int H_I, int d_I);
 int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *q_pos, int batch,
                     int nq, long long N, int H_I, int d_I, int m, float *scores, const DevCtx &ctx,
                     cudaStream_t st);
@@ -65,5 +67,11 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
                   void *ws, size_t ws_bytes, const DevCtx &ctx, cudaStream_t st);
 
 int launch_selftest_wait(const DevCtx &ctx, cudaStream_t st);
+
+// Host-side argument checks of csa_attend (everything but the workspace).
+int check_attend_args(const uint16_t *q, const float *q_gain, const float *sinks, const float *rope_cos,
+                      const float *rope_sin, long long rope_positions, const uint16_t *kv, long long N,
+                      const int *idx, int k, const uint16_t *win, long long win_pos0, long long win_rows, int W,
+                      const int *q_pos, int batch, int nq, int H, int D, float eps, const void *out);
 
 }  // namespace csa

@@ -10,71 +10,16 @@
 // operands, fp32 arithmetic), and the k best candidates are kept:
 //   S_c[j] = sum_h w_h * max(0, q_I[h] . K_I[cand[j]])    (cand[j] < 0 -> -inf)
 //   idx    = cand[ top-k of S_c ]   (ascending entry order, -1 padded)
-// When the tensor-core indexer takes the shape, the candidate key rows are
-// gathered into a contiguous buffer and scored by it (each query is its own
-// sequence of kc entries, all visible), invalid slots are set to -inf, the
-// top-k selector runs over the kc scores and the chosen positions are mapped
-// back to entry indices.  Otherwise a CUDA-core kernel scores the candidates
-// in place (thread per candidate, query in shared memory).
+// The candidate key rows are gathered into a contiguous buffer and scored by
+// the tensor-core indexer (each query is its own sequence of kc entries, all
+// visible), invalid slots are set to -inf, the top-k selector runs over the kc
+// scores and the chosen positions are mapped back to entry indices.  Shapes the tensor-core indexer does not take return
+// CSA_ERR_UNSUPPORTED.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace csa {
 namespace {
-
-constexpr int kThreadsPerBlock = 128;
-
-// q_s: [H_I][d_I] fp32, w_s: [H_I]
-__global__ void __launch_bounds__(kThreadsPerBlock)
-    rescore_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
-                   const uint16_t *__restrict__ k_idx, const int *__restrict__ cand, int kc, int nq,
-                   long long N, int H_I, int d_I, float *__restrict__ sc) {
-    extern __shared__ __align__(16) float sm[];
-    float *q_s = sm;
-    float *w_s = sm + H_I * d_I;
-    const long long bq = blockIdx.y;
-    const long long b = bq / nq;
-    const uint16_t *q = q_idx + (size_t)bq * H_I * d_I;
-    for (int i = threadIdx.x; i < H_I * d_I; i += blockDim.x) q_s[i] = __uint_as_float((uint32_t)q[i] << 16);
-    for (int h = threadIdx.x; h < H_I; h += blockDim.x) w_s[h] = w[bq * H_I + h];
-    __syncthreads();
-    const int j = blockIdx.x * kThreadsPerBlock + threadIdx.x;
-    if (j >= kc) return;
-    const int c = cand[bq * kc + j];
-    float score = -INFINITY;
-    if (c >= 0 && c < N) {
-        score = 0.f;
-        const uint16_t *kr = k_idx + ((size_t)b * N + c) * d_I;
-        for (int h0 = 0; h0 < H_I; h0 += 16) {
-            float acc[16];
-#pragma unroll
-            for (int h = 0; h < 16; ++h) acc[h] = 0.f;
-            for (int d0 = 0; d0 < d_I; d0 += 16) {
-                float kf[16];
-                unpack8(ldg16(kr + d0), kf);
-                unpack8(ldg16(kr + d0 + 8), kf + 8);
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    if (h0 + h < H_I) {
-                        const float4 *qv = reinterpret_cast<const float4 *>(q_s + (size_t)(h0 + h) * d_I + d0);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            const float4 qq = qv[v4];
-                            acc[h] = fmaf(qq.x, kf[4 * v4 + 0], acc[h]);
-                            acc[h] = fmaf(qq.y, kf[4 * v4 + 1], acc[h]);
-                            acc[h] = fmaf(qq.z, kf[4 * v4 + 2], acc[h]);
-                            acc[h] = fmaf(qq.w, kf[4 * v4 + 3], acc[h]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int h = 0; h < 16; ++h)
-                if (h0 + h < H_I) score = fmaf(w_s[h0 + h], fmaxf(acc[h], 0.f), score);
-        }
-    }
-    sc[bq * kc + j] = score;
-}
 
 // idx[bq][i] = cand[bq][local[bq][i]] (local < 0, or a candidate slot holding -1, stays -1)
 __global__ void remap_kernel(const int *__restrict__ cand, const int *__restrict__ local, int kc, int k,
@@ -122,7 +67,7 @@ size_t rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I) {
            align256(nbq * kc * (size_t)d_I * 2) + align256(nbq * sizeof(int));
 }
 
-bool rescore_supported(int H_I, int d_I) { return (size_t)H_I * d_I * 4 + (size_t)H_I * 4 <= 200 * 1024; }
+bool rescore_supported(int H_I, int d_I) { return index_tc_supported(H_I, d_I); }
 
 int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, const int *cand, int kc,
                         int batch, int nq, long long N, int H_I, int d_I, int k, int *idx, void *ws,
@@ -136,34 +81,20 @@ int launch_rescore_topk(const uint16_t *q_idx, const float *w, const uint16_t *k
     uint16_t *gathered = reinterpret_cast<uint16_t *>(wsb);
     wsb += align256((size_t)nbq * kc * (size_t)d_I * 2);
     int *pos = reinterpret_cast<int *>(wsb);
-    if (index_tc_supported(H_I, d_I)) {
-        const long long n16 = nbq * kc * (d_I / 8);
-        gather_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(k_idx, cand, kc, nq, N, d_I, n16, gathered, pos);
-        if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
-        // every (sequence, query) is one sequence of kc entries with its query at position kc - 1 (m = 1)
-        int rc = launch_index_tc(q_idx, w, gathered, pos, (int)nbq, 1, kc, H_I, d_I, 1, sc, ctx, st);
-        if (rc != CSA_OK) return rc;
-        const long long n = nbq * kc;
-        mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cand, n, N, sc);
-        if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
-        rc = launch_topk(sc, nullptr, batch, nq, kc, 1, k, local, st);
-        if (rc != CSA_OK) return rc;
-        const long long nk = nbq * k;
-        remap_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, st>>>(cand, local, kc, k, nk, idx);
-        return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
-    }
-    const size_t smem = ((size_t)H_I * d_I + H_I) * sizeof(float);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return CSA_ERR_CUDA;
-    const dim3 grid((unsigned)((kc + kThreadsPerBlock - 1) / kThreadsPerBlock), (unsigned)nbq);
-    rescore_kernel<<<grid, kThreadsPerBlock, smem, st>>>(q_idx, w, k_idx, cand, kc, nq, N, H_I, d_I, sc);
+    if (!index_tc_supported(H_I, d_I)) return CSA_ERR_UNSUPPORTED;
+    const long long n16 = nbq * kc * (d_I / 8);
+    gather_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(k_idx, cand, kc, nq, N, d_I, n16, gathered, pos);
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
-    // every candidate slot is eligible: no causal threshold (q_pos = null)
-    const int rc = launch_topk(sc, nullptr, batch, nq, kc, 1, k, local, st);
+    // every (sequence, query) is one sequence of kc entries with its query at position kc - 1 (m = 1)
+    int rc = launch_index_tc(q_idx, w, gathered, pos, (int)nbq, 1, kc, H_I, d_I, 1, sc, ctx, st);
     if (rc != CSA_OK) return rc;
-    const long long n = nbq * k;
-    remap_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cand, local, kc, k, n, idx);
+    const long long n = nbq * kc;
+    mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cand, n, N, sc);
+    if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+    rc = launch_topk(sc, nullptr, batch, nq, kc, 1, k, local, st);
+    if (rc != CSA_OK) return rc;
+    const long long nk = nbq * k;
+    remap_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, st>>>(cand, local, kc, k, nk, idx);
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 

@@ -130,8 +130,15 @@ def test_index_validation(lib):
     assert f(*ok, 1, 1, 100, 64, 128, 0, A16b, NULL) == csa.CSA_ERR_INVALID          # m
     assert f(*ok, 1, 1, 100, 512, 128, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED     # H_I
     assert f(*ok, 1, 1, 100, 64, 128, 4, MIS, NULL) == csa.CSA_ERR_INVALID
+    # one implementation (the tensor-core kernel): other head dims are refused on the host
+    assert f(*ok, 1, 1, 100, 8, 48, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED        # d_I = 48
+    assert f(*ok, 1, 1, 100, 8, 272, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED       # d_I > 256
     g = lib.csa_index_fp4
     assert g(A16, NULL, A16, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID
+    assert g(A16, A16, A16, A16, A16, A16, 1, 1, 100, 4, 32, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED  # d_I = 32
+    odd = ctypes.c_void_p(0x10001)
+    assert g(A16, A16, A16, A16, odd, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID  # k4s
+    assert g(A16, odd, A16, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID  # q4s
 
 
 def test_quantize_validation(lib):
@@ -159,7 +166,8 @@ def test_rescore_validation_and_workspace(lib):
     assert f(*args[:3], NULL, *args[4:], ws, need, NULL) == csa.CSA_ERR_INVALID        # cand
     assert f(*args[:10], 0, A16b, ws, need, NULL) == csa.CSA_ERR_INVALID               # k
     assert f(*args[:10], 9000, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED
-    assert f(*args[:8], 256, 256, 1024, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED  # query too big
+    assert f(*args[:8], 256, 256, 1024, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED  # query + 2 stages > smem
+    assert f(*args[:8], 8, 48, 1024, A16b, ws, need, NULL) == csa.CSA_ERR_UNSUPPORTED    # d_I = 48
     assert f(*args, ws, need - 1, NULL) == csa.CSA_ERR_WORKSPACE
     assert f(*args, ctypes.c_void_p(0x40010), need, NULL) == csa.CSA_ERR_WORKSPACE     # misaligned workspace
     assert f(*args, NULL, need, NULL) == csa.CSA_ERR_WORKSPACE
@@ -194,6 +202,25 @@ def test_attend_validation_and_workspace(lib):
     h = lib.hca_attend
     assert h(A16, NULL, NULL, NULL, NULL, 0, A16, 300, 0, A16, 0, 2048, 16, A16, 1, 1, 8, 64, 0.125, 1e-6, A16b,
              NULL, 0, NULL) == csa.CSA_ERR_INVALID    # m
+
+
+def test_attend_noalloc_checks_arguments_before_its_size_limit(lib):
+    """The allocation-free entry point reports a bad argument as csa_attend
+    does (its own size limit is checked only after the arguments).  Only
+    invalid calls here: a valid one would launch."""
+    f = lib.csa_attend_noalloc
+
+    def call(q=A16, idx=A16, W=16, D=512, H=128, k=1024, out=A16b):
+        return f(q, NULL, NULL, NULL, NULL, 0, A16, 1 << 16, idx, k, A16, 0, 1 << 18, W, A16, 8, 1,
+                 H, D, 0.05, 1e-6, out, NULL)
+
+    assert call(q=NULL) == csa.CSA_ERR_INVALID
+    assert call(out=MIS) == csa.CSA_ERR_INVALID
+    assert call(idx=ctypes.c_void_p(0x10002)) == csa.CSA_ERR_INVALID   # idx not 4-byte aligned
+    assert call(k=-1) == csa.CSA_ERR_INVALID
+    assert call(W=0) == csa.CSA_ERR_INVALID
+    assert call(D=96) == csa.CSA_ERR_UNSUPPORTED
+    assert call(H=256) == csa.CSA_ERR_UNSUPPORTED
     # workspace sizing is monotone in the key count and batch
     assert lib.csa_attend_workspace_bytes(8, 1, 128, 512, 1152) >= lib.csa_attend_workspace_bytes(1, 1, 128, 512, 1152)
 

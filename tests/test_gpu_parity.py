@@ -196,7 +196,6 @@ def _check_scores(got, ref, rel):
     (2, 1, 8, 256, 300, 2, [599, 100]),
     (1, 9, 64, 128, 2000, 4, [7999 - 3 * i for i in range(9)]),     # query groups of 4 (+1 ragged)
     (3, 5, 4, 32, 700, 4, [2799, 2000, 1000, 10, 3] * 3),          # H_I padded to 16, 5 queries per tile
-    (1, 2, 8, 48, 200, 4, [799, 400]),                             # d_I = 48: CUDA-core kernel
     (8, 1, 64, 128, 32768, 4, [131071] * 8),                       # CSA decode shape
 ])
 def test_index_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
@@ -609,7 +608,6 @@ def test_quantize_fp4_bit_exact(cuda):
     (2, 2, 16, 64, 777, 4, [3107, 50, 3000, 7]),
     (1, 40, 64, 128, 2048, 4, [8191 - 197 * i for i in range(40)]),   # several query groups per sequence
     (2, 1, 32, 256, 1500, 4, [5999, 2001]),                              # d_I = 256, ragged last tile
-    (1, 1, 4, 32, 300, 4, [1199]),                                       # d_I = 32: CUDA-core path
 ])
 def test_index_fp4_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
     qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts, seed=80)

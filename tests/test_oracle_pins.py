@@ -117,6 +117,34 @@ def test_compress_rmsnorm_closed_form():
     np.testing.assert_allclose(ng, nrm * g.astype(np.float64), rtol=1e-13)
 
 
+def test_rmsnorm_rows_closed_form():
+    """The row RMSNorm helper: output RMS = sqrt(ms / (ms + eps)) (closed form),
+    the direction of every row kept, gain applied per channel, and rows scaled
+    by a power of two (exact in bf16) give outputs that follow the closed form
+    for their own mean square.  A dropped 1/d, a missing eps, the gain applied
+    per row instead of per channel, or a sum of |x| instead of x^2 fails it."""
+    r = rng(41)
+    rows, d, eps = 37, 48, 1e-2
+    x = r.standard_normal((rows, d))
+    x[3] *= 2.0 ** -6                      # small rows, where eps matters
+    x[5] = 0.0                             # zero row -> zero output, no NaN
+    xb = bf16_bits(x)
+    xv = bf16_val(xb)
+    out = oracle.rmsnorm(xb, eps=eps)
+    ms = (xv ** 2).mean(-1)
+    np.testing.assert_allclose(np.sqrt((out ** 2).mean(-1)), np.sqrt(ms / (ms + eps)), rtol=1e-12)
+    np.testing.assert_allclose(out * np.sqrt(ms + eps)[:, None], xv, rtol=1e-12, atol=1e-300)
+    assert np.all(out[5] == 0.0)
+    g = r.uniform(0.5, 2.0, d).astype(np.float32)
+    np.testing.assert_allclose(oracle.rmsnorm(xb, eps=eps, gain=g), out * g.astype(np.float64), rtol=1e-13)
+    # with eps -> 0 the output no longer depends on the row's scale
+    big = bf16_bits(xv * 8.0)
+    np.testing.assert_allclose(oracle.rmsnorm(big, eps=1e-30), oracle.rmsnorm(xb, eps=1e-30), rtol=1e-12)
+    # hand-worked row: x = (3, 4), ms = 12.5, eps = 0 -> x / sqrt(12.5)
+    np.testing.assert_allclose(oracle.rmsnorm(bf16_bits([[3.0, 4.0]]), eps=0.0),
+                               [[3.0 / math.sqrt(12.5), 4.0 / math.sqrt(12.5)]], rtol=1e-15)
+
+
 def test_compress_entry_range_matches_full():
     r = rng(5)
     m, T, d = 4, 80, 16
