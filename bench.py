@@ -318,17 +318,10 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
     barrier(world)
     t_max = max_over_ranks(t_graph, world, device)
     value = job_rate(wl.batch * wl.nq, args.steps, world, t_max)
-    # per-kernel breakdown: eager steps over the same rotation, events between the kernels
-    seg = [0.0, 0.0, 0.0]
-    for i in range(args.warmup + args.steps):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        evs[0].record()
-        csa_decode_step(csa, states[i % len(states)], lambda k: evs[1 + k].record())
-        evs[3].record()
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            for k in range(3):
-                seg[k] += evs[k].elapsed_time(evs[k + 1]) / 1e3 / args.steps
+    # per-kernel breakdown: each kernel of the step captured alone in a graph per
+    # decode state; K back-to-back replays over the same rotation between two
+    # events on the launch stream (no host launch gaps inside the interval)
+    seg = kernel_breakdown(csa, states, args)
     t_index = seg[0]
     idx_bytes = index_bytes(wl)
     src_hash = kernel_source_hash("index_tc.cu", "tc.cuh")
@@ -348,6 +341,45 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
                       "hbm_frac_of_measured": round(step_bytes / step_s / 1e9 / peaks["hbm_gbs"], 4),
                       "kernel_ms": {"csa_index": round(seg[0] * 1e3, 4), "csa_topk": round(seg[1] * 1e3, 4),
                                     "csa_attend+combine": round(seg[2] * 1e3, 4)}}), st
+
+
+def kernel_breakdown(csa, states, args):
+    """Seconds per launch of csa_index, csa_topk and csa_attend (+ its split
+    combine) in the decode step: each captured alone per decode state and
+    replayed back to back over the rotation, timed by events around the run."""
+    parts = []
+    for S in states:
+        wl = S["wl"]
+        gs = []
+        for k in range(3):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                if k == 0:
+                    csa.csa_index(S["qI"], S["w"], S["kI"], S["qp"], wl.m, scores=S["S"])
+                elif k == 1:
+                    csa.csa_topk(S["S"], S["qp"], wl.m, wl.k, idx=S["idx"])
+                else:
+                    csa.csa_attend(S["q"], S["C"], S["idx"], S.get("win", S.get("A")), S["qp"], wl.W, wl.scale,
+                                   wl.eps, out=S["out"], workspace=S["ws"], win_pos0=S.get("win_pos0", 0))
+            gs.append(g)
+        parts.append(gs)
+    torch.cuda.synchronize()
+    seg = []
+    n = max(args.steps, 6)
+    for k in range(3):
+        for i in range(args.warmup):
+            parts[i % len(parts)][k].replay()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            parts[i % len(parts)][k].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        seg.append(e0.elapsed_time(e1) / 1e3 / n)
+    del parts
+    return seg
 
 
 E2E_STATES = 4
@@ -559,7 +591,13 @@ def bench_fp4(csa, args, device, peaks):
     wl = W.FP4_DECODE
     kI = W.index_keys(wl, device)
     k4, k4s = csa.csa_quantize_fp4(kI)
-    C = W.direct_kv(wl, device)
+    # compressed KV rows drawn N(0,1), then RMSNorm'd like every compressed entry:
+    # csa_compress with m = 1 and logits (-inf for the B row, 0 for the A row)
+    # pools each row with weight 1 alone and applies the RMSNorm
+    raw = W.direct_kv(wl, device)
+    one = torch.cat([torch.full((1, wl.D), float("-inf"), device=device), torch.zeros((1, wl.D), device=device)])
+    C = csa.csa_compress(raw, raw, one, 1)
+    del raw
     win = W.normal_bf16((wl.batch, wl.W, wl.D), 424242, device)
     qI, w = W.index_queries(wl, device), W.index_weights(wl, device)
     q = W.queries(wl, device)

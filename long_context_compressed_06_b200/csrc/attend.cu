@@ -15,62 +15,82 @@
 namespace csa {
 namespace {
 
-__global__ void __launch_bounds__(128) attend_combine_kernel(AttendArgs a) {
+// One thread per 8 output columns of one head: the splits' (max, sum) first,
+// then their bf16 rows in split order, 8 splits' loads in flight at a time.
+//   out = sum_s 2^(m_s - M) l_s O_s / (sum_s 2^(m_s - M) l_s + sink)
+// with O_s the split's row already divided by its own sum l_s.
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendArgs a) {
+    const int tph = a.D / 8;                              // threads per head
     const long long bq = blockIdx.x;
-    const int h = blockIdx.y;
-    const int i = threadIdx.x * 4;
-    const bool active = i < a.D;  // no early exit: the RoPE shuffles need whole warps
+    const int h = blockIdx.y * (kCombineThreads / tph) + threadIdx.x / tph;
+    const int c0 = (threadIdx.x % tph) * 8;
+    const bool active = h < a.H;  // no early exit: the RoPE shuffles need whole warps
+    const size_t stride = (size_t)a.n_bq * a.H;          // between splits, in rows
+    const size_t row = (size_t)bq * a.H + (active ? h : 0);
     float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((size_t)s * a.n_bq + bq) * a.H + h].x);
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < a.splits && active; ++s) {
-        const size_t off = ((size_t)s * a.n_bq + bq) * a.H + h;
-        const float2 ml = a.part_ml[off];
-        const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-        L = fmaf(w, ml.y, L);
-        const float4 o = *reinterpret_cast<const float4 *>(a.part_o + off * a.D + i);
-        acc.x = fmaf(w, o.x, acc.x);
-        acc.y = fmaf(w, o.y, acc.y);
-        acc.z = fmaf(w, o.z, acc.z);
-        acc.w = fmaf(w, o.w, acc.w);
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[s * stride + row].x);
+    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < a.splits; s0 += 8) {
+        const int ns = a.splits - s0 < 8 ? a.splits - s0 : 8;
+        float2 ml[8];
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < ns) {
+                ml[j] = a.part_ml[(s0 + j) * stride + row];
+                v[j] = *reinterpret_cast<const uint4 *>(a.part_o + ((s0 + j) * stride + row) * a.D + c0);
+            }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < ns) {
+                const float wl = ml[j].x == -INFINITY ? 0.f : exp2f(ml[j].x - M) * ml[j].y;
+                L += wl;
+                float f[8];
+                unpack8(v[j], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wl, f[e], acc[e]);
+            }
     }
     // the head's sink logit (natural units; the partials are in log2 units)
-    if (a.sinks) L += exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - M);
+    if (a.sinks && active) L += exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - M);
     const float inv = L > 0.f ? 1.0f / L : 0.f;
-    float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = acc[e] * inv;
     if (a.rope_cos) {
         // conjugate rotation of the trailing kRopeDim channels: channel D-64+j pairs
-        // with D-32+j, 8 threads (32 channels) away in the same warp
-        float pv[4];
+        // with D-32+j, held by the thread 4 lanes away (32 channels)
+        float pv[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 8);
-        if (active && i >= a.D - kRopeDim) {
+        for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
+        if (c0 >= a.D - kRopeDim) {
             const long long t = __ldg(a.q_pos + bq);
-            const bool first = i < a.D - kRopeDim / 2;
-            const int i0 = (i - (a.D - kRopeDim)) & (kRopeDim / 2 - 1);
+            const bool first = c0 < a.D - kRopeDim / 2;
+            const int i0 = (c0 - (a.D - kRopeDim)) & (kRopeDim / 2 - 1);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 8; ++e) {
                 const float2 cs = rope_cs(a, t, i0 + e);
                 o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
             }
         }
     }
-    if (!active) return;
-    uint16_t *dst = a.out + ((size_t)bq * a.H + h) * a.D + i;
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+    if (active) *reinterpret_cast<uint4 *>(a.out + row * a.D + c0) = pack8(o);
 }
 
+// [splits][n_bq][H][D] bf16 rows, then [splits][n_bq][H] float2 (max, sum)
 size_t ws_bytes_for(long long n_bq, int H, int D, int splits) {
     if (splits <= 1) return 0;
-    return (size_t)splits * n_bq * H * ((size_t)D * sizeof(float) + sizeof(float2));
+    return (size_t)splits * n_bq * H * ((size_t)D * sizeof(uint16_t) + sizeof(float2));
 }
 
 }  // namespace
 
 int launch_attend_combine(const AttendArgs &a, cudaStream_t st) {
-    dim3 grid((unsigned)a.n_bq, (unsigned)a.H);
-    attend_combine_kernel<<<grid, std::max(32, a.D / 4), 0, st>>>(a);
+    const int hpb = kCombineThreads / (a.D / 8);  // heads per block (D in {64, ..., 512})
+    dim3 grid((unsigned)a.n_bq, (unsigned)((a.H + hpb - 1) / hpb));
+    attend_combine_kernel<<<grid, kCombineThreads, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
@@ -119,9 +139,9 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
     const size_t need = ws_bytes_for(a.n_bq, H, D, a.splits);
     if (need > 0) {
         if (!ws || ws_bytes < need) return CSA_ERR_WORKSPACE;
-        a.part_o = reinterpret_cast<float *>(ws);
+        a.part_o = reinterpret_cast<uint16_t *>(ws);
         a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
-                                               (size_t)a.splits * a.n_bq * H * D * sizeof(float));
+                                               (size_t)a.splits * a.n_bq * H * D * sizeof(uint16_t));
     }
     return launch_attend_tc(a, ctx, st);
 }

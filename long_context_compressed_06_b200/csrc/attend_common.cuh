@@ -1,5 +1,5 @@
-// attend_common.cuh -- argument block, key-set enumeration and split-KV
-// workspace layout shared by the attention kernels.
+// attend_common.cuh -- argument block and split-KV workspace layout shared by
+// the attention kernel and the split combine.
 #pragma once
 
 #include "common.cuh"
@@ -38,7 +38,7 @@ struct AttendArgs {
     int H, D;
     float scale, eps;
     uint16_t *out;          // [n_bq][H][D]
-    float *part_o;          // [splits][n_bq][H][D] unnormalised partial outputs
+    uint16_t *part_o;       // [splits][n_bq][H][D] bf16 partial outputs, each divided by its own sum
     float2 *part_ml;        // [splits][n_bq][H] (running max in log2 units, sum)
     int splits;
     long long keys_per_split;
@@ -50,50 +50,6 @@ CSA_DEVINL float2 rope_cs(const AttendArgs &a, long long t, int i) {
     if (!a.rope_cos || t < 0 || t >= a.rope_npos) return make_float2(1.f, 0.f);
     const size_t o = (size_t)t * (kRopeDim / 2) + i;
     return make_float2(__ldg(a.rope_cos + o), __ldg(a.rope_sin + o));
-}
-
-// The key set J of one query is enumerated as e = 0 .. total-1: first the
-// nsel selected (CSA: idx slots, HCA: entries 0..n_vis-1), then the window
-// positions u0 .. u0 + nwin - 1 of stream A held by the window buffer.
-struct KeySet {
-    long long nsel, u0, total;
-};
-
-CSA_DEVINL KeySet key_set(const AttendArgs &a, long long /*b*/, long long /*bq*/, long long t) {
-    KeySet ks;
-    ks.nsel = a.dense ? n_visible(t, a.m, a.N) : a.k;
-    long long u0 = t - a.W + 1;
-    u0 = u0 < 0 ? 0 : u0;
-    ks.u0 = u0 < a.win_pos0 ? a.win_pos0 : u0;
-    const long long last = a.win_pos0 + a.win_rows - 1;
-    const long long u1 = t < last ? t : last;
-    const long long nwin = u1 >= ks.u0 ? u1 - ks.u0 + 1 : 0;
-    ks.total = ks.nsel + nwin;
-    return ks;
-}
-
-// Row of key e, or null for an invalid selection slot (-1 or out of range).
-CSA_DEVINL const uint16_t *key_row(const AttendArgs &a, const KeySet &ks, long long b, long long bq,
-                                   long long e) {
-    if (e < ks.nsel) {
-        const long long j = a.dense ? e : (long long)__ldg(a.idx + bq * a.k + e);
-        if (j < 0 || j >= a.N) return nullptr;
-        return a.kv + ((size_t)b * a.N + j) * a.D;
-    }
-    return a.win + ((size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + (e - ks.nsel)) * a.D;
-}
-
-template <int DPL>
-CSA_DEVINL void store_lane_dims(uint16_t *row, int lane, const float f[DPL]) {
-    uint16_t *p = row + lane * DPL;
-    if constexpr (DPL >= 8) {
-#pragma unroll
-        for (int i = 0; i < DPL; i += 8) *reinterpret_cast<uint4 *>(p + i) = pack8(f + i);
-    } else if constexpr (DPL == 4) {
-        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
-    } else {
-        *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(f[0], f[1]);
-    }
 }
 
 int launch_attend_combine(const AttendArgs &a, cudaStream_t st);

@@ -30,8 +30,8 @@
 // the output through shared memory for coalesced stores.  The roles only
 // meet at mbarriers, so the gathers of the next work item overlap the output
 // of the current one.  Work items are (query, key split, head half); splits
-// write fp32 partials + (max, sum) that attend_combine merges in a fixed
-// order.  Every wait is bounded and every role warp stays converged.
+// write bf16 partial rows (each divided by its own sum) + (max, sum) that
+// attend_combine merges in a fixed order.  Every wait is bounded and every role warp stays converged.
 #include <algorithm>
 
 #include "attend_common.cuh"
@@ -676,9 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_after_sync();
             }
             // one split: normalise here, the head's sink logit (natural units ->
-            // log2 units) joining the denominator; several: the merge does it
-            const float L = l + ((a.sinks && h < a.H) ? exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - m_run) : 0.f);
-            const float inv = a.splits == 1 ? (L > 0.f ? 1.0f / L : 0.f) : 1.0f;
+            // log2 units) joining the denominator; several: each split's rows are
+            // divided by its own sum and the merge weighs them (and adds the sink)
+            const float L = a.splits == 1
+                                ? l + ((a.sinks && h < a.H) ? exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - m_run) : 0.f)
+                                : l;
+            const float inv = L > 0.f ? 1.0f / L : 0.f;
             uint8_t *stg = s.p;
             for (int c = 0; c < D; c += 64) {
                 float v[32];
@@ -694,41 +697,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<float4 *>(stg + hl * 256 + (((8 * kh + u) ^ (hl & 7)) << 4)) =
                         make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
                 __syncwarp();  // a warp stages and stores only its own 16 heads
-                if (a.splits == 1) {
-                    // bf16 rows: 4 heads per instruction, 8 lanes x 8 columns each
+                // bf16 rows (the output, or this split's partial): 4 heads per
+                // instruction, 8 lanes x 8 columns each
+                uint16_t *const dst0 = a.splits == 1 ? a.out + (size_t)it.bq * a.H * D
+                                                     : a.part_o + ((size_t)it.split * a.n_bq + it.bq) * a.H * D;
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4) {
-                        const int r = sp * 16 + i + (lane >> 3), cu = lane & 7, hr = it.head0 + r;
-                        const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
-                        const float4 hi =
-                            *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
-                        float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                        if (a.rope_cos && c == D - kRopeDim) {
-                            // conjugate rotation of the rotated slice (this 64-column slab):
-                            // column 8*cu + e pairs with 8*(cu ^ 4) + e, held by lane ^ 4
-                            float pv[8];
+                for (int i = 0; i < 16; i += 4) {
+                    const int r = sp * 16 + i + (lane >> 3), cu = lane & 7, hr = it.head0 + r;
+                    const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
+                    const float4 hi = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
+                    float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                    if (a.splits == 1 && a.rope_cos && c == D - kRopeDim) {
+                        // conjugate rotation of the rotated slice (this 64-column slab):
+                        // column 8*cu + e pairs with 8*(cu ^ 4) + e, held by lane ^ 4
+                        // (with several splits the merge rotates the merged row)
+                        float pv[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
-                            const bool first = cu < 4;
+                        for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
+                        const bool first = cu < 4;
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const float2 cs = rope_cs(a, tq, (cu & 3) * 8 + e);
-                                o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
-                            }
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 cs = rope_cs(a, tq, (cu & 3) * 8 + e);
+                            o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
                         }
-                        if (hr < a.H)
-                            *reinterpret_cast<uint4 *>(a.out + ((size_t)it.bq * a.H + hr) * D + c + 8 * cu) = pack8(o);
                     }
-                } else {
-                    // fp32 partial rows: 2 heads per instruction, 16 lanes x 4 columns each
-#pragma unroll
-                    for (int i = 0; i < 16; i += 2) {
-                        const int r = sp * 16 + i + (lane >> 4), cu = lane & 15, hr = it.head0 + r;
-                        const float4 v4 = *reinterpret_cast<const float4 *>(stg + r * 256 + ((cu ^ (r & 7)) << 4));
-                        if (hr < a.H)
-                            *reinterpret_cast<float4 *>(
-                                a.part_o + (((size_t)it.split * a.n_bq + it.bq) * a.H + hr) * D + c + 4 * cu) = v4;
-                    }
+                    if (hr < a.H) *reinterpret_cast<uint4 *>(dst0 + (size_t)hr * D + c + 8 * cu) = pack8(o);
                 }
                 __syncwarp();  // a warp stages and stores only its own 16 heads
             }

@@ -13,9 +13,8 @@
 //
 // The weights differ per entry and channel, so unlike csa_compress nothing is
 // precomputed: a thread owns 8 channels of one entry and runs an online softmax
-// over the 2m rows in fp32, in log2 units, batch by batch: the maximum over the
-// batch's rows first, one rescale of the running denominator and accumulator,
-// then the batch's weights -- no per-element branch.  Every stream row is read once, so the op
+// over the 2m rows in fp32 (running maximum, rescaled denominator and
+// accumulator, in log2 units).  Every stream row is read once, so the op
 // streams 4*T*d*2 bytes (A, B, Z_a, Z_b) plus the T/m*d*2 written: it is HBM
 // bound.  The loads of kRows rows are issued before the first is used.  The
 // RMSNorm sum of squares is reduced in a fixed order (warp shuffles, then the
@@ -30,20 +29,9 @@
 namespace csa {
 namespace {
 
-constexpr int kRows = 4;                         // rows whose loads are in flight together
+constexpr int kRows = 8;                         // rows whose loads are in flight together
 constexpr int kMaxThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
-
-// logits of one row's 8 channels in log2 units: (Z + bias) * log2(e)
-CSA_DEVINL void logits8(const uint4 &z, const float *__restrict__ b, float l[8]) {
-    float zf[8];
-    unpack8(z, zf);
-    const float4 b0 = __ldg(reinterpret_cast<const float4 *>(b));
-    const float4 b1 = __ldg(reinterpret_cast<const float4 *>(b + 4));
-    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-    for (int q = 0; q < 8; ++q) l[q] = (zf[q] + bb[q]) * kLog2e;
-}
 
 __global__ void __launch_bounds__(kMaxThreads) compress_dynamic_kernel(
     const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, const uint16_t *__restrict__ Za,
@@ -85,38 +73,26 @@ __global__ void __launch_bounds__(kMaxThreads) compress_dynamic_kernel(
                     if (z) zv[k] = ldg_stream(z + off);
                 }
             }
-            // pass 1: the batch's maximum logit per channel (rows past 2m stay out)
-            float bm[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) bm[q] = mx[q];
 #pragma unroll
             for (int k = 0; k < kRows; ++k) {
                 const int r = r0 + k;
                 if (r < 2 * m) {
-                    float l[8];
-                    logits8(zv[k], bias + (size_t)r * d + c0, l);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) bm[q] = fmaxf(bm[q], l[q]);
-                }
-            }
-            // one rescale of the running sums per batch, then every weight against the new maximum
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float s = bm[q] == -INFINITY ? 1.f : exp2f(mx[q] - bm[q]);  // mx = -inf -> 0
-                den[q] *= s;
-                acc[q] *= s;
-                mx[q] = bm[q];
-            }
-#pragma unroll
-            for (int k = 0; k < kRows; ++k) {
-                const int r = r0 + k;
-                if (r < 2 * m) {
-                    float l[8], xf[8];
-                    logits8(zv[k], bias + (size_t)r * d + c0, l);
+                    float zf[8], xf[8];
+                    unpack8(zv[k], zf);
                     unpack8(xv[k], xf);
+                    const float4 b0 = __ldg(reinterpret_cast<const float4 *>(bias + (size_t)r * d + c0));
+                    const float4 b1 = __ldg(reinterpret_cast<const float4 *>(bias + (size_t)r * d + c0 + 4));
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float w = mx[q] == -INFINITY ? 0.f : exp2f(l[q] - mx[q]);
+                        const float l = (zf[q] + bb[q]) * kLog2e;
+                        if (l > mx[q]) {  // new maximum: rescale what has been summed so far
+                            const float s = exp2f(mx[q] - l);
+                            den[q] *= s;
+                            acc[q] *= s;
+                            mx[q] = l;
+                        }
+                        const float w = l == -INFINITY ? 0.f : exp2f(l - mx[q]);
                         den[q] += w;
                         acc[q] = fmaf(w, xf[q], acc[q]);
                     }

@@ -6,8 +6,9 @@
 // become -1).  Output indices are in ascending order.
 //
 // Design: a radix select over the scores mapped to order-preserving uint32
-// keys.  One query is handled by a thread-block cluster of CS CTAs x 1024
-// threads; each thread keeps R consecutive keys in registers (CS*1024*R >= N),
+// keys.  One query is handled by one CTA of 1024 threads when its row fits in
+// their registers (N <= 32768), else by a thread-block cluster of CS CTAs;
+// each thread keeps R consecutive keys in registers (CS*1024*R >= N),
 // so the scores are read from memory exactly once.  The digits start at the
 // highest bit where the cluster-wide smallest and largest key differ (the bits
 // above are shared by every candidate), 11 bits per pass; each CTA counts its
@@ -65,13 +66,22 @@ CSA_DEVINL T block_scan_incl(T v, T *warp_buf, T *total) {
     return v;
 }
 
-template <int R>
+// CL: the query's row is split over a cluster of CS CTAs (histograms and CTA
+// totals merged through distributed shared memory, cluster barriers); without
+// it one CTA holds the row and every barrier is a block barrier.
+template <int R, bool CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__restrict__ scores,
                                                                const int *__restrict__ q_pos, long long N,
                                                                int m, int k, int *__restrict__ idx, int CS) {
     cg::cluster_group cluster = cg::this_cluster();
-    const int rank = (int)cluster.block_rank();
+    const int rank = CL ? (int)cluster.block_rank() : 0;
     const long long bq = blockIdx.x / CS;
+    const auto sync_all = [&]() {
+        if constexpr (CL) cluster.sync(); else __syncthreads();
+    };
+    const auto peer = [&](auto *p, int r) {
+        if constexpr (CL) return cluster.map_shared_rank(p, r); else return p;
+    };
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     __shared__ __align__(8) uint32_t hist[2][kBins];  // this CTA's histogram, double-buffered over passes
@@ -125,10 +135,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
             cta_max = b;
         }
     }
-    cluster.sync();  // key ranges published, histograms cleared
+    sync_all();  // key ranges published, histograms cleared
     if (warp == 0) {
-        const uint32_t a = lane < CS ? *cluster.map_shared_rank(&cta_min, lane) : 0xffffffffu;
-        const uint32_t b = lane < CS ? *cluster.map_shared_rank(&cta_max, lane) : 0u;
+        const uint32_t a = lane < CS ? *peer(&cta_min, lane) : 0xffffffffu;
+        const uint32_t b = lane < CS ? *peer(&cta_max, lane) : 0u;
         const uint32_t ga = __reduce_min_sync(0xffffffffu, a), gb = __reduce_max_sync(0xffffffffu, b);
         if (lane == 0) {
             s_min = ga;
@@ -166,11 +176,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
 #pragma unroll
         for (int r = 0; r < R; ++r)
             if (r < nloc && (key[r] & mask) == prefix) atomicAdd(hloc + ((key[r] >> sh) & dmask), 1u);
-        cluster.sync();  // every CTA's histogram of this pass is complete
+        sync_all();  // every CTA's histogram of this pass is complete
         // cluster-wide counts of this thread's two bins: read every rank's histogram
         uint32_t c_lo = 0u, c_hi = 0u;
         for (int r2 = 0; r2 < CS; ++r2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(cluster.map_shared_rank(hloc, r2) + 2 * threadIdx.x);
+            const uint2 v = *reinterpret_cast<const uint2 *>(peer(hloc, r2) + 2 * threadIdx.x);
             c_lo += v.x;
             c_hi += v.y;
         }
@@ -207,10 +217,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     unsigned long long blk_tot;
     const unsigned long long mine = ((unsigned long long)gt << 32) | eq;
     const unsigned long long excl = block_scan_incl<unsigned long long>(mine, warp_u64, &blk_tot) - mine;
-    if (threadIdx.x == 0) cta_total = blk_tot;
-    cluster.sync();
     unsigned long long base = 0ull;
-    for (int r2 = 0; r2 < rank; ++r2) base += *cluster.map_shared_rank(&cta_total, r2);
+    if constexpr (CL) {
+        if (threadIdx.x == 0) cta_total = blk_tot;
+        cluster.sync();
+        for (int r2 = 0; r2 < rank; ++r2) base += *cluster.map_shared_rank(&cta_total, r2);
+    }
     long long gt_before = (long long)((base + excl) >> 32);
     long long eq_before = (long long)((base + excl) & 0xffffffffull);
     int *out = idx + bq * k;
@@ -230,7 +242,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     }
     if (rank == 0)
         for (long long i = kk + threadIdx.x; i < k; i += kTopkThreads) out[i] = -1;
-    cluster.sync();  // peers may still read this CTA's histogram / cta_total
+    if constexpr (CL) cluster.sync();  // peers may still read this CTA's histogram / cta_total
 }
 
 struct TopkPlan {
@@ -243,12 +255,11 @@ TopkPlan plan(long long n_queries, long long N) {
     while ((need + CS - 1) / CS > 32) CS *= 2;
     int R = 4;
     while ((long long)R * CS < need) R *= 2;
-    // spread small batches over more SMs; measured at 8 queries x 32768 entries,
-    // clusters of 4 beat 2 and 8 (the histogram merge reads every peer)
-    while (n_queries * CS < 148 && CS < 4 && R > 4) {
-        CS *= 2;
-        R /= 2;
-    }
+    // One CTA per query whenever its 1024 threads can hold the row (up to 32
+    // keys each): the cluster's barriers and peer-histogram reads cost more
+    // than they save (measured on the 8-query decode batch at 32768 entries:
+    // a cluster of 4 took 14.7 us).
+    (void)n_queries;
     return {CS, R};
 }
 
@@ -263,11 +274,12 @@ int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long l
     const TopkPlan pl = plan(nqry, N);
     if (pl.CS > 16 || pl.R > 32) return CSA_ERR_UNSUPPORTED;
     void (*kern)(const float *, const int *, long long, int, int, int *, int) = nullptr;
+    const bool cl = pl.CS > 1;
     switch (pl.R) {
-        case 4: kern = topk_kernel<4>; break;
-        case 8: kern = topk_kernel<8>; break;
-        case 16: kern = topk_kernel<16>; break;
-        case 32: kern = topk_kernel<32>; break;
+        case 4: kern = cl ? topk_kernel<4, true> : topk_kernel<4, false>; break;
+        case 8: kern = cl ? topk_kernel<8, true> : topk_kernel<8, false>; break;
+        case 16: kern = cl ? topk_kernel<16, true> : topk_kernel<16, false>; break;
+        case 32: kern = cl ? topk_kernel<32, true> : topk_kernel<32, false>; break;
         default: return CSA_ERR_UNSUPPORTED;
     }
     if (pl.CS > 8 &&
@@ -284,7 +296,7 @@ int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long l
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = cl ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, scores, q_pos, N, m, k, idx, pl.CS);
     return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
