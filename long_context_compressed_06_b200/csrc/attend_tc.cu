@@ -33,6 +33,7 @@
 // write bf16 partial rows (each divided by its own sum) + (max, sum) that
 // attend_combine merges in a fixed order.  Every wait is bounded and every role warp stays converged.
 #include <algorithm>
+#include <cstring>
 
 #include "attend_common.cuh"
 #include "common.cuh"
@@ -52,6 +53,7 @@ constexpr int kMaxStages = 4;
 
 struct AttTcParams {
     AttendArgs a;
+    int kv_tma;         // dense key set over bf16 rows: whole tiles of entries arrive by TMA
     int HH;             // head halves per query (1 or 2)
     int stages;
     uint32_t idesc_qk, idesc_pv;
@@ -334,7 +336,8 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const AttTcParams p) {
+    attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                     const AttTcParams p) {
     using Lt = Layout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem s = carve<D>(smem_raw, p.stages);
@@ -361,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *s.abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&qmap);
+        if (p.kv_tma) tc::prefetch_tmap(&kvmap);
     }
     // per-dimension query gains of this lane's units (softmax warps), read once
     float qg[QLanes<D>::UPL][8];
@@ -421,6 +425,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint32_t stage = smem_u32(s.k + (size_t)st * Lt::kStageBytes);
+                // HCA: a tile of 64 consecutive visible entries is one contiguous run of
+                // kv rows, loaded by TMA tiles (one per 64-dim chunk) instead of row gathers
+                const bool tma_tile = !FP8 && p.kv_tma && ebase + kTileKeys <= it.ks.nsel;
+                if (tma_tile) {
+                    if (pw == 0) {  // the mask arrive carries the TMA byte count
+                        if (lane == 0) s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
+                        mbar_arrive_expect_tx(smem_u32(s.kfull + st), Lt::kStageBytes, lane == 0);
+                        for (int c = 0; c < Lt::kChunks; ++c)
+                            tc::tma_load_3d(stage + c * (kTileKeys * 128), &kvmap, smem_u32(s.kfull + st), c * 64,
+                                            (int)ebase, (int)it.b, lane == 0);
+                    }
+                    // the producers' cp.async arrivals (none pending for this tile)
+                    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
+                                 : "memory");
+                    continue;
+                }
                 if constexpr (FP8) {
                     // FP8 rows: lane l converts the 8 codes of each of its 16-byte output units
                     // (8 bytes in, 8 bf16 out) and stores them where cp.async would have put the
@@ -771,8 +791,20 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
                                CU_TENSOR_MAP_SWIZZLE_128B))
             return CSA_ERR_CUDA;
     }
+    CUtensorMap kvmap;
+    memset(&kvmap, 0, sizeof(kvmap));
+    p.kv_tma = a.dense && !FP8 ? 1 : 0;
+    if (p.kv_tma) {
+        // kv [batch][N][D] bf16: boxes of 64 dims x 64 entries, 128-byte swizzle
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.N, (uint64_t)(a.n_bq / a.nq)};
+        const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.N * D * 2};
+        const uint32_t box[3] = {64, (uint32_t)kTileKeys, 1};
+        if (!encode_tensor_map(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.kv, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B))
+            return CSA_ERR_CUDA;
+    }
     const int grid = (int)std::min<long long>(p.n_work, num_sms());
-    kern<<<grid, kThreads, smem, st>>>(qmap, p);
+    kern<<<grid, kThreads, smem, st>>>(qmap, kvmap, p);
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
     return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
 }
