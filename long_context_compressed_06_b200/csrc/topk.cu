@@ -6,9 +6,9 @@
 // become -1).  Output indices are in ascending order.
 //
 // Design: a radix select over the scores mapped to order-preserving uint32
-// keys.  One query is handled by one CTA of 1024 threads when its row fits in
-// their registers (N <= 32768), else by a thread-block cluster of CS CTAs;
-// each thread keeps R consecutive keys in registers (CS*1024*R >= N),
+// keys.  One query is handled by one CTA of 1024 threads or, for long rows and
+// for small batches, by a thread-block cluster of CS CTAs; each thread keeps R
+// consecutive keys in registers (CS*1024*R >= N),
 // so the scores are read from memory exactly once.  The digits start at the
 // highest bit where the cluster-wide smallest and largest key differ (the bits
 // above are shared by every candidate), 11 bits per pass; each CTA counts its
@@ -255,11 +255,14 @@ TopkPlan plan(long long n_queries, long long N) {
     while ((need + CS - 1) / CS > 32) CS *= 2;
     int R = 4;
     while ((long long)R * CS < need) R *= 2;
-    // One CTA per query whenever its 1024 threads can hold the row (up to 32
-    // keys each): the cluster's barriers and peer-histogram reads cost more
-    // than they save (measured on the 8-query decode batch at 32768 entries:
-    // a cluster of 4 took 14.7 us).
-    (void)n_queries;
+    // Spread small batches over more SMs: measured on the 8-query decode batch
+    // at 32768 entries, clusters of 4 (8 keys per thread) take 13.7 us per
+    // launch against 19.9 us for one CTA per query (32 keys per thread), and
+    // beat clusters of 2 and 8.
+    while (n_queries * CS < 148 && CS < 4 && R > 4) {
+        CS *= 2;
+        R /= 2;
+    }
     return {CS, R};
 }
 
