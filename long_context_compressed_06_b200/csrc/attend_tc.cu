@@ -5,7 +5,8 @@
 // visible entries (HCA) plus the sliding window of raw stream-A rows
 // (techniques map rows "Grouped-query attention", "Sliding-window attention",
 // "QK normalization").  Flash-style, per tile of 64 keys:
-//   S = Q_hat K^T   (tcgen05.mma M = 64 heads, N = 64 keys, fp32 in TMEM)
+//   S = Q K^T       (tcgen05.mma M = 64 heads, N = 64 keys, fp32 in TMEM),
+//                   scaled per head by its 1/RMS (the RMSNorm of the query)
 //   online softmax in fp32, log2 domain; the running max is raised only when
 //   it grows by more than 2^8, so the O rescale in TMEM is rare
 //   O += P V        (tcgen05.mma M = 64 heads, N <= 256 dims per MMA, V read
@@ -14,7 +15,8 @@
 // TMEM budget: O for 128 heads x 512 dims in fp32 would take all of one SM's
 // tensor memory, so each CTA owns 64 heads (M = 64).  An M = 64 accumulator
 // occupies lanes 0-15 of every 32-lane sub-partition; O sits there (all D
-// columns) and the two S buffers sit at lane offset 16 (columns 0..127).  The
+// columns) and the two S buffers sit at lane offset 16 (columns 0..127), with
+// the item's Q Q^T beside them (columns 128..191).  The
 // 16x32bx2 TMEM access shape keeps every warp inside the lane half it means
 // to touch.  The two head halves of a query are independent CTAs: no cluster,
 // no exchange; each streams the gathered rows itself (the second read of a
@@ -22,16 +24,19 @@
 //
 // Warp roles (256 threads): warp 0 TMEM owner, TMA loader of each work
 // item's raw query rows and MMA issuer (lane 0 issues through guarded
-// instructions); warps 1..3 gather the key rows with 16-byte cp.async into
-// the 128-byte swizzled layout (one 512-byte coalesced row segment per warp
-// instruction) from kernel entry on, each tile's key-validity mask travelling
-// with it; warps 4..7 normalise Q_hat in place, then run the softmax, two
+// instructions); warps 1..3 gather the key rows into the 128-byte swizzled
+// layout from kernel entry on (warps 1, 2: 16-byte cp.async, one 512-byte
+// coalesced row segment per warp instruction; warp 3: TMA gather4 of groups of
+// 4 rows; HCA tiles of consecutive entries: TMA tiles), each tile's
+// key-validity mask travelling with it; warps 4..7 take each head's 1/RMS from the diagonal of Q Q^T
+// (rewriting the query tile only for a gain or RoPE), then run the softmax, two
 // threads per head (keys 0-31 / 32-63, D/2 output columns each), and stage
-// the output through shared memory for coalesced stores.  The roles only
+// the output in shared memory for TMA tile stores.  The roles only
 // meet at mbarriers, so the gathers of the next work item overlap the output
 // of the current one.  Work items are (query, key split, head half); splits
 // write bf16 partial rows (each divided by its own sum) + (max, sum) that
-// attend_combine merges in a fixed order.  Every wait is bounded and every role warp stays converged.
+// attend_combine merges in a fixed order.  Every wait is bounded and every
+// role warp stays converged.
 #include <algorithm>
 #include <cstring>
 
@@ -72,7 +77,7 @@ struct Layout {
 
 struct Smem {
     uint8_t *q, *k, *p;
-    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready, *qready, *qempty, *qfull;
+    uint64_t *kfull, *kempty, *sfull, *sempty, *pfull, *pempty, *oready, *qready, *qempty, *qfull, *qqready;
     uint64_t *kmask;  // [stage] validity of the 64 keys in the stage
     uint32_t *tmem_slot;
     int *abort_flag;
@@ -97,7 +102,8 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
     s.qready = s.oready + 2;
     s.qempty = s.qready + 1;
     s.qfull = s.qempty + 1;
-    s.kmask = s.qfull + 1;
+    s.qqready = s.qfull + 1;
+    s.kmask = s.qqready + 1;
     s.tmem_slot = reinterpret_cast<uint32_t *>(s.kmask + kMaxStages);
     s.abort_flag = reinterpret_cast<int *>(s.tmem_slot + 1);
     return s;
@@ -106,7 +112,7 @@ CSA_DEVINL Smem carve(uint8_t *raw, int stages) {
 template <int D>
 size_t smem_bytes(int stages) {
     using Lt = Layout<D>;
-    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (3 * kMaxStages + 13) * 8 + 16;
+    return 1024 + Lt::kQBytes + (size_t)stages * Lt::kStageBytes + 2 * Lt::kPBytes + (3 * kMaxStages + 14) * 8 + 16;
 }
 
 // ---------------------------------------------------------------- TMEM, 16-lane access shape
@@ -240,19 +246,31 @@ CSA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, 
         : "memory");
 }
 
+// TMA tile store of a [rows][128 B] swizzled shared-memory box (one bulk group
+// per issuing thread; pred selects the issuing lane).
+CSA_DEVINL void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, bool pred) {
+    asm volatile(
+        "{\n\t.reg .pred g;\n\tsetp.ne.b32 g, %5, 0;\n\t"
+        "@g cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];\n\t}"
+        ::"l"(map), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"((int)pred)
+        : "memory");
+}
+
 // Warp-uniform bounded wait.  Every lane polls and the outcome is voted: a
 // wait polled by one lane while the others park at a shuffle leaves the warp
-// running its following code far slower (measured: 4x on the Q_hat pass).
+// running its following code far slower (measured: 4x on a pass over the query tile).
 CSA_DEVINL bool warp_wait(uint32_t bar, uint32_t parity, const DevCtx &ctx, volatile int *abort) {
     const bool ok = mbar_wait(bar, parity, ctx, abort);
     return __all_sync(0xffffffffu, ok);
 }
 
-// ---------------------------------------------------------------- Q_hat
+// ---------------------------------------------------------------- query rows
 // The raw query rows of a work item arrive by TMA, already in the swizzled
 // K-major tile [D/64][64 heads][128 B] (heads past H are zero-filled).  The
-// four softmax warps then normalise them in place, 16 heads each:
-//   Q_hat = RMSNorm(q) * gain * scale * log2(e), bf16.
+// RMSNorm is applied to the scores (each head's 1/RMS from the diagonal of
+// Q Q^T, computed by the tensor cores on the raw rows), so the tile is used as
+// it landed unless a per-channel gain or partial RoPE asks for a rewrite:
+//   Q' = q * gain, then the rotation of the trailing kRopeDim channels.
 // A lane owns whole 16-byte units (8 dims) of a row; every shared-memory
 // access is a conflict-free 16-byte access.
 template <int D>
@@ -269,8 +287,8 @@ struct QLanes {
 // with r0 + j + 4, held by lane ^ 4 in the same slot, so one shuffle fetches
 // the partner values.
 template <int D>
-CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8],
-                            long long t) {
+CSA_DEVINL void rewrite_q(const AttendArgs &a, const Smem &s, int sw, const float (&g)[QLanes<D>::UPL][8],
+                          long long t) {
     using QL = QLanes<D>;
     static_assert(D >= kRopeDim && kRopeDim / 8 == 8, "rope units: 8 per row, partners 4 units apart");
     const int lane = threadIdx.x & 31;
@@ -280,7 +298,6 @@ CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const fl
         const int hl = sw * (kHeads / 4) + pass * QL::RPI + sub;
         uint4 *ptr[QL::UPL];
         float x[QL::UPL][8];
-        float ss = 0.f;
 #pragma unroll
         for (int u = 0; u < QL::UPL; ++u) {
             const int unit = ul + u * QL::LPR;
@@ -288,15 +305,8 @@ CSA_DEVINL void normalize_q(const AttendArgs &a, const Smem &s, int sw, const fl
                                                (((unit & 7) ^ (hl & 7)) << 4));
             unpack8(*ptr[u], x[u]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(x[u][e], x[u][e], ss);
+            for (int e = 0; e < 8; ++e) x[u][e] *= g[u][e];
         }
-#pragma unroll
-        for (int o = QL::LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float r = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
-#pragma unroll
-        for (int u = 0; u < QL::UPL; ++u)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[u][e] = x[u][e] * r * g[u][e];
         if (a.rope_cos) {  // uniform over the grid: every lane takes the shuffles
             constexpr int u = QL::UPL - 1;
             constexpr int r0 = QL::UR - kRopeDim / 8;  // first rotated unit
@@ -348,7 +358,8 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                     const __grid_constant__ CUtensorMap kvgmap, const AttTcParams p) {
+                     const __grid_constant__ CUtensorMap kvgmap, const __grid_constant__ CUtensorMap omap,
+                     const AttTcParams p) {
     using Lt = Layout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem s = carve<D>(smem_raw, p.stages);
@@ -372,9 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(s.qready, 128);
         mbar_init(s.qempty, 1);
         mbar_init(s.qfull, 1);
+        mbar_init(s.qqready, 1);
         *s.abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&qmap);
+        tc::prefetch_tmap(&omap);
         if (p.kv_tma) tc::prefetch_tmap(&kvmap);
         if (!FP8) tc::prefetch_tmap(&kvgmap);
     }
@@ -397,10 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *s.tmem_slot;
     const uint32_t tmem_o = tmem;                  // lanes 0-15 of each sub-partition, columns 0..D-1
     const uint32_t tmem_s = tmem + (16u << 16);    // lanes 16-31, columns 0..127 (two S buffers)
+    const uint32_t tmem_qq = tmem_s + 128;          // lanes 16-31, columns 128..191 (Q Q^T of the item)
+    // the query tile is rewritten in shared memory only for a gain or partial RoPE
+    const bool q_rw = a.q_gain != nullptr || a.rope_cos != nullptr;
 
     // The roles run decoupled across work items; their only contacts are the
     // mbarriers (key ring kfull/kempty, S buffers sfull/sempty, P buffers
-    // pfull/pempty, Q_hat qready/qempty, and oready[g & 1], committed after the
+    // pfull/pempty, the query tile qfull/qqready/qready/qempty, and oready[g & 1], committed after the
     // P.V of tile g).  A parity wait is exact only if the barrier's previous
     // phase is known complete; oready alternates between two barriers because
     // the softmax may wait for P.V g while P.V g-1 is still running, whereas
@@ -556,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x, ++n_items) {
             const Item it = work_item(p, wi);
-            // raw query rows of this item by TMA, once the previous item's QK MMAs are done with Q_hat
+            // raw query rows of this item by TMA, once the previous item's QK MMAs are done with the tile
             if (n_items > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx,
                                                                  s.abort_flag)))
                 break;
@@ -564,6 +580,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < Lt::kChunks; ++c)
                 tc::tma_load_3d(smem_u32(s.q + (size_t)c * kHeads * 128), &qmap, smem_u32(s.qfull), c * 64,
                                 it.head0, (int)it.bq, lane == 0);
+            // Q Q^T of the raw rows: its diagonal gives every head's sum of squares
+            // for the RMSNorm (applied to the scores in fp32)
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag))) break;
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < Lt::kChunks; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16(tmem_qq, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                                qdesc + ((c * kHeads * 128 + kk * 32) >> 4), p.idesc_qk, (c | kk) ? 1u : 0u,
+                                lane == 0);
+            tc::mma_commit(smem_u32(s.qqready), lane == 0);
+            // the softmax warps have read the diagonal (so the next item's Q Q^T may
+            // overwrite it) and, with a gain or RoPE, rewritten the tile
             if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qready), n_items & 1u, p.ctx, s.abort_flag))) break;
             tc::fence_after_sync();
             if (it.ntiles == 0) mbar_arrive(smem_u32(s.qempty), lane == 0);
@@ -589,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
                                             (c | kk) ? 1u : 0u, issuer);
                         tc::mma_commit(smem_u32(s.sfull + sb), issuer);
-                        if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty), issuer);  // Q_hat no longer read
+                        if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty), issuer);  // query tile no longer read
                         ++nqk;
                         progressed = true;
                     }
@@ -653,8 +683,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h = it.head0 + hl;
             if (!warp_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag)) break;
             const long long tq = __ldg(a.q_pos + it.bq);
-            normalize_q<D>(a, s, sp, qg, tq);
-            tc::fence_proxy_async_smem();
+            // this head's 1 / RMS (times the softmax scale, in log2 units) from the
+            // diagonal of Q Q^T: column hl of row hl, held by the thread of the
+            // head's pair whose 32 columns contain it
+            if (!warp_wait(smem_u32(s.qqready), n_items & 1u, p.ctx, s.abort_flag)) break;
+            tc::fence_after_sync();
+            float rq;
+            {
+                float v[32];
+                tmem_ld_half32(tmem_qq + lane_base, v);
+                tc::tmem_wait_ld();
+                // select v[hl & 31] without an indexed (local-memory) access
+                const int di = hl & 31;
+                float d = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) d += (i == di) ? v[i] : 0.f;
+                const float other = __shfl_xor_sync(0xffffffffu, d, 16);
+                const float ss = kh == (hl >> 5) ? d : other;
+                rq = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
+            }
+            tc::fence_before_sync();
+            if (q_rw) {
+                rewrite_q<D>(a, s, sp, qg, tq);
+                tc::fence_proxy_async_smem();
+            }
             mbar_arrive(smem_u32(s.qready));
 
             float m_run = -INFINITY, l = 0.f;
@@ -681,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float mt = -INFINITY;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    if (!((vmask >> i) & 1u)) sc[i] = -INFINITY;
+                    sc[i] = (vmask >> i) & 1u ? sc[i] * rq : -INFINITY;
                     mt = fmaxf(mt, sc[i]);
                 }
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
@@ -736,10 +788,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(smem_u32(s.pfull + pb));
             }
             if (!ok) break;
-            // output: O / l (one split) or the unnormalised partial + (max, sum).
-            // After the last P.V both P buffers are free; they stage one 64-column
-            // slab of O (64 heads x 64 fp32, 16-byte units swizzled by head) so the
-            // global stores are whole row segments.
+            // output: O / l (one split, the output rows) or O / l of this split (a
+            // partial row; the merge weighs the splits).  After the last P.V both P
+            // buffers are free: each warp stages its 16 heads' bf16 values of one
+            // 64-column slab there (alternating buffers) and stores them with one TMA
+            // tile store, the next slab's staging overlapping the previous store.
             if (it.ntiles > 0) {
                 const long long gl = jt + it.ntiles - 1;
                 if (!warp_wait(smem_u32(s.oready + (gl & 1)), (uint32_t)((gl >> 1) & 1), p.ctx, s.abort_flag)) break;
@@ -752,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ? l + ((a.sinks && h < a.H) ? exp2f(__ldg(a.sinks + h) * 1.4426950408889634f - m_run) : 0.f)
                                 : l;
             const float inv = L > 0.f ? 1.0f / L : 0.f;
-            uint8_t *stg = s.p;
+            const int orow = (int)(a.splits == 1 ? it.bq : (long long)it.split * a.n_bq + it.bq);
             for (int c = 0; c < D; c += 64) {
                 float v[32];
                 if (it.ntiles > 0) {
@@ -763,44 +816,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) v[i] = 0.f;
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<float4 *>(stg + hl * 256 + (((8 * kh + u) ^ (hl & 7)) << 4)) =
-                        make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
-                __syncwarp();  // a warp stages and stores only its own 16 heads
-                // bf16 rows (the output, or this split's partial): 4 heads per
-                // instruction, 8 lanes x 8 columns each
-                uint16_t *const dst0 = a.splits == 1 ? a.out + (size_t)it.bq * a.H * D
-                                                     : a.part_o + ((size_t)it.split * a.n_bq + it.bq) * a.H * D;
+                for (int i = 0; i < 32; ++i) v[i] *= inv;
+                if (a.splits == 1 && a.rope_cos && c == D - kRopeDim) {
+                    // conjugate rotation of the rotated slice (this 64-column slab):
+                    // column i pairs with i + 32, held by the head's other thread
+                    // (with several splits the merge rotates the merged row)
+                    const bool first = kh == 0;
 #pragma unroll
-                for (int i = 0; i < 16; i += 4) {
-                    const int r = sp * 16 + i + (lane >> 3), cu = lane & 7, hr = it.head0 + r;
-                    const float4 lo = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu) ^ (r & 7)) << 4));
-                    const float4 hi = *reinterpret_cast<const float4 *>(stg + r * 256 + (((2 * cu + 1) ^ (r & 7)) << 4));
-                    float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                    if (a.splits == 1 && a.rope_cos && c == D - kRopeDim) {
-                        // conjugate rotation of the rotated slice (this 64-column slab):
-                        // column 8*cu + e pairs with 8*(cu ^ 4) + e, held by lane ^ 4
-                        // (with several splits the merge rotates the merged row)
-                        float pv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
-                        const bool first = cu < 4;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float2 cs = rope_cs(a, tq, (cu & 3) * 8 + e);
-                            o[e] = first ? o[e] * cs.x + pv[e] * cs.y : o[e] * cs.x - pv[e] * cs.y;
-                        }
+                    for (int i = 0; i < 32; ++i) {
+                        const float pv = __shfl_xor_sync(0xffffffffu, v[i], 16);
+                        const float2 cs = rope_cs(a, tq, i);
+                        v[i] = first ? v[i] * cs.x + pv * cs.y : v[i] * cs.x - pv * cs.y;
                     }
-                    if (hr < a.H) *reinterpret_cast<uint4 *>(dst0 + (size_t)hr * D + c + 8 * cu) = pack8(o);
                 }
-                __syncwarp();  // a warp stages and stores only its own 16 heads
+                uint8_t *buf = s.p + (size_t)((c >> 6) & 1) * Lt::kPBytes;
+                // the store that last read this buffer (two slabs ago) is done with it
+                if (c >= 128) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4 *>(buf + hl * 128 + (((4 * kh + j) ^ (hl & 7)) << 4)) = pack8(v + 8 * j);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                // (a warp whose 16 heads all lie past H stores nothing; a box that
+                // crosses H is clipped by the tensor map)
+                tma_store_3d(&omap, smem_u32(buf + sp * 16 * 128), c, it.head0 + sp * 16, orow,
+                             lane == 0 && it.head0 + sp * 16 < a.H);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
+            // the P buffers are written again by the next item's softmax
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
             if (h < a.H && a.splits > 1 && kh == 0)
                 a.part_ml[((size_t)it.split * a.n_bq + it.bq) * a.H + h] =
                     it.ntiles > 0 ? make_float2(m_run, l) : make_float2(-INFINITY, 0.f);
             jt += it.ntiles;
         }
     }
+    if (warp >= kSoftmaxWarp0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // output stores complete
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -865,8 +918,21 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
                                CU_TENSOR_MAP_SWIZZLE_128B))
             return CSA_ERR_CUDA;
     }
+    CUtensorMap omap;
+    {
+        // the output rows (one split) or the split partial rows: [rows][H][D] bf16,
+        // boxes of 64 dims x 16 heads (one warp's heads), 128-byte swizzle
+        const uint64_t rows = (uint64_t)(a.splits == 1 ? a.n_bq : (long long)a.splits * a.n_bq);
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.H, rows};
+        const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2};
+        const uint32_t box[3] = {64, 16, 1};
+        if (rows > 0x7fffffffULL ||
+            !encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.splits == 1 ? a.out : a.part_o, dims,
+                               strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return CSA_ERR_CUDA;
+    }
     const int grid = (int)std::min<long long>(p.n_work, num_sms());
-    kern<<<grid, kThreads, smem, st>>>(qmap, kvmap, kvgmap, p);
+    kern<<<grid, kThreads, smem, st>>>(qmap, kvmap, kvgmap, omap, p);
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
     return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
 }
