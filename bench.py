@@ -4,8 +4,9 @@
 Headline (one JSON line on rank 0): CSA decode at 128K context -- batch 8, one
 query per sequence at position 131071, m = 4 (32768 compressed entries), 64x128
 indexer, top-k 1024, 128 heads x 512, window 128.  A step is one pass of the
-decode hot path over the resident cache: csa_index -> csa_topk -> csa_attend
-(+ split combine), replayed as a CUDA graph per decode state.  Six decode
+decode hot path over the resident cache: csa_decode_step, i.e. csa_index ->
+csa_topk -> csa_attend (+ split combine) with the top-k and attention kernels
+launched as programmatic dependents, replayed as a CUDA graph per decode state.  Six decode
 states rotate (each has 79 MB of step inputs; 5 x 79 MB pass through the
 126 MB L2 between two uses of one state), so no step finds its inputs in L2
 and no flush is needed between steps.
@@ -241,14 +242,13 @@ def decode_cache_state(csa, wl: W.Workload, device, seed: int):
     return st
 
 
-def csa_decode_step(csa, st, mark=lambda i: None):
+def decode_step(csa, st):
+    """One decode step through the public API: csa_decode_step (csa_index ->
+    csa_topk -> csa_attend, the last two launched as programmatic dependents)."""
     wl = st["wl"]
-    csa.csa_index(st["qI"], st["w"], st["kI"], st["qp"], wl.m, scores=st["S"])
-    mark(0)
-    csa.csa_topk(st["S"], st["qp"], wl.m, wl.k, idx=st["idx"])
-    mark(1)
-    csa.csa_attend(st["q"], st["C"], st["idx"], st.get("win", st.get("A")), st["qp"], wl.W, wl.scale, wl.eps,
-                   out=st["out"], workspace=st["ws"], win_pos0=st.get("win_pos0", 0))
+    csa.csa_decode_step(st["qI"], st["w"], st["kI"], st["q"], st["C"], st.get("win", st.get("A")), st["qp"], wl.m,
+                        wl.k, wl.W, wl.scale, wl.eps, scores=st["S"], idx=st["idx"], out=st["out"],
+                        workspace=st["ws"], win_pos0=st.get("win_pos0", 0))
 
 
 def index_bytes(wl: W.Workload, fp4=False) -> int:
@@ -286,11 +286,11 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
     st = states[0]
     graphs = []
     for S in states:
-        csa_decode_step(csa, S)  # eager first (lazy initialisation outside the capture)
+        decode_step(csa, S)  # eager first (lazy initialisation outside the capture)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            csa_decode_step(csa, S)
+            decode_step(csa, S)
         graphs.append(g)
     torch.cuda.synchronize()
 
@@ -389,8 +389,8 @@ def e2e_csa_decode(csa, states, args, device, world, rank):
     """Same metric through the public API with the step's inputs on the host.
     Every step copies q, q_I, w and q_pos from pinned host memory and reads the
     attention output back.  As a serving loop would, each decode state's step
-    (the H2D copies, the csa_index / csa_topk / csa_attend calls, the D2H
-    copy) is captured once in a CUDA graph; consecutive steps use different
+    (the H2D copies, the csa_decode_step call, the D2H copy) is captured once
+    in a CUDA graph; consecutive steps use different
     states, replayed on their own streams, so one step's copies overlap its
     neighbours' kernels.  The states' step inputs (4 x 79 MB) exceed the L2,
     so no step finds its inputs in L2 and no flush is needed between steps."""
@@ -407,7 +407,7 @@ def e2e_csa_decode(csa, states, args, device, world, rank):
         S = states[j]
         for k in names:
             S[k].copy_(host_in[j][k], non_blocking=True)
-        csa_decode_step(csa, S)
+        decode_step(csa, S)
         host_out[j].copy_(S["out"], non_blocking=True)
 
     graphs = []

@@ -272,6 +272,28 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
                uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * csa_decode_step -- one CSA step as a single call: csa_index -> csa_topk ->
+ * csa_attend on the same stream, with the results of the three calls
+ * (scores, idx, out).  The top-k and attention kernels are launched as
+ * programmatic dependents of their predecessor: each starts while the
+ * previous kernel finishes and waits for it only before reading its output,
+ * so the attention's query load and RMSNorm overlap the top-k.  This is safe
+ * because the predecessors are the library's own kernels; the separate calls
+ * are ordinary launches.
+ *   q_idx, w, k_idx, H_I, d_I, m: as csa_index (scores [batch][nq][N] fp32 is
+ *   written, caller-owned); k, idx: as csa_topk; q .. out, workspace: as
+ *   csa_attend (workspace: csa_attend_workspace_bytes(batch, nq, H, D, k + W)).
+ * Requirements: those of the three calls; every argument is checked before
+ * anything is launched.
+ */
+int csa_decode_step(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, int H_I, int d_I, int m, int k,
+                    float *scores, int *idx, const uint16_t *q, const float *q_gain, const float *sinks,
+                    const float *rope_cos, const float *rope_sin, long long rope_positions, const uint16_t *kv,
+                    long long N, const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
+                    const int *q_pos, int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * csa_attend_noalloc -- csa_attend for callers that cannot allocate device
  * memory.  No passage of the pages corresponds to it: it is a deployment
  * convenience of this library.

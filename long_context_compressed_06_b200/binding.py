@@ -58,6 +58,8 @@ def load() -> ctypes.CDLL:
         "csa_attend": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P],
                        i32),
         "hca_attend": ([P, P, P, P, P, i64, P, i64, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P, sz, P], i32),
+        "csa_decode_step": ([P, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, i64, P, i64, P, i64, i64, i32, P, i32, i32,
+                             i32, i32, f32, f32, P, P, sz, P], i32),
         "csa_attend_noalloc": ([P, P, P, P, P, i64, P, i64, P, i32, P, i64, i64, i32, P, i32, i32, i32, i32, f32, f32, P, P],
                                i32),
         "csa_sync_status": ([P], i32),
@@ -291,6 +293,38 @@ def csa_attend(q, kv, idx, win, q_pos, W: int, scale: float, eps: float = 1e-6, 
                         _p(q_pos),
                         batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()), "csa_attend")
     return out
+
+
+def csa_decode_step(q_idx, w, k_idx, q, kv, win, q_pos, m: int, k: int, W: int, scale: float, eps: float = 1e-6,
+                    q_gain=None, scores=None, idx=None, out=None, workspace=None, win_pos0: int = 0, sinks=None,
+                    rope=None):
+    """csa_index -> csa_topk -> csa_attend as one call (the top-k and attention kernels launched as
+    programmatic dependents of their predecessor); returns (scores, idx, out)."""
+    L = load()
+    _need(q_idx, torch.bfloat16, "q_idx", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(k_idx, torch.bfloat16, "k_idx", 3)
+    _need(q, torch.bfloat16, "q", 4)
+    _need(kv, torch.bfloat16, "kv", 3)
+    _need(win, torch.bfloat16, "win", 3)
+    _need(q_pos, torch.int32, "q_pos", 2)
+    batch, nq, H_I, d_I = q_idx.shape
+    H, D = q.shape[2], q.shape[3]
+    N, rows = k_idx.shape[1], win.shape[1]
+    if kv.shape[1] != N:
+        raise ValueError("kv and k_idx must hold the same number of entries")
+    if scores is None:
+        scores = torch.empty((batch, nq, N), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((batch, nq, k), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _workspace(attend_workspace_bytes(batch, nq, H, D, k + W), q.device, workspace)
+    _check(L.csa_decode_step(_p(q_idx), _p(w), _p(k_idx), H_I, d_I, m, k, _p(scores), _p(idx), _p(q), _p(q_gain),
+                             _sinks(sinks, H), *_rope(rope, D), _p(kv), N, _p(win), int(win_pos0), rows, W, _p(q_pos),
+                             batch, nq, H, D, float(scale), float(eps), _p(out), _p(ws), wsb, _stream()),
+           "csa_decode_step")
+    return scores, idx, out
 
 
 def hca_attend(q, kv, m: int, win, q_pos, W: int, scale: float, eps: float = 1e-6, q_gain=None, out=None,

@@ -270,6 +270,35 @@ int hca_attend(const uint16_t *q, const float *q_gain, const float *sinks, const
                               nq, H, D, scale, eps, out, workspace, workspace_bytes, ctx, S(stream));
 }
 
+int csa_decode_step(const uint16_t *q_idx, const float *w, const uint16_t *k_idx, int H_I, int d_I, int m, int k,
+                    float *scores, int *idx, const uint16_t *q, const float *q_gain, const float *sinks,
+                    const float *rope_cos, const float *rope_sin, long long rope_positions, const uint16_t *kv,
+                    long long N, const uint16_t *win_src, long long win_pos0, long long win_rows, int W,
+                    const int *q_pos, int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    // every argument of the three calls first: nothing is launched for a bad one
+    if (!al16(q_idx) || !al4(w) || !al16(k_idx) || !al4(q_pos) || !al16(scores) || !al4(idx)) return CSA_ERR_INVALID;
+    if (batch < 1 || nq < 1 || N < 1 || H_I < 1 || d_I < 16 || d_I % 16 != 0 || m < 1 || k < 1)
+        return CSA_ERR_INVALID;
+    if (!csa::index_tc_supported(H_I, d_I) || k > 8192 || N > (1LL << 19)) return CSA_ERR_UNSUPPORTED;
+    if (csa::topk_workspace_bytes(batch, nq, N, k) != 0) return CSA_ERR_UNSUPPORTED;
+    int rc = csa::check_attend_args(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, kv, N, idx, k, win_src,
+                                    win_pos0, win_rows, W, q_pos, batch, nq, H, D, eps, out);
+    if (rc != CSA_OK) return rc;
+    if (workspace_bytes < csa::attend_workspace_bytes(batch, nq, H, D, (long long)k + W) ||
+        (workspace_bytes > 0 && !al16(workspace)))
+        return CSA_ERR_WORKSPACE;
+    csa::DevCtx ctx;
+    if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
+    rc = csa::launch_index(q_idx, w, k_idx, q_pos, batch, nq, N, H_I, d_I, m, scores, ctx, S(stream));
+    if (rc != CSA_OK) return rc;
+    rc = csa::launch_topk(scores, q_pos, batch, nq, N, m, k, idx, S(stream), /*pdl=*/true);
+    if (rc != CSA_OK) return rc;
+    return csa::launch_attend(q, q_gain, sinks, rope_cos, rope_sin, rope_positions, nullptr, kv, N, 1, idx, k, false,
+                              win_src, win_pos0, win_rows, W, q_pos, batch, nq, H, D, scale, eps, out, workspace,
+                              workspace_bytes, ctx, S(stream), /*pdl=*/true);
+}
+
 int csa_quantize_fp8_kv(const uint16_t *x, long long rows, int d, uint8_t *codes, uint8_t *exps, void *stream) {
     if (!al16(x) || !al16(codes) || !exps) return CSA_ERR_INVALID;
     if (rows < 0 || d < 128 || d % 128 != 0) return CSA_ERR_INVALID;

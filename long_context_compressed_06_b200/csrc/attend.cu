@@ -96,7 +96,7 @@ int launch_attend_combine(const AttendArgs &a, cudaStream_t st) {
 
 bool attend_tc_supported(int H, int D);
 void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long long *kps);
-int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st);
+int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st, bool pdl);
 
 // Split plan of the tensor-core kernel for these shapes (one split when the
 // shapes are outside the compiled tiles: the launch then returns
@@ -123,7 +123,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out, void *ws,
-                  size_t ws_bytes, const DevCtx &ctx, cudaStream_t st) {
+                  size_t ws_bytes, const DevCtx &ctx, cudaStream_t st, bool pdl) {
     AttendArgs a = {};
     a.q = q; a.q_gain = q_gain; a.sinks = sinks; a.rope_cos = rope_cos; a.rope_sin = rope_sin;
     a.rope_npos = rope_npos; a.kv = kv;
@@ -143,7 +143,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
         a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(uint16_t));
     }
-    return launch_attend_tc(a, ctx, st);
+    return launch_attend_tc(a, ctx, st, pdl);
 }
 
 }  // namespace csa

@@ -24,14 +24,14 @@
 //
 // Warp roles (256 threads): warp 0 TMEM owner, TMA loader of each work
 // item's raw query rows and MMA issuer (lane 0 issues through guarded
-// instructions); warps 1..3 gather the key rows into the 128-byte swizzled
-// layout from kernel entry on (warps 1, 2: 16-byte cp.async, one 512-byte
-// coalesced row segment per warp instruction; warp 3: TMA gather4 of groups of
-// 4 rows; HCA tiles of consecutive entries: TMA tiles), each tile's
-// key-validity mask travelling with it; warps 4..7 take each head's 1/RMS from the diagonal of Q Q^T
-// (rewriting the query tile only for a gain or RoPE), then run the softmax, two
-// threads per head (keys 0-31 / 32-63, D/2 output columns each), and stage
-// the output in shared memory for TMA tile stores.  The roles only
+// instructions); warps 1..3 gather the key rows with 16-byte cp.async into
+// the 128-byte swizzled layout (one 512-byte coalesced row segment per warp
+// instruction; HCA tiles of consecutive entries arrive as TMA tiles instead)
+// from kernel entry on, each tile's key-validity mask travelling with it;
+// warps 4..7 take each head's 1/RMS from the diagonal of Q Q^T (rewriting the
+// query tile only for a gain or RoPE), then run the softmax, two threads per
+// head (keys 0-31 / 32-63, D/2 output columns each), and stage the output in
+// shared memory for TMA tile stores.  The roles only
 // meet at mbarriers, so the gathers of the next work item overlap the output
 // of the current one.  Work items are (query, key split, head half); splits
 // write bf16 partial rows (each divided by its own sum) + (max, sum) that
@@ -235,17 +235,6 @@ CSA_DEVINL uint4 e4m3x8_bf16x8(uint2 raw, uint32_t e) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// TMA gather of 4 rows (row indices r0..r3 of a [rows][D] map with a 64 x 1
-// box) x 64 dims into 4 consecutive 128-byte rows at dst (swizzled by address).
-CSA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int r0, int r1, int r2,
-                            int r3, bool pred) {
-    asm volatile(
-        "{\n\t.reg .pred g;\n\tsetp.ne.b32 g, %8, 0;\n\t"
-        "@g cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n\t}"
-        ::"r"(dst), "l"(map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar), "r"((int)pred)
-        : "memory");
-}
-
 // TMA tile store of a [rows][128 B] swizzled shared-memory box (one bulk group
 // per issuing thread; pred selects the issuing lane).
 CSA_DEVINL void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, bool pred) {
@@ -358,8 +347,7 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                     const __grid_constant__ CUtensorMap kvgmap, const __grid_constant__ CUtensorMap omap,
-                     const AttTcParams p) {
+                     const __grid_constant__ CUtensorMap omap, const AttTcParams p) {
     using Lt = Layout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem s = carve<D>(smem_raw, p.stages);
@@ -389,7 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::prefetch_tmap(&qmap);
         tc::prefetch_tmap(&omap);
         if (p.kv_tma) tc::prefetch_tmap(&kvmap);
-        if (!FP8) tc::prefetch_tmap(&kvgmap);
     }
     // per-dimension query gains of this lane's units (softmax warps), read once
     float qg[QLanes<D>::UPL][8];
@@ -431,14 +418,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pw = warp - kProducerWarp0;
         long long jt = 0;
         bool ok = true;
+        bool dep_done = false;
         for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x) {
             const Item it = work_item(p, wi);
+            // As a programmatic dependent (csa_decode_step) the selection is
+            // complete only once the top-k grid is: wait before the first item
+            // that reads selected slots (the query prologue and the window-only
+            // items run meanwhile).  A no-op for an ordinary launch.
+            if (!dep_done && !a.dense && it.e0 < it.ks.nsel4) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                dep_done = true;
+            }
             for (int j = 0; j < it.ntiles; ++j) {
                 const long long g = jt + j;
                 const int st = (int)(g % p.stages);
                 const long long ebase = it.e0 + (long long)j * kTileKeys;
-                bool v0, v1, w1 = true;
-                int row1 = 0;  // kv row (b * N + entry) of key 32 + lane when w1 is false
+                bool v0, v1;
                 const uint16_t *r0 = nullptr, *r1 = nullptr;
                 const uint8_t *c0 = nullptr, *c1 = nullptr, *x0 = nullptr, *x1 = nullptr;
                 if constexpr (FP8) {
@@ -446,9 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     c1 = key_slot8(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1, x1);
                 } else {
                     r0 = key_slot(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0);
-                    const size_t ri = key_row_index(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1, w1);
-                    r1 = (w1 ? a.win : a.kv) + ri * a.D;
-                    row1 = (int)ri;
+                    r1 = key_slot(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1);
                 }
                 const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
                 if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag)) {
@@ -500,11 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(smem_u32(s.kfull + st), lane == 0);
                     }
                 } else {
-                    // Two paths into the swizzled stage at once (their in-flight limits add
-                    // up): warps 0 and 1 copy keys 0..31 with 16-byte cp.async; warp 2 loads
-                    // each group of 4 of keys 32..63 whose rows all lie in kv with TMA
-                    // gather4 (one per 64-dim chunk), and cp.asyncs the other groups' rows.
-                    const auto cp_row = [&](int key, const uint16_t *row) {
+                    // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l,
+                    // l+32, .. of the row (coalesced 512 B per instruction).
+#pragma unroll 2
+                    for (int key = pw; key < kTileKeys; key += kProducerWarps) {
+                        const uint16_t *row = reinterpret_cast<const uint16_t *>(
+                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? r0 : r1), key & 31));
                         const uint32_t krow = stage + key * 128;
 #pragma unroll
                         for (int u = lane; u < D / 8; u += 32) {  // 16-byte units of the row
@@ -512,40 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(row + u * 8)
                                          : "memory");
                         }
-                    };
-                    if (pw < kProducerWarps - 1) {
-#pragma unroll 2
-                        for (int key = pw; key < 32; key += kProducerWarps - 1)
-                            cp_row(key, reinterpret_cast<const uint16_t *>(
-                                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(r0), key)));
-                    } else {
-                        const uint32_t kvm = __ballot_sync(0xffffffffu, !w1);
-                        uint32_t groups = 0;  // bit q: keys 32+4q .. 32+4q+3 all in kv
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) groups |= ((kvm >> (4 * q)) & 0xfu) == 0xfu ? (1u << q) : 0u;
+                    }
+                    if (pw == 0) {  // the mask travels with the tile (release by lane 0's arrive)
                         if (lane == 0) s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
-                        // the mask arrive carries the TMA byte count (release by lane 0)
-                        mbar_arrive_expect_tx(smem_u32(s.kfull + st), (uint32_t)__popc(groups) * 4u * D * 2u,
-                                              lane == 0);
-#pragma unroll 1
-                        for (int q = 0; q < 8; ++q) {
-                            if ((groups >> q) & 1u) {
-                                const int g0 = __shfl_sync(0xffffffffu, row1, 4 * q);
-                                const int g1 = __shfl_sync(0xffffffffu, row1, 4 * q + 1);
-                                const int g2 = __shfl_sync(0xffffffffu, row1, 4 * q + 2);
-                                const int g3 = __shfl_sync(0xffffffffu, row1, 4 * q + 3);
-#pragma unroll
-                                for (int c = 0; c < Lt::kChunks; ++c)
-                                    tma_gather4(stage + c * (kTileKeys * 128) + (32 + 4 * q) * 128, &kvgmap,
-                                                smem_u32(s.kfull + st), c * 64, g0, g1, g2, g3, lane == 0);
-                            } else {
-                                for (int k4 = 0; k4 < 4; ++k4) {
-                                    const int key = 32 + 4 * q + k4;
-                                    cp_row(key, reinterpret_cast<const uint16_t *>(__shfl_sync(
-                                                    0xffffffffu, reinterpret_cast<uintptr_t>(r1), key - 32)));
-                                }
-                            }
-                        }
+                        mbar_arrive(smem_u32(s.kfull + st), lane == 0);
                     }
                     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(s.kfull + st))
                                  : "memory");
@@ -869,7 +833,7 @@ constexpr uint32_t idesc_m64(int n, bool b_mn) {
 }
 
 template <int D, bool FP8>
-int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
+int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st, bool pdl) {
     AttTcParams p = {};
     p.a = a;
     p.ctx = ctx;
@@ -906,18 +870,6 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
                                CU_TENSOR_MAP_SWIZZLE_128B))
             return CSA_ERR_CUDA;
     }
-    CUtensorMap kvgmap;
-    memset(&kvgmap, 0, sizeof(kvgmap));
-    if (!FP8) {
-        if ((a.n_bq / a.nq) * a.N > 0x7fffffffLL) return CSA_ERR_UNSUPPORTED;  // gather4 rows are int32
-        // kv as [batch * N rows][D] bf16: boxes of 64 dims x 1 row for gather4, 128-byte swizzle
-        const uint64_t dims[2] = {(uint64_t)D, (uint64_t)(a.n_bq / a.nq) * (uint64_t)a.N};
-        const uint64_t strides[1] = {(uint64_t)D * 2};
-        const uint32_t box[2] = {64, 1};
-        if (!encode_tensor_map(&kvgmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.kv, dims, strides, box,
-                               CU_TENSOR_MAP_SWIZZLE_128B))
-            return CSA_ERR_CUDA;
-    }
     CUtensorMap omap;
     {
         // the output rows (one split) or the split partial rows: [rows][H][D] bf16,
@@ -932,8 +884,17 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st) {
             return CSA_ERR_CUDA;
     }
     const int grid = (int)std::min<long long>(p.n_work, num_sms());
-    kern<<<grid, kThreads, smem, st>>>(qmap, kvmap, kvgmap, omap, p);
-    if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, qmap, kvmap, omap, p) != cudaSuccess) return CSA_ERR_CUDA;
     return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
 }
 
@@ -966,20 +927,20 @@ void attend_tc_plan(long long n_bq, int H, long long max_keys, int *splits, long
     *kps = ((tiles + best - 1) / best) * kTileKeys;
 }
 
-int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st) {
+int launch_attend_tc(AttendArgs a, const DevCtx &ctx, cudaStream_t st, bool pdl) {
     if (a.kv8) {  // FP8 rows: 128-channel scale blocks
         switch (a.D) {
-            case 128: return launch_d<128, true>(a, ctx, st);
-            case 256: return launch_d<256, true>(a, ctx, st);
-            case 512: return launch_d<512, true>(a, ctx, st);
+            case 128: return launch_d<128, true>(a, ctx, st, pdl);
+            case 256: return launch_d<256, true>(a, ctx, st, pdl);
+            case 512: return launch_d<512, true>(a, ctx, st, pdl);
             default: return CSA_ERR_UNSUPPORTED;
         }
     }
     switch (a.D) {
-        case 64: return launch_d<64, false>(a, ctx, st);
-        case 128: return launch_d<128, false>(a, ctx, st);
-        case 256: return launch_d<256, false>(a, ctx, st);
-        case 512: return launch_d<512, false>(a, ctx, st);
+        case 64: return launch_d<64, false>(a, ctx, st, pdl);
+        case 128: return launch_d<128, false>(a, ctx, st, pdl);
+        case 256: return launch_d<256, false>(a, ctx, st, pdl);
+        case 512: return launch_d<512, false>(a, ctx, st, pdl);
         default: return CSA_ERR_UNSUPPORTED;
     }
 }

@@ -114,6 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
+    // a successor launched as a programmatic dependent (csa_decode_step's top-k)
+    // may start now; it waits for this grid before reading the scores
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long w0 = (long long)blockIdx.x * p.total_work / gridDim.x;
     const long long w1 = (long long)(blockIdx.x + 1) * p.total_work / gridDim.x;

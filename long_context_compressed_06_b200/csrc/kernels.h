@@ -34,8 +34,11 @@ int launch_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, cons
 
 size_t topk_workspace_bytes(int batch, int nq, long long N, int k);
 // q_pos may be null inside the library: every entry is then eligible.
+// pdl: launched as a programmatic dependent of the stream's previous kernel
+// (the kernel waits for it before reading scores) -- only for chains whose
+// predecessor is this library's own kernel (csa_decode_step).
 int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k,
-                int *idx, cudaStream_t st);
+                int *idx, cudaStream_t st, bool pdl = false);
 
 size_t rescore_workspace_bytes(int batch, int nq, int kc, int k, int d_I);
 bool rescore_supported(int H_I, int d_I);
@@ -64,7 +67,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
                   const int *idx, int k, bool dense, const uint16_t *win, long long win_pos0, long long win_rows,
                   int W, const int *q_pos,
                   int batch, int nq, int H, int D, float scale, float eps, uint16_t *out,
-                  void *ws, size_t ws_bytes, const DevCtx &ctx, cudaStream_t st);
+                  void *ws, size_t ws_bytes, const DevCtx &ctx, cudaStream_t st, bool pdl = false);
 
 int launch_selftest_wait(const DevCtx &ctx, cudaStream_t st);
 

@@ -92,6 +92,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     __shared__ uint32_t s_min, s_max, s_bin, s_cnt;
     __shared__ long long s_krem;
 
+    // as a programmatic dependent: the scores are complete only once the
+    // predecessor grid is (a no-op otherwise); the successor may launch now
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = threadIdx.x; i < 2 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
 
     const long long nv = q_pos ? n_visible(q_pos[bq], m, N) : N;  // no q_pos: every entry is eligible
@@ -271,7 +275,7 @@ TopkPlan plan(long long n_queries, long long N) {
 size_t topk_workspace_bytes(int, int, long long, int) { return 0; }
 
 int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long long N, int m, int k, int *idx,
-                cudaStream_t st) {
+                cudaStream_t st, bool pdl) {
     const long long nqry = (long long)batch * nq;
     if (nqry == 0) return CSA_OK;
     const TopkPlan pl = plan(nqry, N);
@@ -293,13 +297,22 @@ int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long l
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.CS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (cl) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = pl.CS;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = cl ? 1 : 0;
+    cfg.numAttrs = na;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, scores, q_pos, N, m, k, idx, pl.CS);
     return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }

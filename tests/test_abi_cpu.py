@@ -248,3 +248,28 @@ def test_missing_library_raises(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="not built"):
         binding.load()
+
+
+def test_decode_step_validates_every_argument_first(lib):
+    """csa_decode_step refuses a bad argument of any of its three calls before
+    launching anything (only invalid calls here: a valid one would launch)."""
+    f = lib.csa_decode_step
+
+    def call(q_idx=A16, k_idx=A16, H_I=64, d_I=128, m=4, k=1024, scores=A16b, idx=A16, q=A16, kv=A16, W=128,
+             H=128, D=512, out=A16b, ws=NULL, wsb=0):
+        return f(q_idx, A16, k_idx, H_I, d_I, m, k, scores, idx, q, NULL, NULL, NULL, NULL, 0, kv, 32768, A16, 0,
+                 128, W, A16, 8, 1, H, D, 0.05, 1e-6, out, ws, wsb, NULL)
+
+    assert call(q_idx=NULL) == csa.CSA_ERR_INVALID
+    assert call(scores=MIS) == csa.CSA_ERR_INVALID
+    assert call(idx=ctypes.c_void_p(0x10002)) == csa.CSA_ERR_INVALID
+    assert call(d_I=120) == csa.CSA_ERR_INVALID
+    assert call(m=0) == csa.CSA_ERR_INVALID
+    assert call(k=0) == csa.CSA_ERR_INVALID
+    assert call(d_I=48) == csa.CSA_ERR_UNSUPPORTED
+    assert call(k=9000) == csa.CSA_ERR_UNSUPPORTED
+    assert call(q=NULL) == csa.CSA_ERR_INVALID
+    assert call(W=0) == csa.CSA_ERR_INVALID
+    assert call(D=96) == csa.CSA_ERR_UNSUPPORTED
+    assert call(H=256) == csa.CSA_ERR_UNSUPPORTED
+    assert call() == csa.CSA_ERR_WORKSPACE        # 8 decode queries need split scratch

@@ -198,3 +198,27 @@ def test_fp4_index_1m_scores_and_recall(cuda):
           % (wl.k, r1, 4 * wl.k, r2))
     assert r2 >= 0.99, r2
     assert r1 >= 0.8, r1
+
+
+# ----------------------------------------------------------------------------- the step as one call
+@pytest.mark.parametrize("wl", [W.TINY, W.CSA_DECODE], ids=lambda w: w.name)
+def test_decode_step_equals_the_three_calls(cuda, wl):
+    """csa_decode_step (top-k and attention launched as programmatic dependents)
+    gives bit for bit the scores, selection and output of csa_index, csa_topk
+    and csa_attend called one after the other, twice in a row."""
+    qI, w, kI = W.index_queries(wl, DEV), W.index_weights(wl, DEV), W.index_keys(wl, DEV)
+    qp = wl.q_positions().to(DEV)
+    q = W.queries(wl, DEV)
+    kv = W.direct_kv(wl, DEV)
+    win = W.normal_bf16((wl.batch, wl.W, wl.D), 31, DEV)
+    p0 = wl.T - wl.W
+    S = cuda.csa_index(qI, w, kI, qp, wl.m)
+    idx = cuda.csa_topk(S, qp, wl.m, wl.k)
+    out = cuda.csa_attend(q, kv, idx, win, qp, wl.W, wl.scale, wl.eps, win_pos0=p0)
+    for _ in range(2):
+        S2, idx2, out2 = cuda.csa_decode_step(qI, w, kI, q, kv, win, qp, wl.m, wl.k, wl.W, wl.scale, wl.eps,
+                                              win_pos0=p0)
+        assert cuda.csa_sync_status() == 0
+        assert torch.equal(S2, S)
+        assert torch.equal(idx2, idx)
+        assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
