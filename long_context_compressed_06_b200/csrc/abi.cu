@@ -148,8 +148,9 @@ int csa_index_fp4(const uint8_t *q4, const uint8_t *q4s, const float *w, const u
     if (batch < 1 || nq < 1 || N < 1 || H_I < 1 || d_I < 16 || d_I % 16 != 0 || m < 1)
         return CSA_ERR_INVALID;
     if (!csa::index_fp4_tc_supported(H_I, d_I) || N > (1LL << 31) - 1) return CSA_ERR_UNSUPPORTED;
-    // each key's d_I/16 scale bytes move as one copy aligned to their size
-    if (reinterpret_cast<uintptr_t>(k4s) % (uintptr_t)(d_I / 16) != 0 || reinterpret_cast<uintptr_t>(q4s) % 2 != 0)
+    // each key's d_I/16 scale bytes move as one copy aligned to their size; the
+    // query scales are read as 32-bit words
+    if (reinterpret_cast<uintptr_t>(k4s) % (uintptr_t)(d_I / 16) != 0 || reinterpret_cast<uintptr_t>(q4s) % 4 != 0)
         return CSA_ERR_INVALID;
     csa::DevCtx ctx;
     if (!ctx_for_launch(&ctx)) return CSA_ERR_CUDA;
