@@ -712,6 +712,17 @@ def run_reference(args):
     return 0
 
 
+def decode_for_profiling(csa, args, device):
+    """One 128K decode state (cache built by csa_compress) and warmup + steps
+    eager decode steps, for kernel profilers: a few hundred MB on the device
+    and no other launches than the cache build and the steps."""
+    st = decode_cache_state(csa, W.CSA_DECODE, device, 0)
+    for _ in range(args.warmup + args.steps):
+        decode_step(csa, st)
+    torch.cuda.synchronize()
+    return {"workload": "csa_decode_128k", "steps": args.warmup + args.steps, "note": "profiling run, not timed"}
+
+
 def decode_config(wl: W.Workload, world: int) -> dict:
     """The headline workload as both arms name it."""
     return {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.T, "m": wl.m, "entries": wl.N,
@@ -729,8 +740,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress", "compress_dynamic", "fp8kv"],
-                    help="run one of the other workloads alone and print its JSON (for profiling)")
+    ap.add_argument("--only", choices=["prefill", "hca", "fp4", "compress", "compress_dynamic", "fp8kv", "decode"],
+                    help="run one workload alone and print its JSON (for profiling); 'decode' builds one 128K "
+                         "decode state and runs warmup + steps eager csa_decode_step calls")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -750,6 +762,7 @@ def main():
                    "compress": lambda: bench_compress(csa, args, device, peaks, W.HCA_DECODE),
                    "compress_dynamic": lambda: bench_compress_dynamic(csa, args, device, peaks, W.CSA_DECODE),
                    "fp8kv": lambda: bench_fp8kv_decode(csa, args, device, peaks),
+                   "decode": lambda: decode_for_profiling(csa, args, device),
                    }[args.only]
         res = run_one()
         rc = csa.csa_sync_status()
