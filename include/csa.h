@@ -160,9 +160,10 @@ int csa_quantize_fp4(const uint16_t *x, long long rows, int d,
 /*
  * csa_index_fp4 -- csa_index on FP4 operands (layouts of csa_quantize_fp4):
  * the score is the same formula on the dequantised values e2m1 * e4m3, with
- * exact products and fp32 accumulation, on the tensor cores.  d_I in
- * {64, 128, 256} (else CSA_ERR_UNSUPPORTED); k4s aligned to d_I/16 bytes and
- * q4s to 4 bytes (else CSA_ERR_INVALID).
+ * exact products and fp32 accumulation: block-scaled FP4 tensor-core MMAs
+ * multiply the e2m1 codes and apply both operands' e4m3 block scales.  d_I in
+ * {64, 128, 256}, H_I <= 128 (else CSA_ERR_UNSUPPORTED); k4s aligned to d_I/16
+ * bytes and q4s to 4 bytes (else CSA_ERR_INVALID).
  *   q4 [batch][nq][H_I][d_I/2]   q4s [batch][nq][H_I][d_I/16]   w [batch][nq][H_I] fp32
  *   k4 [batch][N][d_I/2]         k4s [batch][N][d_I/16]         scores [batch][nq][N] fp32
  * Requirements: as csa_index.

@@ -141,7 +141,7 @@ def test_index_validation(lib):
     assert g(A16, odd, A16, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == csa.CSA_ERR_INVALID  # q4s
     assert g(A16, ctypes.c_void_p(0x10002), A16, A16, A16, A16, 1, 1, 100, 64, 128, 4, A16b, NULL) == \
         csa.CSA_ERR_INVALID                                                                             # q4s % 4
-    assert g(A16, A16, A16, A16, A16, A16, 1, 1, 100, 512, 128, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED  # H_I
+    assert g(A16, A16, A16, A16, A16, A16, 1, 1, 100, 256, 128, 4, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED  # H_I
 
 
 def test_quantize_validation(lib):
