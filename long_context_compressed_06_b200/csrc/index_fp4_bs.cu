@@ -22,14 +22,16 @@
 // n % 32, column n / 32 of the block, copied into each of the four lane
 // quarters (the rows of A in a quarter read B's scale factors there).
 //
-// Warp roles (448 threads): warp 0 -- TMA producer (key tiles into a ring of
+// Warp roles (704 threads): warp 0 -- TMA producer (key tiles into a ring of
 // stages, the query group's codes once per group); warp 1 -- TMEM owner and
 // MMA issuer (lane 0 issues through guarded instructions); warps 2..5 -- scale
 // movers (each thread stages its key row's scale bytes with cp.async several
 // tiles ahead and writes them into the tile's tensor-memory slot; the
-// query-head scales once per group); warps 6..13 -- two epilogue groups of four
-// warps taking alternate tiles (tcgen05.ld, ReLU, weighted head sum, causal
-// mask, store).  Every wait is bounded and every role warp stays converged.
+// query-head scales once per group); warps 6..21 -- four epilogue groups of
+// four warps taking the tiles in turn (tcgen05.ld, ReLU, weighted head sum,
+// causal mask, store): at 9 KiB per tile the tiles arrive every ~0.2 us per
+// SM at HBM speed, faster than one group's per-tile latency.  Every wait is
+// bounded and every role warp stays converged.
 #include <algorithm>
 #include <cstring>
 
@@ -40,9 +42,10 @@
 namespace csa {
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kEpiGroups = 4;  // epilogue groups of four warps, taking tiles in turn
+constexpr int kThreads = 192 + 128 * kEpiGroups;
 constexpr int kTileKeys = 128;
-constexpr int kMaxStages = 12;
+constexpr int kMaxStages = 20;
 constexpr int kMaxAcc = 4;
 constexpr int kSfSlots = 8;     // key-scale slots in tensor memory (tiles in flight)
 constexpr int kSfAhead = 4;     // tiles whose key scales a mover thread prefetches
@@ -101,12 +104,8 @@ struct Ring {
     }
 };
 
-CSA_DEVINL void group_bar(int eg) {
-    if (eg == 0)
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-    else
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-}
+// Named barrier of one epilogue group (128 threads), ids 1..kEpiGroups.
+CSA_DEVINL void group_bar(int eg) { asm volatile("bar.sync %0, 128;" ::"r"(eg + 1) : "memory"); }
 
 // Block-scaled FP4 MMA: D (+)= A . B^T with per-16-element scale factors of A
 // and B read from tensor memory at sfa / sfb.
@@ -148,10 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *k_smem = base;
     uint8_t *q_smem = k_smem + (size_t)p.stages * p.stage_bytes;
     uint8_t *sf_smem = q_smem + ((p.q_bytes + 1023u) & ~1023u);            // [kSfAhead][128 rows][KB]
-    float *w_s = reinterpret_cast<float *>(sf_smem + kSfAhead * kTileKeys * KB);  // [2 groups][NQ][H_pad]
-    int *nvis_s = reinterpret_cast<int *>(w_s + 2 * p.NQ * p.H_pad);      // [2 groups][NQ]
+    float *w_s = reinterpret_cast<float *>(sf_smem + kSfAhead * kTileKeys * KB);  // [groups][NQ][H_pad]
+    int *nvis_s = reinterpret_cast<int *>(w_s + kEpiGroups * p.NQ * p.H_pad);     // [groups][NQ]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
-        (reinterpret_cast<uintptr_t>(nvis_s + 2 * p.NQ) + 7) & ~uintptr_t(7));
+        (reinterpret_cast<uintptr_t>(nvis_s + kEpiGroups * p.NQ) + 7) & ~uintptr_t(7));
     uint64_t *full = bars, *empty = bars + kMaxStages;
     uint64_t *tfull = empty + kMaxStages, *tempty = tfull + kMaxAcc;
     uint64_t *sfull = tempty + kMaxAcc, *sempty = sfull + kSfSlots;       // key-scale slots
@@ -342,19 +341,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
-        // ------------------------------------------------------------ epilogue (warps 6..13)
-        // Two groups of four warps take alternate tiles (tile i -> group i & 1,
-        // accumulator i % n_acc).
+        // ------------------------------------------------------------ epilogue (warps 6..21)
+        // kEpiGroups groups of four warps take the tiles in turn (tile i -> group
+        // i % kEpiGroups, accumulator i % n_acc).
         const int eg = (warp - 6) >> 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
-        const int et = (threadIdx.x - 192) & 127;
+        const int et = (threadIdx.x - 192) & 127;  // thread within its group
         float *ws_g = w_s + eg * p.NQ * p.H_pad;
         int *nv_g = nvis_s + eg * p.NQ;
         int loaded_b = -1, loaded_g = -1;
         for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
             const int li = (int)(cu.w - w0);
-            if ((li & 1) != eg) continue;
+            if (li % kEpiGroups != eg) continue;
             const int b = cu.b, g = cu.g;
             if (b != loaded_b || g != loaded_g) {
                 group_bar(eg);
@@ -381,24 +380,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int qi = 0; qi < p.NQ; ++qi) {
                 const int q = g * p.NQ + qi;
                 if (q >= p.nq) break;
-                float part[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int hc = 0; hc < p.H_pad; hc += 64) {
-                    float v[64];
-                    const int nl = min(4, (p.H_pad - hc) >> 4);
+                // 32 columns per TMEM load round (two 16-column loads in flight), two
+                // partial sums per round keep the FMA chains short
+                float part[2] = {0.f, 0.f};
+                for (int hc = 0; hc < p.H_pad; hc += 32) {
+                    float v[32];
+                    const int nl = min(2, (p.H_pad - hc) >> 4);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 2; ++u)
                         if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
                     tc::tmem_wait_ld();
                     const float *ws = ws_g + qi * p.H_pad + hc;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 2; ++u)
                         if (u < nl) {
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
                                 part[u] = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), part[u]);
                         }
                 }
-                const float score = (part[0] + part[1]) + (part[2] + part[3]);
+                const float score = part[0] + part[1];
                 if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nv_g[qi] ? score : -INFINITY;
             }
             tc::fence_before_sync();
@@ -450,7 +451,7 @@ int launch_index_fp4_tc(const uint8_t *q4, const uint8_t *q4s, const float *w, c
     p.q_bytes = (uint32_t)p.n_cols * row_bytes;
     const size_t smem_cap = 200 * 1024;
     const size_t fixed = ((p.q_bytes + 1023u) & ~1023u) + (size_t)kSfAhead * kTileKeys * p.kb +
-                         2 * ((size_t)NQ * p.H_pad * 4 + NQ * 4) + 1024;
+                         kEpiGroups * ((size_t)NQ * p.H_pad * 4 + NQ * 4) + 1024;
     p.stages = (int)std::min<size_t>(kMaxStages, (smem_cap - fixed) / p.stage_bytes);
     if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
     // tensor memory: accumulators, then the key-scale slots, then the query-head
