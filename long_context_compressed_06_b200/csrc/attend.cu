@@ -27,6 +27,9 @@ __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendA
     const int h = blockIdx.y * (kCombineThreads / tph) + threadIdx.x / tph;
     const int c0 = (threadIdx.x % tph) * 8;
     const bool active = h < a.H;  // no early exit: the RoPE shuffles need whole warps
+    // launched as a programmatic dependent of the attention kernel: its partials
+    // are complete only once that grid is
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const size_t stride = (size_t)a.n_bq * a.H;          // between splits, in rows
     const size_t row = (size_t)bq * a.H + (active ? h : 0);
     float M = -INFINITY;
@@ -89,9 +92,19 @@ size_t ws_bytes_for(long long n_bq, int H, int D, int splits) {
 
 int launch_attend_combine(const AttendArgs &a, cudaStream_t st) {
     const int hpb = kCombineThreads / (a.D / 8);  // heads per block (D in {64, ..., 512})
-    dim3 grid((unsigned)a.n_bq, (unsigned)((a.H + hpb - 1) / hpb));
-    attend_combine_kernel<<<grid, kCombineThreads, 0, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    // a programmatic dependent of the attention kernel just launched on st (which
+    // lets it launch once every attention CTA has started): the combine CTAs are
+    // resident and waiting when the last partial lands
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.n_bq, (unsigned)((a.H + hpb - 1) / hpb));
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_combine_kernel, a) == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
 bool attend_tc_supported(int H, int D);

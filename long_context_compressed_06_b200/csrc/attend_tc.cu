@@ -394,6 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    // the split merge (a programmatic dependent) may launch once every CTA is here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *s.tmem_slot;
     const uint32_t tmem_o = tmem;                  // lanes 0-15 of each sub-partition, columns 0..D-1
     const uint32_t tmem_s = tmem + (16u << 16);    // lanes 16-31, columns 0..127 (two S buffers)

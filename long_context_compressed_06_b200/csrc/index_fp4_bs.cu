@@ -12,9 +12,11 @@
 // The keys stream from HBM as they are stored, 64 code bytes per key at
 // d_I = 128, plus 8 scale bytes.
 //
-// GEMM view per sequence: D[s][(q,h)] = sum_k A[s][k] B[(q,h)][k] with A = the
-// key tile (M = 128 keys, K-major packed rows of d_I/2 bytes), B = the query
-// group's heads (N = NQ x H_pad <= 128 rows), K = d_I in steps of 64.  The
+// GEMM view per sequence: D[s][(q,h)] = sum_k A[s][k] B[(q,h)][k] with A = a
+// 128-key sub-tile (M = 128, K-major packed rows of d_I/2 bytes), B = the query
+// group's heads (N = NQ x H_pad <= 128 rows), K = d_I in steps of 64.  A tile
+// (one TMA box, one ring stage) holds two sub-tiles when their accumulators fit
+// three tiles deep in tensor memory, else one.  The
 // scale factors live in tensor memory, a block of 4 columns per K step (byte j
 // of a 32-bit cell scales 16-element block j of the step): the key scales of
 // each tile in a ring of slots, key row m at lane m, column m / 32 of the
@@ -27,10 +29,9 @@
 // MMA issuer (lane 0 issues through guarded instructions); warps 2..5 -- scale
 // movers (each thread stages its key row's scale bytes with cp.async several
 // tiles ahead and writes them into the tile's tensor-memory slot; the
-// query-head scales once per group); warps 6..21 -- four epilogue groups of
-// four warps taking the tiles in turn (tcgen05.ld, ReLU, weighted head sum,
-// causal mask, store): at 9 KiB per tile the tiles arrive every ~0.2 us per
-// SM at HBM speed, faster than one group's per-tile latency.  Every wait is
+// query-head scales once per group); warps 6..21 -- up to four epilogue
+// groups of four warps, one per accumulator, taking the tiles in turn
+// (tcgen05.ld, ReLU, weighted head sum, causal mask, store).  Every wait is
 // bounded and every role warp stays converged.
 #include <algorithm>
 #include <cstring>
@@ -44,11 +45,11 @@ namespace {
 
 constexpr int kEpiGroups = 4;  // epilogue groups of four warps, taking tiles in turn
 constexpr int kThreads = 192 + 128 * kEpiGroups;
-constexpr int kTileKeys = 128;
+constexpr int kSubKeys = 128;   // keys of one MMA (M); a tile holds p.sub of them
 constexpr int kMaxStages = 20;
 constexpr int kMaxAcc = 4;
-constexpr int kSfSlots = 8;     // key-scale slots in tensor memory (tiles in flight)
-constexpr int kSfAhead = 4;     // tiles whose key scales a mover thread prefetches
+constexpr int kSfSlots = 4;     // key-scale slots in tensor memory (tiles in flight)
+constexpr int kSfAhead = 8;     // tiles whose key scales a mover thread prefetches
 
 struct Fp4BsParams {
     const uint8_t *k4s;   // [batch][N][d_I/16] key scales (e4m3, non-negative)
@@ -61,6 +62,8 @@ struct Fp4BsParams {
     int groups_per_batch, n_ktiles;
     long long total_work;
     int stages, kb, nks;  // ring depth, scale bytes per row (d_I/16), MMA K steps (d_I/64)
+    int sub, tile_keys;   // M = 128 sub-tiles per tile (1 or 2) and keys per tile
+    uint32_t sub_desc;    // start-address step of the second sub-tile in a smem descriptor
     uint32_t stage_bytes, q_bytes, idesc, sbo, layout;
     int n_cols, n_acc;
     uint32_t tmem_cols, sfa_col, sfb_col;
@@ -146,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *k_smem = base;
     uint8_t *q_smem = k_smem + (size_t)p.stages * p.stage_bytes;
-    uint8_t *sf_smem = q_smem + ((p.q_bytes + 1023u) & ~1023u);            // [kSfAhead][128 rows][KB]
-    float *w_s = reinterpret_cast<float *>(sf_smem + kSfAhead * kTileKeys * KB);  // [groups][NQ][H_pad]
+    uint8_t *sf_smem = q_smem + ((p.q_bytes + 1023u) & ~1023u);            // [kSfAhead][tile rows][KB]
+    float *w_s = reinterpret_cast<float *>(sf_smem + kSfAhead * p.tile_keys * KB);  // [groups][NQ][H_pad]
     int *nvis_s = reinterpret_cast<int *>(w_s + kEpiGroups * p.NQ * p.H_pad);     // [groups][NQ]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(nvis_s + kEpiGroups * p.NQ) + 7) & ~uintptr_t(7));
@@ -156,7 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *sfull = tempty + kMaxAcc, *sempty = sfull + kSfSlots;       // key-scale slots
     uint64_t *qfull = sempty + kSfSlots, *qempty = qfull + 1;             // query codes (TMA)
     uint64_t *qsfull = qempty + 1, *qsempty = qsfull + 1;                 // query-head scales
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qsempty + 1);
+    uint64_t *sfld = qsempty + 1;                                         // key-scale staging slots
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfld + kSfAhead);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(qempty, 1);
         mbar_init(qsfull, 4);
         mbar_init(qsempty, 1);
+        for (int s = 0; s < kSfAhead; ++s) mbar_init(sfld + s, 128);  // one cp.async arrival per mover thread
         *abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&kmap);
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_all(empty + st, kr.phase ^ 1u)) break;
             mbar_arrive_expect_tx(smem_u32(full + st), p.stage_bytes, lane == 0);
             tc::tma_load_3d(smem_u32(k_smem + (size_t)st * p.stage_bytes), &kmap, smem_u32(full + st), 0,
-                            cu.kt * kTileKeys, cu.b, lane == 0);
+                            cu.kt * p.tile_keys, cu.b, lane == 0);
             kr.next(p.stages);
             ++it;
         }
@@ -241,14 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int sl = sr.idx;
             if (!wait_all(sfull + sl, sr.phase)) break;
             tc::fence_after_sync();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols);
             const uint64_t kd = kdesc0 + ((uint64_t)(st * p.stage_bytes) >> 4);
-            for (int ks = 0; ks < NKS; ++ks)
-                // K step ks: 64 codes = 32 bytes into each swizzled row; its scale
-                // factors in the 4-column blocks of the tile's slot and of the group
-                mma_fp4(d_tmem, kd + (uint64_t)(ks * 2), qdesc0 + (uint64_t)(ks * 2), p.idesc,
-                        tmem_base + p.sfa_col + (uint32_t)(4 * (sl * NKS + ks)), tmem_base + p.sfb_col + (uint32_t)(4 * ks),
-                        ks > 0 ? 1u : 0u, issuer);
+            for (int h = 0; h < p.sub; ++h) {
+                // sub-tile h: keys 128h.. of the tile into its own accumulator
+                const uint32_t d_tmem = tmem_base + (uint32_t)((acc * p.sub + h) * p.n_cols);
+                for (int ks = 0; ks < NKS; ++ks)
+                    // K step ks: 64 codes = 32 bytes into each swizzled row; its scale
+                    // factors in the 4-column blocks of the sub-tile's slot and of the group
+                    mma_fp4(d_tmem, kd + (uint64_t)(h * p.sub_desc + ks * 2), qdesc0 + (uint64_t)(ks * 2), p.idesc,
+                            tmem_base + p.sfa_col + (uint32_t)(4 * ((sl * p.sub + h) * NKS + ks)),
+                            tmem_base + p.sfb_col + (uint32_t)(4 * ks), ks > 0 ? 1u : 0u, issuer);
+            }
             tc::mma_commit(smem_u32(empty + st), issuer);
             tc::mma_commit(smem_u32(sempty + sl), issuer);
             tc::mma_commit(smem_u32(tfull + acc), issuer);
@@ -262,21 +270,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ scale movers (warps 2..5)
-        // Thread r (0..127) owns tile row r: the key of that row in every tile, and
-        // query-head row r of every group.  Its key-scale bytes are staged with
-        // cp.async kSfAhead tiles ahead (one commit group per tile).
+        // Thread r (0..127) owns row r of every sub-tile (the keys r and 128 + r of
+        // a two-sub-tile tile) and query-head row r of every group.  Its key-scale bytes are staged with
+        // cp.async kSfAhead tiles ahead, each staging slot completed by an mbarrier
+        // that counts the movers' cp.async arrivals: issued only a few tiles ahead,
+        // these small loads wait behind the deep ring of key-tile copies in the
+        // memory queues and set the pace.  A thread reads and refills only its own
+        // row of a slot, so a slot needs no barrier between the movers.
         const int sub = warp & 3;  // tensor-memory lanes this warp may access
         const int r = sub * 32 + lane;
         const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
         const uint32_t stage_row = smem_u32(sf_smem + r * KB);
         const auto prefetch = [&](const Cursor &c, long long i) {
             if (c.w < w1) {
-                const long long key = (long long)c.kt * kTileKeys + r;
-                const bool valid = key < p.N;
-                cp_async_row<KB>(stage_row + (uint32_t)((i % kSfAhead) * kTileKeys * KB),
-                                 p.k4s + ((size_t)c.b * p.N + (valid ? key : 0)) * KB, valid);
+                for (int h = 0; h < p.sub; ++h) {
+                    const long long key = (long long)c.kt * p.tile_keys + h * kSubKeys + r;
+                    const bool valid = key < p.N;
+                    cp_async_row<KB>(stage_row + (uint32_t)(((i % kSfAhead) * p.tile_keys + h * kSubKeys) * KB),
+                                     p.k4s + ((size_t)c.b * p.N + (valid ? key : 0)) * KB, valid);
+                }
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                             ::"r"(smem_u32(sfld + (int)(i % kSfAhead))) : "memory");
             }
-            asm volatile("cp.async.commit_group;" ::: "memory");
         };
         Cursor pf = cursor_at(p, w0);
         for (int i = 0; i < kSfAhead; ++i) {
@@ -317,18 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++gi;
             }
             // this tile's key scales: staged kSfAhead tiles ago
-            asm volatile("cp.async.wait_group %0;" ::"n"(kSfAhead - 1) : "memory");
-            uint32_t v[NKS];
-            const uint8_t *row = sf_smem + (size_t)(i % kSfAhead) * kTileKeys * KB + r * KB;
-#pragma unroll
-            for (int j = 0; j < NKS; ++j) v[j] = reinterpret_cast<const uint32_t *>(row)[j];
+            if (!wait_all(sfld + (int)(i % kSfAhead), (uint32_t)((i / kSfAhead) & 1))) break;
             const int sl = sr.idx;
             if (!wait_all(sempty + sl, sr.phase ^ 1u)) break;
             tc::fence_after_sync();
-            // key row r at lane r, column r / 32 = sub of each K step's block
+            for (int h = 0; h < p.sub; ++h) {
+                uint32_t v[NKS];
+                const uint8_t *row = sf_smem + ((size_t)(i % kSfAhead) * p.tile_keys + h * kSubKeys + r) * KB;
 #pragma unroll
-            for (int j = 0; j < NKS; ++j)
-                tmem_st1(tmem_base + lane_off + p.sfa_col + (uint32_t)(4 * (sl * NKS + j) + sub), v[j]);
+                for (int j = 0; j < NKS; ++j) v[j] = reinterpret_cast<const uint32_t *>(row)[j];
+                // key row r of sub-tile h at lane r, column r / 32 = sub of each K step's block
+#pragma unroll
+                for (int j = 0; j < NKS; ++j)
+                    tmem_st1(tmem_base + lane_off + p.sfa_col + (uint32_t)(4 * ((sl * p.sub + h) * NKS + j) + sub), v[j]);
+            }
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
@@ -342,8 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ------------------------------------------------------------ epilogue (warps 6..21)
-        // kEpiGroups groups of four warps take the tiles in turn (tile i -> group
-        // i % kEpiGroups, accumulator i % n_acc).
+        // Groups of four warps, one per accumulator (n_acc <= kEpiGroups; the rest
+        // idle): tile i -> accumulator and group i % n_acc.  Each accumulator's
+        // tiles then reach one group in order, so a group never waits on a
+        // tfull phase parity two phases ahead of the one it means.
         const int eg = (warp - 6) >> 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
@@ -353,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int loaded_b = -1, loaded_g = -1;
         for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
             const int li = (int)(cu.w - w0);
-            if (li % kEpiGroups != eg) continue;
+            if (li % p.n_acc != eg) continue;
             const int b = cu.b, g = cu.g;
             if (b != loaded_b || g != loaded_g) {
                 group_bar(eg);
@@ -375,32 +394,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(tfull + acc), aph, p.ctx, abort_flag));
             if (!ok) break;
             tc::fence_after_sync();
-            const long long s = (long long)cu.kt * kTileKeys + row;
-            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.n_cols);
-            for (int qi = 0; qi < p.NQ; ++qi) {
-                const int q = g * p.NQ + qi;
-                if (q >= p.nq) break;
-                // 32 columns per TMEM load round (two 16-column loads in flight), two
-                // partial sums per round keep the FMA chains short
-                float part[2] = {0.f, 0.f};
-                for (int hc = 0; hc < p.H_pad; hc += 32) {
-                    float v[32];
-                    const int nl = min(2, (p.H_pad - hc) >> 4);
+            for (int h = 0; h < p.sub; ++h) {
+                const long long s = (long long)cu.kt * p.tile_keys + h * kSubKeys + row;
+                const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * p.sub + h) * p.n_cols);
+                for (int qi = 0; qi < p.NQ; ++qi) {
+                    const int q = g * p.NQ + qi;
+                    if (q >= p.nq) break;
+                    // 32 columns per TMEM load round (two 16-column loads in flight), two
+                    // partial sums per round keep the FMA chains short
+                    float part[2] = {0.f, 0.f};
+                    for (int hc = 0; hc < p.H_pad; hc += 32) {
+                        float v[32];
+                        const int nl = min(2, (p.H_pad - hc) >> 4);
 #pragma unroll
-                    for (int u = 0; u < 2; ++u)
-                        if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
-                    tc::tmem_wait_ld();
-                    const float *ws = ws_g + qi * p.H_pad + hc;
+                        for (int u = 0; u < 2; ++u)
+                            if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
+                        tc::tmem_wait_ld();
+                        const float *ws = ws_g + qi * p.H_pad + hc;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u)
-                        if (u < nl) {
+                        for (int u = 0; u < 2; ++u)
+                            if (u < nl) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                part[u] = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), part[u]);
-                        }
+                                for (int i = 0; i < 16; ++i)
+                                    part[u] = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), part[u]);
+                            }
+                    }
+                    const float score = part[0] + part[1];
+                    if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nv_g[qi] ? score : -INFINITY;
                 }
-                const float score = part[0] + part[1];
-                if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nv_g[qi] ? score : -INFINITY;
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -443,28 +464,36 @@ int launch_index_fp4_tc(const uint8_t *q4, const uint8_t *q4s, const float *w, c
                                                    : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                                       : CU_TENSOR_MAP_SWIZZLE_32B);
     p.sbo = 8u * row_bytes;
-    p.stage_bytes = (uint32_t)kTileKeys * row_bytes;
     // queries per tile: as many as fit in N <= 128 rows
     const int NQ = std::max(1, std::min(nq, 128 / p.H_pad));
     p.NQ = NQ;
     p.n_cols = NQ * p.H_pad;
     p.q_bytes = (uint32_t)p.n_cols * row_bytes;
+    // Tensor memory: accumulators, then the key-scale slots, then the query-head
+    // scales (a 4-column block per K step).  A tile is two M = 128 sub-tiles
+    // (256 keys) when three tiles' accumulators still fit: the MMA warp's fixed
+    // cost per tile (barrier waits, commits) is then spread over twice the keys.
+    int sf_cols = 0;
+    for (p.sub = 2;; p.sub = 1) {
+        sf_cols = (kSfSlots * p.sub + 1) * 4 * p.nks;
+        p.n_acc = std::min(kMaxAcc, (512 - sf_cols) / (p.n_cols * p.sub));
+        if (p.n_acc >= 3 || p.sub == 1) break;
+    }
+    if (p.n_acc < 2) return CSA_ERR_UNSUPPORTED;
+    p.tile_keys = kSubKeys * p.sub;
+    p.sub_desc = (uint32_t)(kSubKeys * row_bytes) >> 4;
+    p.stage_bytes = (uint32_t)p.tile_keys * row_bytes;
     const size_t smem_cap = 200 * 1024;
-    const size_t fixed = ((p.q_bytes + 1023u) & ~1023u) + (size_t)kSfAhead * kTileKeys * p.kb +
+    const size_t fixed = ((p.q_bytes + 1023u) & ~1023u) + (size_t)kSfAhead * p.tile_keys * p.kb +
                          kEpiGroups * ((size_t)NQ * p.H_pad * 4 + NQ * 4) + 1024;
     p.stages = (int)std::min<size_t>(kMaxStages, (smem_cap - fixed) / p.stage_bytes);
     if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
-    // tensor memory: accumulators, then the key-scale slots, then the query-head
-    // scales (a 4-column block per K step)
-    const int sf_cols = (kSfSlots + 1) * 4 * p.nks;
-    p.n_acc = std::min(kMaxAcc, (512 - sf_cols) / p.n_cols);
-    if (p.n_acc < 2) return CSA_ERR_UNSUPPORTED;
-    p.sfa_col = (uint32_t)(p.n_acc * p.n_cols);
-    p.sfb_col = p.sfa_col + (uint32_t)(kSfSlots * 4 * p.nks);
+    p.sfa_col = (uint32_t)(p.n_acc * p.sub * p.n_cols);
+    p.sfb_col = p.sfa_col + (uint32_t)(kSfSlots * p.sub * 4 * p.nks);
     p.tmem_cols = 512;
-    p.idesc = idesc_mxf4nvf4(128, p.n_cols);
+    p.idesc = idesc_mxf4nvf4(kSubKeys, p.n_cols);
     p.groups_per_batch = (nq + NQ - 1) / NQ;
-    p.n_ktiles = (int)((N + kTileKeys - 1) / kTileKeys);
+    p.n_ktiles = (int)((N + p.tile_keys - 1) / p.tile_keys);
     p.total_work = (long long)batch * p.groups_per_batch * p.n_ktiles;
 
     CUtensorMap kmap, qmap;
@@ -473,7 +502,7 @@ int launch_index_fp4_tc(const uint8_t *q4, const uint8_t *q4s, const float *w, c
     {
         const uint64_t dims[3] = {row_bytes, (uint64_t)N, (uint64_t)batch};
         const uint64_t strides[2] = {row_bytes, (uint64_t)N * row_bytes};
-        const uint32_t box[3] = {row_bytes, (uint32_t)kTileKeys, 1};
+        const uint32_t box[3] = {row_bytes, (uint32_t)p.tile_keys, 1};
         if (!encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k4, dims, strides, box, sw))
             return CSA_ERR_CUDA;
     }
@@ -485,7 +514,7 @@ int launch_index_fp4_tc(const uint8_t *q4, const uint8_t *q4s, const float *w, c
             return CSA_ERR_CUDA;
     }
     const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + fixed +
-                        (2 * kMaxStages + 2 * kMaxAcc + 2 * kSfSlots + 4) * 8 + 16;
+                        (2 * kMaxStages + 2 * kMaxAcc + 2 * kSfSlots + 4 + kSfAhead) * 8 + 16;
     void (*kern)(const CUtensorMap, const CUtensorMap, const Fp4BsParams) =
         p.kb == 16 ? index_fp4_bs_kernel<16> : (p.kb == 8 ? index_fp4_bs_kernel<8> : index_fp4_bs_kernel<4>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -5,18 +5,26 @@
 // -> top-k selector; techniques map: indices at or beyond the causal threshold
 // become -1).  Output indices are in ascending order.
 //
-// Design: a radix select over the scores mapped to order-preserving uint32
-// keys.  One query is handled by one CTA of 1024 threads or, for long rows and
-// for small batches, by a thread-block cluster of CS CTAs; each thread keeps R
-// consecutive keys in registers (CS*1024*R >= N),
-// so the scores are read from memory exactly once.  The digits start at the
-// highest bit where the cluster-wide smallest and largest key differ (the bits
-// above are shared by every candidate), 11 bits per pass; each CTA counts its
-// candidates into its own shared-memory histogram and, after one cluster
-// barrier, reads its peers' histograms through distributed shared memory.
-// The selection stops once the threshold bin holds exactly the number of
-// elements still needed.  Selection is a stable compaction: per-thread
-// counts, a block scan, and a cluster scan over CTA totals via DSMEM.
+// Design: one query is handled by one CTA of 1024 threads or, for long rows
+// and for small batches, by a thread-block cluster of CS CTAs; each thread
+// keeps R consecutive scores (CS*1024*R >= N) in registers as order-preserving
+// uint32 keys, so the scores are read from memory once.
+//
+// First pass: a histogram over 1024 bins linear in the score between the
+// smallest and largest visible score (pushed by every CTA into every other's
+// shared memory before one cluster barrier).  The threshold bin -- the bin that
+// holds the k-th largest score -- then has few keys: every key above it is
+// selected, and the keys inside it (at most 256) are pushed, with the per-CTA
+// counts, into every CTA's shared memory, where each CTA ranks them directly
+// (score descending, index ascending) and writes its own selected indices in
+// index order.  After that barrier no CTA touches another's memory.
+//
+// Fallback (a non-finite score range, or a threshold bin above 256 keys): a
+// radix select on the key bits, from the highest bit where the smallest and
+// largest key differ, 11 bits per pass, with per-CTA shared-memory histograms
+// read by the peers through distributed shared memory after a cluster barrier;
+// it stops once the threshold bin holds exactly the number still needed, and
+// compacts stably (block scan plus a cluster scan over the CTA totals).
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -28,13 +36,21 @@ namespace csa {
 namespace {
 
 constexpr int kTopkThreads = 1024;
-constexpr int kBins = 2048;
+constexpr int kBins = 2048;      // bins of a radix pass over the key bits (two per thread)
+constexpr int kLinBins = 1024;   // bins of the value-linear pass (one per thread)
+constexpr int kCandCap = 256;    // threshold-bin keys ranked directly (larger bins: radix passes)
+constexpr int kMaxCluster = 16;  // CTAs per query at most
 
 // order-preserving map fp32 -> uint32 (-0 folded onto +0)
 CSA_DEVINL uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// its inverse (the score of a key, -0 read back as +0)
+CSA_DEVINL float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 // Inclusive scan over the 1024 threads of the block; returns this thread's
@@ -66,9 +82,19 @@ CSA_DEVINL T block_scan_incl(T v, T *warp_buf, T *total) {
     return v;
 }
 
-// CL: the query's row is split over a cluster of CS CTAs (histograms and CTA
-// totals merged through distributed shared memory, cluster barriers); without
-// it one CTA holds the row and every barrier is a block barrier.
+// Value-linear digit of a key: floor((v - vmin) * scale), capped at the last bin.
+// Rounded subtraction and multiplication by a positive constant preserve order,
+// so the digit is non-decreasing in the key; the explicit roundings keep it the
+// same function of the key in every thread.
+CSA_DEVINL int lin_digit(uint32_t key, float vmin, float scale) {
+    const float x = __fmul_rn(__fsub_rn(key_value(key), vmin), scale);
+    return __float2int_rz(fminf(x, (float)(kLinBins - 1)));
+}
+
+// CL: the query's row is split over a cluster of CS CTAs (ranges, candidates
+// and counts pushed into every rank's shared memory, histograms read through
+// distributed shared memory, cluster barriers); without it one CTA holds the
+// row and every barrier is a block barrier.
 template <int R, bool CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__restrict__ scores,
                                                                const int *__restrict__ q_pos, long long N,
@@ -87,10 +113,16 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     __shared__ __align__(8) uint32_t hist[2][kBins];  // this CTA's histogram, double-buffered over passes
     __shared__ uint32_t warp_u32[32];
     __shared__ unsigned long long warp_u64[32];
-    __shared__ unsigned long long cta_total;           // (gt << 32) | eq, read by higher ranks
-    __shared__ uint32_t cta_min, cta_max;               // this CTA's key range, read by peers
-    __shared__ uint32_t s_min, s_max, s_bin, s_cnt;
-    __shared__ long long s_krem;
+    __shared__ unsigned long long cta_total;           // radix passes: (gt << 32) | eq, read by higher ranks
+    __shared__ uint32_t r_min[kMaxCluster], r_max[kMaxCluster];  // every rank's key range (pushed by that rank)
+    __shared__ unsigned long long r_tot[kMaxCluster];  // every rank's (above << 32) | in-bin counts (pushed)
+    __shared__ uint32_t seg_key[kMaxCluster][kCandCap];  // every rank's threshold-bin keys in index order (pushed)
+    __shared__ uint32_t all_key[kCandCap];              // the segments concatenated (index order)
+    __shared__ uint32_t rank_part[kTopkThreads / kCandCap][kCandCap];
+    __shared__ uint32_t sel_pre[kCandCap + 1];          // selected among the first x candidates
+    __shared__ uint32_t s_off[kMaxCluster + 1];         // list offset of each rank, then the total
+    __shared__ uint32_t s_bin, s_cnt;
+    __shared__ long long s_krem, s_above_before;
 
     // as a programmatic dependent: the scores are complete only once the
     // predecessor grid is (a no-op otherwise); the successor may launch now
@@ -98,14 +130,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = threadIdx.x; i < 2 * kBins; i += kTopkThreads) (&hist[0][0])[i] = 0u;
 
-    const long long nv = q_pos ? n_visible(q_pos[bq], m, N) : N;  // no q_pos: every entry is eligible
-    const long long kk = nv < k ? nv : k;
+    // the score loads do not wait for the query position (they stay inside the
+    // row); entries past n_vis are masked afterwards
+    const int t_q = q_pos ? __ldg(q_pos + bq) : 0;
     const long long seg0 = ((long long)rank * kTopkThreads + threadIdx.x) * R;
-    const int nloc = (int)(nv - seg0 <= 0 ? 0 : (nv - seg0 >= R ? R : nv - seg0));
-
+    const int nrow = (int)(N - seg0 <= 0 ? 0 : (N - seg0 >= R ? R : N - seg0));
     uint32_t key[R];
     const float *row = scores + bq * N;
-    if (nloc == R && (N & 3) == 0) {
+    if (nrow == R && (N & 3) == 0) {
 #pragma unroll
         for (int r = 0; r < R; r += 4) {
             const float4 v = __ldg(reinterpret_cast<const float4 *>(row + seg0 + r));
@@ -114,9 +146,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         }
     } else {
 #pragma unroll
-        for (int r = 0; r < R; ++r) key[r] = r < nloc ? order_key(__ldg(row + seg0 + r)) : 0u;
+        for (int r = 0; r < R; ++r) key[r] = r < nrow ? order_key(__ldg(row + seg0 + r)) : 0u;
     }
-    // key range of the visible entries (cluster-wide)
+    const long long nv = q_pos ? n_visible(t_q, m, N) : N;  // no q_pos: every entry is eligible
+    const long long kk = nv < k ? nv : k;
+    const int nloc = (int)(nv - seg0 <= 0 ? 0 : (nv - seg0 >= R ? R : nv - seg0));
+
+    // key range of the visible entries, pushed into every rank
     uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -134,45 +170,227 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     if (warp == 0) {
         const uint32_t a = __reduce_min_sync(0xffffffffu, warp_u32[lane]);
         const uint32_t b = __reduce_max_sync(0xffffffffu, reinterpret_cast<uint32_t *>(warp_u64)[lane]);
-        if (lane == 0) {
-            cta_min = a;
-            cta_max = b;
+        if (lane < CS) {
+            *peer(&r_min[rank], lane) = a;
+            *peer(&r_max[rank], lane) = b;
         }
     }
-    sync_all();  // key ranges published, histograms cleared
-    if (warp == 0) {
-        const uint32_t a = lane < CS ? *peer(&cta_min, lane) : 0xffffffffu;
-        const uint32_t b = lane < CS ? *peer(&cta_max, lane) : 0u;
-        const uint32_t ga = __reduce_min_sync(0xffffffffu, a), gb = __reduce_max_sync(0xffffffffu, b);
-        if (lane == 0) {
-            s_min = ga;
-            s_max = gb;
-            s_bin = 0u;
-            s_cnt = 0u;
-            s_krem = 0;
-        }
+    sync_all();  // every rank's range delivered, histograms cleared
+    uint32_t gmin = 0xffffffffu, gmax = 0u;
+    for (int r2 = 0; r2 < CS; ++r2) {
+        gmin = min(gmin, r_min[r2]);
+        gmax = max(gmax, r_max[r2]);
     }
-    __syncthreads();
 
-    // Radix select from the highest bit where the smallest and largest key
-    // differ (bits above it are shared by every candidate), 11 bits per pass.
+    // Threshold bin of the cluster-wide 2048-bin histogram in hloc (every rank's
+    // copy): the highest bin b with (count above b) < krem_in <= (count above b)
+    // + count(b), into s_bin, s_cnt and s_krem (what is still needed from b).
+    const auto find_bin = [&](const uint32_t *hloc, long long krem_in) {
+        uint32_t c_lo = 0u, c_hi = 0u;
+        for (int r0 = 0; r0 < CS; r0 += 4) {
+            uint2 v[4];  // this thread's two bins of up to four ranks, loads issued together
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                v[j] = r0 + j < CS ? *reinterpret_cast<const uint2 *>(peer(hloc, r0 + j) + 2 * threadIdx.x)
+                                   : make_uint2(0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                c_lo += v[j].x;
+                c_hi += v[j].y;
+            }
+        }
+        uint32_t tot;
+        const uint32_t incl = block_scan_incl<uint32_t>(c_lo + c_hi, warp_u32, &tot);
+        const long long above = (long long)tot - incl;  // count in bins of higher threads
+        if (above < krem_in && above + c_hi >= krem_in) {
+            s_bin = 2 * threadIdx.x + 1; s_cnt = c_hi; s_krem = krem_in - above;
+        } else if (above + c_hi < krem_in && above + c_hi + c_lo >= krem_in) {
+            s_bin = 2 * threadIdx.x; s_cnt = c_lo; s_krem = krem_in - above - c_hi;
+        }
+        __syncthreads();
+    };
+
     uint32_t prefix = 0u, mask = 0u;
     long long krem = kk;
     bool done = nv <= k;  // every visible entry is selected
     int top = -1;
+    bool lin = false;     // value-linear first pass possible (finite, distinct range)
+    float vmin = 0.f, lscale = 0.f;
     if (!done) {
-        if (s_min == s_max) {
-            prefix = s_max;
+        if (gmin == gmax) {
+            prefix = gmax;
             mask = 0xffffffffu;  // all keys equal: the lowest indices win
             done = true;
         } else {
-            top = 31 - __clz(s_min ^ s_max);
+            top = 31 - __clz(gmin ^ gmax);
             mask = top == 31 ? 0u : ~((2u << top) - 1u);
-            prefix = s_max & mask;
+            prefix = gmax & mask;
+            vmin = key_value(gmin);
+            const float vmax = key_value(gmax);
+            const float range = __fsub_rn(vmax, vmin);
+            lscale = __fdiv_rn((float)kLinBins, range);
+            lin = isfinite(vmin) && isfinite(vmax) && isfinite(range) && range > 0.f && isfinite(lscale);
         }
     }
+    // Pass 1: bins linear in the score between the smallest and largest visible
+    // score.  Scores bunch in a few binary exponents, so bins taken from the key
+    // bits would pile most keys into a handful of bins (shared-memory atomics on
+    // one address serialise); linear bins spread them, and the threshold bin
+    // holds few keys.  Those candidates are ranked directly below.
+    int p0 = 0;
+    int t1 = 0;
+    // the value-linear digits, two per register, kept when the registers allow
+    // (1024 threads have 64 each); otherwise recomputed from the keys
+    constexpr bool kKeepDigits = R <= 8;
+    uint32_t dg[kKeepDigits ? R / 2 : 1];
+    const auto digit = [&](int r) -> int {
+        if constexpr (kKeepDigits) return (int)((dg[r / 2] >> (16 * (r & 1))) & 0xffffu);
+        else return lin_digit(key[r], vmin, lscale);
+    };
+    if (lin) {
+        if constexpr (kKeepDigits) {
+#pragma unroll
+            for (int r = 0; r < R; r += 2) {
+                const uint32_t d0 = (uint32_t)lin_digit(key[r], vmin, lscale);
+                const uint32_t d1 = (uint32_t)lin_digit(key[r + 1], vmin, lscale);
+                dg[r / 2] = d0 | (d1 << 16);
+                if (r < nloc) atomicAdd(&hist[0][d0], 1u);
+                if (r + 1 < nloc) atomicAdd(&hist[0][d1], 1u);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (r < nloc) atomicAdd(&hist[0][lin_digit(key[r], vmin, lscale)], 1u);
+        }
+        sync_all();  // every CTA's histogram is complete
+        // cluster-wide count of bin threadIdx.x (one bin per thread)
+        uint32_t c = 0u;
+        for (int r0 = 0; r0 < CS; r0 += 4) {
+            uint32_t v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = r0 + j < CS ? *peer(&hist[0][threadIdx.x], r0 + j) : 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c += v[j];
+        }
+        uint32_t tot;
+        const uint32_t incl = block_scan_incl<uint32_t>(c, warp_u32, &tot);
+        const long long above = (long long)tot - incl;
+        if (above < krem && above + c >= krem) {
+            s_bin = threadIdx.x;
+            s_cnt = c;
+            s_krem = krem - above;
+        }
+        __syncthreads();
+        p0 = 1;  // a radix pass after this one starts on the other buffer
+        lin = s_cnt <= (uint32_t)kCandCap;  // the same cluster-wide count in every CTA
+        if (lin) {
+            t1 = (int)s_bin;
+            krem = s_krem;
+        }
+    }
+
+    int *out = idx + bq * k;
+    if (lin) {
+        // ------------------------------------------------ threshold bin ranked directly
+        uint32_t n_above = 0u, n_in = 0u;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if (r < nloc) {
+                const int d = digit(r);
+                n_above += d > t1;
+                n_in += d == t1;
+            }
+        unsigned long long blk_tot;
+        const unsigned long long mine = ((unsigned long long)n_above << 32) | n_in;
+        const unsigned long long excl = block_scan_incl<unsigned long long>(mine, warp_u64, &blk_tot) - mine;
+        // this CTA's candidates into its segment of every rank's list, in index order
+        uint32_t cp = (uint32_t)excl;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if (r < nloc && digit(r) == t1) {
+                for (int r2 = 0; r2 < CS; ++r2) *peer(&seg_key[rank][cp], r2) = key[r];
+                ++cp;
+            }
+        if ((int)threadIdx.x < CS) *peer(&r_tot[rank], (int)threadIdx.x) = blk_tot;
+        // every rank's candidates and counts delivered; from here on no CTA
+        // touches another's shared memory, so none waits for the others to exit
+        sync_all();
+        if (warp == 0) {
+            // prefix over ranks of the (above, in-bin) counts: list offsets, and the
+            // keys above the bin in lower ranks (this rank's first output slot)
+            const unsigned long long t = lane < CS ? r_tot[lane] : 0ull;
+            unsigned long long inc = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long n = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += n;
+            }
+            if (lane < CS) s_off[lane] = (uint32_t)(inc - t);
+            if (lane == CS - 1) s_off[CS] = (uint32_t)inc;
+            if (lane == rank) s_above_before = (long long)((inc - t) >> 32);
+        }
+        __syncthreads();
+        const int C = (int)s_off[CS];
+        for (int i = threadIdx.x; i < C; i += kTopkThreads) {
+            int r2 = 0;
+            while (r2 + 1 < CS && s_off[r2 + 1] <= (uint32_t)i) ++r2;
+            all_key[i] = seg_key[r2][i - (int)s_off[r2]];
+        }
+        __syncthreads();
+        {
+            // candidates preceding candidate i in (score desc, index asc), counted
+            // over four slices of the list by four threads
+            constexpr int kParts = kTopkThreads / kCandCap;
+            const int i = threadIdx.x % kCandCap, part = threadIdx.x / kCandCap;
+            if (i < C) {
+                const int chunk = (C + kParts - 1) / kParts;
+                const int j0 = part * chunk, j1 = min(C, j0 + chunk);
+                const uint32_t ki = all_key[i];
+                uint32_t cnt = 0u;
+                for (int j = j0; j < j1; ++j) {
+                    const uint32_t kj = all_key[j];
+                    cnt += (kj > ki) || (kj == ki && j < i);
+                }
+                rank_part[part][i] = cnt;
+            }
+        }
+        __syncthreads();
+        uint32_t sel = 0u;
+        if ((int)threadIdx.x < C) {
+            uint32_t rk = 0u;
+#pragma unroll
+            for (int q = 0; q < kTopkThreads / kCandCap; ++q) rk += rank_part[q][threadIdx.x];
+            sel = (long long)rk < krem;
+        }
+        uint32_t sel_tot;
+        const uint32_t sel_incl = block_scan_incl<uint32_t>(sel, warp_u32, &sel_tot);
+        if ((int)threadIdx.x < C) sel_pre[threadIdx.x + 1] = sel_incl;
+        if (threadIdx.x == 0) sel_pre[0] = 0u;
+        __syncthreads();
+        // outputs in index order: keys above the threshold bin and selected candidates
+        uint32_t ci = s_off[rank] + (uint32_t)excl;
+        long long pos = s_above_before + (long long)(excl >> 32) + sel_pre[ci];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if (r < nloc) {
+                const int d = digit(r);
+                // pos < kk by construction (kk - krem keys above the bin, krem selected in it)
+                if (d > t1 || (d == t1 && sel_pre[ci + 1] != sel_pre[ci])) {
+                    if (pos < kk) out[pos] = (int)(seg0 + r);
+                    ++pos;
+                }
+                ci += d == t1;
+            }
+        if (rank == 0)
+            for (long long i = kk + threadIdx.x; i < k; i += kTopkThreads) out[i] = -1;
+        return;
+    }
+
+    // ---------------------------------------------------- radix select on the key bits
+    // From the highest bit where the smallest and largest key differ (bits above
+    // it are shared by every candidate), 11 bits per pass.
 #pragma unroll 1
-    for (int p = 0; !done && top >= 0; ++p) {
+    for (int p = p0; !done && top >= 0; ++p) {
         const int width = top + 1 < 11 ? top + 1 : 11;
         const int sh = top - width + 1;
         const uint32_t dmask = (1u << width) - 1u;
@@ -181,25 +399,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         for (int r = 0; r < R; ++r)
             if (r < nloc && (key[r] & mask) == prefix) atomicAdd(hloc + ((key[r] >> sh) & dmask), 1u);
         sync_all();  // every CTA's histogram of this pass is complete
-        // cluster-wide counts of this thread's two bins: read every rank's histogram
-        uint32_t c_lo = 0u, c_hi = 0u;
-        for (int r2 = 0; r2 < CS; ++r2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(peer(hloc, r2) + 2 * threadIdx.x);
-            c_lo += v.x;
-            c_hi += v.y;
-        }
+        find_bin(hloc, krem);
         hist[(p + 1) & 1][2 * threadIdx.x] = 0u;      // peers finished reading it in the previous pass
         hist[(p + 1) & 1][2 * threadIdx.x + 1] = 0u;
-        // threshold bin: the highest bin b with (count above b) < krem <= (count above b) + hist[b]
-        uint32_t tot;
-        const uint32_t incl = block_scan_incl<uint32_t>(c_lo + c_hi, warp_u32, &tot);
-        const long long above = (long long)tot - incl;  // count in bins of higher threads
-        if (above < krem && above + c_hi >= krem) {
-            s_bin = 2 * threadIdx.x + 1; s_cnt = c_hi; s_krem = krem - above;
-        } else if (above + c_hi < krem && above + c_hi + c_lo >= krem) {
-            s_bin = 2 * threadIdx.x; s_cnt = c_lo; s_krem = krem - above - c_hi;
-        }
-        __syncthreads();
         prefix |= s_bin << sh;
         mask |= dmask << sh;
         krem = s_krem;
@@ -229,7 +431,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     }
     long long gt_before = (long long)((base + excl) >> 32);
     long long eq_before = (long long)((base + excl) & 0xffffffffull);
-    int *out = idx + bq * k;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         if (r < nloc) {
@@ -279,7 +480,7 @@ int launch_topk(const float *scores, const int *q_pos, int batch, int nq, long l
     const long long nqry = (long long)batch * nq;
     if (nqry == 0) return CSA_OK;
     const TopkPlan pl = plan(nqry, N);
-    if (pl.CS > 16 || pl.R > 32) return CSA_ERR_UNSUPPORTED;
+    if (pl.CS > kMaxCluster || pl.R > 32) return CSA_ERR_UNSUPPORTED;
     void (*kern)(const float *, const int *, long long, int, int, int *, int) = nullptr;
     const bool cl = pl.CS > 1;
     switch (pl.R) {

@@ -249,6 +249,40 @@ def test_topk_exact_on_identical_scores(cuda, batch, nq, N, m, k, ts, levels):
     _check_topk_exact(got, ref, qp.cpu().numpy(), m, N)
 
 
+@pytest.mark.parametrize("batch,nq,N,k,mode", [
+    (8, 1, 32768, 1024, "threshold_ties"),   # ties inside the threshold bin (ranked directly)
+    (2, 1, 32768, 1024, "outlier"),          # one huge score: linear bins collapse, radix passes
+    (2, 1, 4096, 256, "neg_inf"),            # -inf among the visible scores
+    (2, 80, 16384, 1024, "normal"),          # one CTA per query (many queries)
+    (1, 160, 16384, 1024, "threshold_ties"),
+    (2, 1, 32768, 1024, "shifted"),          # scores far from zero (large exponent, narrow range)
+])
+def test_topk_exact_value_cases(cuda, batch, nq, N, k, mode):
+    """Exact top-k (ties -> lower index) on score sets that take each branch of
+    the selector: the threshold bin of the value-linear pass ranked directly,
+    and the radix passes over the key bits when that bin is large or the range
+    is not finite."""
+    r = np.random.default_rng(70 + N + nq)
+    s = r.standard_normal((batch, nq, N)).astype(np.float32)
+    if mode == "threshold_ties":
+        for q in np.ndindex(batch, nq):
+            kth = np.sort(s[q])[-k]
+            s[q][r.choice(N, 6, replace=False)] = kth      # six more copies of the k-th largest score
+    elif mode == "outlier":
+        s[:, :, 100] = 1e30
+    elif mode == "neg_inf":
+        s[:, :, ::7] = -np.inf
+    elif mode == "shifted":
+        s = (s * 1e-3 + 3000.0).astype(np.float32)
+    m = 4
+    qp = torch.full((batch, nq), 4 * N - 1, dtype=torch.int32)
+    qp[0, 0] = 4 * (N // 2)                             # one query sees half the entries
+    qp = qp.to(DEV)
+    got = cuda.csa_topk(torch.from_numpy(s).to(DEV), qp, m, k).cpu().numpy()
+    ref = oracle.topk(s.astype(np.float64), qp.cpu().numpy(), m, k)
+    _check_topk_exact(got, ref, qp.cpu().numpy(), m, N)
+
+
 def _check_topk_band(got, ref_scores, qp, m, k, N):
     """Set difference only inside the 1e-4 relative band around the k-th oracle score."""
     for q in np.ndindex(ref_scores.shape[:-1]):
@@ -625,6 +659,8 @@ def test_quantize_fp4_bit_exact(cuda):
     (2, 2, 16, 64, 777, 4, [3107, 50, 3000, 7]),
     (1, 40, 64, 128, 2048, 4, [8191 - 197 * i for i in range(40)]),   # several query groups per sequence
     (2, 1, 32, 256, 1500, 4, [5999, 2001]),                              # d_I = 256, ragged last tile
+    (1, 2, 64, 128, 131072, 4, [524287, 300001]),                        # 128-key tiles, three accumulators, ~7 tiles per CTA
+    (1, 1, 64, 128, 200000, 4, [799999]),                                # 256-key tiles, ~5 per CTA, ragged last tile
 ])
 def test_index_fp4_parity(cuda, batch, nq, H_I, d_I, N, m, ts):
     qI, w, kI, qp = _index_case(batch, nq, H_I, d_I, N, m, ts, seed=80)
