@@ -30,8 +30,9 @@
 // from kernel entry on, each tile's key-validity mask travelling with it;
 // warps 4..7 take each head's 1/RMS from the diagonal of Q Q^T (rewriting the
 // query tile only for a gain or RoPE), then run the softmax, two threads per
-// head (keys 0-31 / 32-63, D/2 output columns each), and stage the output in
-// shared memory for TMA tile stores.  The roles only
+// head (keys 0-31 / 32-63, D/2 output columns each), and store the output
+// rows from registers (64 contiguous bytes per thread and 64-column slab; a
+// shared-memory staging for TMA tile stores measured slower).  The roles only
 // meet at mbarriers, so the gathers of the next work item overlap the output
 // of the current one.  Work items are (query, key split, head half); splits
 // write bf16 partial rows (each divided by its own sum) + (max, sum) that
@@ -235,16 +236,6 @@ CSA_DEVINL uint4 e4m3x8_bf16x8(uint2 raw, uint32_t e) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// TMA tile store of a [rows][128 B] swizzled shared-memory box (one bulk group
-// per issuing thread; pred selects the issuing lane).
-CSA_DEVINL void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, bool pred) {
-    asm volatile(
-        "{\n\t.reg .pred g;\n\tsetp.ne.b32 g, %5, 0;\n\t"
-        "@g cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];\n\t}"
-        ::"l"(map), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"((int)pred)
-        : "memory");
-}
-
 // Warp-uniform bounded wait.  Every lane polls and the outcome is voted: a
 // wait polled by one lane while the others park at a shuffle leaves the warp
 // running its following code far slower (measured: 4x on a pass over the query tile).
@@ -347,7 +338,7 @@ CSA_DEVINL Item work_item(const AttTcParams &p, long long wi) {
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                     const __grid_constant__ CUtensorMap omap, const AttTcParams p) {
+                     const AttTcParams p) {
     using Lt = Layout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem s = carve<D>(smem_raw, p.stages);
@@ -375,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         *s.abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&qmap);
-        tc::prefetch_tmap(&omap);
         if (p.kv_tma) tc::prefetch_tmap(&kvmap);
     }
     // per-dimension query gains of this lane's units (softmax warps), read once
@@ -755,10 +745,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // output: O / l (one split, the output rows) or O / l of this split (a
-            // partial row; the merge weighs the splits).  After the last P.V both P
-            // buffers are free: each warp stages its 16 heads' bf16 values of one
-            // 64-column slab there (alternating buffers) and stores them with one TMA
-            // tile store, the next slab's staging overlapping the previous store.
+            // partial row; the merge weighs the splits), each thread storing its
+            // head's 32 columns of every 64-column slab as four 16-byte stores.
             if (it.ntiles > 0) {
                 const long long gl = jt + it.ntiles - 1;
                 if (!warp_wait(smem_u32(s.oready + (gl & 1)), (uint32_t)((gl >> 1) & 1), p.ctx, s.abort_flag)) break;
@@ -795,31 +783,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v[i] = first ? v[i] * cs.x + pv * cs.y : v[i] * cs.x - pv * cs.y;
                     }
                 }
-                uint8_t *buf = s.p + (size_t)((c >> 6) & 1) * Lt::kPBytes;
-                // the store that last read this buffer (two slabs ago) is done with it
-                if (c >= 128) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                __syncwarp();
+                if (h < a.H) {
+                    uint16_t *dst = (a.splits == 1 ? a.out : a.part_o) + ((size_t)orow * a.H + h) * D + c + 32 * kh;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4 *>(buf + hl * 128 + (((4 * kh + j) ^ (hl & 7)) << 4)) = pack8(v + 8 * j);
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                // (a warp whose 16 heads all lie past H stores nothing; a box that
-                // crosses H is clipped by the tensor map)
-                tma_store_3d(&omap, smem_u32(buf + sp * 16 * 128), c, it.head0 + sp * 16, orow,
-                             lane == 0 && it.head0 + sp * 16 < a.H);
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    for (int j = 0; j < 4; ++j) reinterpret_cast<uint4 *>(dst)[j] = pack8(v + 8 * j);
+                }
             }
-            // the P buffers are written again by the next item's softmax
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            __syncwarp();
             if (h < a.H && a.splits > 1 && kh == 0)
                 a.part_ml[((size_t)it.split * a.n_bq + it.bq) * a.H + h] =
                     it.ntiles > 0 ? make_float2(m_run, l) : make_float2(-INFINITY, 0.f);
             jt += it.ntiles;
         }
     }
-    if (warp >= kSoftmaxWarp0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // output stores complete
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -872,19 +847,6 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st, bool pdl) 
                                CU_TENSOR_MAP_SWIZZLE_128B))
             return CSA_ERR_CUDA;
     }
-    CUtensorMap omap;
-    {
-        // the output rows (one split) or the split partial rows: [rows][H][D] bf16,
-        // boxes of 64 dims x 16 heads (one warp's heads), 128-byte swizzle
-        const uint64_t rows = (uint64_t)(a.splits == 1 ? a.n_bq : (long long)a.splits * a.n_bq);
-        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.H, rows};
-        const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2};
-        const uint32_t box[3] = {64, 16, 1};
-        if (rows > 0x7fffffffULL ||
-            !encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.splits == 1 ? a.out : a.part_o, dims,
-                               strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return CSA_ERR_CUDA;
-    }
     const int grid = (int)std::min<long long>(p.n_work, num_sms());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -896,7 +858,7 @@ int launch_d(const AttendArgs &a, const DevCtx &ctx, cudaStream_t st, bool pdl) 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, qmap, kvmap, omap, p) != cudaSuccess) return CSA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, qmap, kvmap, p) != cudaSuccess) return CSA_ERR_CUDA;
     return a.splits > 1 ? launch_attend_combine(a, st) : CSA_OK;
 }
 
