@@ -79,9 +79,10 @@ int csa_version(void);
  *   gain    [d] fp32 or NULL
  *   out     [batch][floor(T/m)][d] bf16
  * Requirements: batch >= 1, T >= m >= 1, d % 8 == 0, 8 <= d <= 1024, m <= 256
- * (m > 16 or 24*m*d > 96 KiB additionally needs d % 64 == 0, and the pooling
- * weights of one channel slice must fit in shared memory -- e.g. m <= 128 at
- * d = 512; CSA_ERR_UNSUPPORTED otherwise).
+ * (m > 16 or 24*m*d > 96 KiB additionally needs logits 16-byte aligned;
+ * CSA_ERR_UNSUPPORTED otherwise).  Those shapes run the csa_compress_dynamic
+ * kernel with no Z rows (its logits Z + bias are then these logits): results
+ * agree with the small-m kernel up to fp32 rounding order.
  */
 int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
                  int batch, long long T, int d, int m,

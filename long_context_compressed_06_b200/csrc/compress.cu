@@ -8,22 +8,21 @@
 // record "Key takeaways": RMSNorm on the single compressed KV head).
 //
 // The op streams 2*T*d bf16 from HBM and writes T/m*d bf16: it is HBM bound.
-// The softmax weights are static, so each CTA computes them once into shared
-// memory and every element costs one FMA.  Two kernels:
-//   * small m (2m*d weights fit comfortably in shared memory): one warp per
-//     entry, the whole row in registers, RMSNorm by a warp reduction;
-//   * large m (HCA, m = 128): a thread-block cluster splits the channels, each
-//     CTA keeps the weights of its channel slice in shared memory, and the
-//     RMSNorm sum of squares is exchanged through distributed shared memory.
-#include <cooperative_groups.h>
-
+//   * small m (2m*d weights fit comfortably in shared memory): the softmax
+//     weights are static, so each CTA computes them once into shared memory
+//     and every element costs one FMA; one warp per entry, the whole row in
+//     registers, RMSNorm by a warp reduction;
+//   * large m (HCA, m = 128): the input-dependent compressor with no Z rows
+//     (its logits Z + bias reduce to the static logits as the bias), a thread
+//     per (entry, 8 channels) with an online softmax over the 2m rows: the
+//     weights of all d channels do not fit in shared memory, and a cluster
+//     that split the channels and exchanged the RMSNorm sums measured 1.18
+//     TB/s against this kernel's rate.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace csa {
 namespace {
@@ -130,119 +129,6 @@ __global__ void __launch_bounds__(256) compress_small_kernel(
     }
 }
 
-// ------------------------------------------------------------------ large m
-// A cluster of G CTAs handles groups of E = 256/dc consecutive entries; CTA
-// `rank` owns channels [rank*dc, (rank+1)*dc).  The 256 threads are RG row
-// groups x (dc/8) channel chunks while pooling (thread sums rows rg, rg+RG, ..)
-// and E entries x dc channels (one output each) while reducing/normalising.
-// A thread issues the 16-byte loads of NR of its rows of every entry of the
-// group before the first FMA, so E*NR loads per thread are in flight (the op
-// is bound by HBM latency x bytes in flight); larger m takes several batches.
-template <int E, int NR>
-__global__ void __launch_bounds__(256, 1) compress_cluster_kernel(
-    const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, const float *__restrict__ logits,
-    int batch, long long T, int d, int m, int apply_rms, const float *__restrict__ gain, float eps,
-    uint16_t *__restrict__ out, long long N, int G) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = (int)cluster.block_rank();
-    const int dc = d / G, c_base = rank * dc;  // E * dc == 256
-    const int nchunk = dc >> 3, RG = 256 / nchunk;
-    extern __shared__ __align__(16) float smem[];
-    float *w_full = smem;                      // [2m][dc]
-    float *w_first = w_full + 2 * m * dc;      // [m][dc]
-    float *red = w_first + m * dc;             // [RG][E][dc]
-    float *part = red + (size_t)RG * E * dc;   // [2][E] partial sums of squares (double buffered)
-    float *wsum = part + 2 * E;                // [8] warp partials
-    pooling_weights(logits, d, m, c_base, dc, w_full, w_first);
-    __syncthreads();
-
-    const int chunk = threadIdx.x % nchunk, rg = threadIdx.x / nchunk;
-    const int my_e = threadIdx.x / dc, my_c = threadIdx.x % dc;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long groups = (N + E - 1) / E;
-    const long long items = (long long)batch * groups;
-    const long long cid = blockIdx.x / G, ncl = gridDim.x / G;
-    int round = 0;
-    for (long long it = cid; it < items; it += ncl, ++round) {
-        const long long b = it / groups, i0 = (it - b * groups) * E;
-        const uint16_t *Ab = A + (size_t)b * T * d + c_base + chunk * 8;
-        const uint16_t *Bb = B + (size_t)b * T * d + c_base + chunk * 8;
-        float acc[E][8];
-#pragma unroll
-        for (int e = 0; e < E; ++e)
-#pragma unroll
-            for (int q = 0; q < 8; ++q) acc[e][q] = 0.f;
-        for (int r0 = rg; r0 < 2 * m; r0 += RG * NR) {
-            // all loads of this batch first (rows past 2m or N, and entry 0's missing B half, read nothing)
-            uint4 x[E][NR];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const long long i = i0 + e;
-#pragma unroll
-                for (int k = 0; k < NR; ++k) {
-                    const int r = r0 + RG * k;
-                    const uint16_t *src = nullptr;
-                    if (i < N && r < 2 * m) {
-                        if (r >= m)
-                            src = Ab + (size_t)(i * m + r - m) * d;
-                        else if (i > 0)
-                            src = Bb + (size_t)((i - 1) * m + r) * d;
-                    }
-                    x[e][k] = src ? ldg_stream(src) : make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const long long i = i0 + e;
-#pragma unroll
-                for (int k = 0; k < NR; ++k) {
-                    const int r = r0 + RG * k;
-                    if (r >= 2 * m) continue;
-                    if (i == 0) {
-                        if (r >= m) fma8(acc[e], w_first + (size_t)(r - m) * dc + chunk * 8, x[e][k]);
-                    } else {
-                        fma8(acc[e], w_full + (size_t)r * dc + chunk * 8, x[e][k]);
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            float4 *dst = reinterpret_cast<float4 *>(red + ((size_t)rg * E + e) * dc + chunk * 8);
-            dst[0] = make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
-            dst[1] = make_float4(acc[e][4], acc[e][5], acc[e][6], acc[e][7]);
-        }
-        __syncthreads();
-        float v = 0.f;
-        for (int g = 0; g < RG; ++g) v += red[((size_t)g * E + my_e) * dc + my_c];
-        float rn = 1.f;
-        if (apply_rms) {
-            const int slot = round & 1;
-            const float s = warp_sum(v * v);
-            if (lane == 0) wsum[warp] = s;
-            __syncthreads();
-            if (threadIdx.x < E) {
-                const int wpe = dc / 32;  // warps per entry
-                float t = 0.f;
-                for (int w8 = 0; w8 < wpe; ++w8) t += wsum[threadIdx.x * wpe + w8];
-                part[slot * E + threadIdx.x] = t;
-            }
-            cluster.sync();
-            float tot = 0.f;
-            for (int g = 0; g < G; ++g) tot += cluster.map_shared_rank(part, g)[slot * E + my_e];
-            rn = 1.0f / sqrtf(tot / (float)d + eps);
-        }
-        const long long i = i0 + my_e;
-        if (i < N) {
-            const float g = (apply_rms && gain) ? __ldg(gain + c_base + my_c) : 1.f;
-            const __nv_bfloat16 o = __float2bfloat16_rn(v * rn * g);
-            out[((size_t)b * N + i) * d + c_base + my_c] = *reinterpret_cast<const uint16_t *>(&o);
-        }
-        __syncthreads();  // red[] and wsum[] are rewritten by the next round
-    }
-    cluster.sync();  // no CTA leaves while a peer may still read its part[]
-}
-
 template <int MT, int CPL>
 cudaError_t run_small(const uint16_t *A, const uint16_t *B, const float *logits, int batch, long long T,
                       int d, int m, int apply_rms, const float *gain, float eps, uint16_t *out,
@@ -280,46 +166,11 @@ int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, i
             err = run_small<0, 4>(A, B, logits, batch, T, d, m, apply_rmsnorm, gain, eps, out, N, small_smem, grid, st);
         return err == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
     }
-    // cluster path: channel slices of dc = d / G, G = min(8, d / 64), E = 256 / dc
-    if (d % 64 != 0) return CSA_ERR_UNSUPPORTED;
-    const int G = std::min(8, d / 64);
-    const int dc = d / G;
-    if (dc > 256 || 256 % dc != 0) return CSA_ERR_UNSUPPORTED;
-    const int E = 256 / dc;
-    const int RG = 256 / (dc / 8);
-    const size_t smem = ((size_t)3 * m * dc + (size_t)RG * E * dc + 2 * E + 8) * sizeof(float);
-    if (smem > 220 * 1024) return CSA_ERR_UNSUPPORTED;
-    // loads in flight per thread: E entries x NR rows (32 registers of uint4 at most)
-    const int rows_per_thread = (2 * m + RG - 1) / RG;
-    int NR = 32 / E;
-    while (NR > 1 && NR / 2 >= rows_per_thread) NR /= 2;
-    void (*k)(const uint16_t *, const uint16_t *, const float *, int, long long, int, int, int, const float *,
-              float, uint16_t *, long long, int) = nullptr;
-#define CSA_CK(e_, nr_) \
-    if (E == e_ && NR == nr_) k = compress_cluster_kernel<e_, nr_>;
-    CSA_CK(4, 1) CSA_CK(4, 2) CSA_CK(4, 4) CSA_CK(4, 8)
-    CSA_CK(2, 1) CSA_CK(2, 2) CSA_CK(2, 4) CSA_CK(2, 8) CSA_CK(2, 16)
-    CSA_CK(1, 1) CSA_CK(1, 2) CSA_CK(1, 4) CSA_CK(1, 8) CSA_CK(1, 16) CSA_CK(1, 32)
-#undef CSA_CK
-    if (!k) return CSA_ERR_UNSUPPORTED;
-    err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return CSA_ERR_CUDA;
-    const long long items = (long long)batch * ((N + E - 1) / E);
-    const long long nclusters = std::min<long long>(items, std::max(1, sms / G));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(nclusters * G));
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, k, A, B, logits, batch, T, d, m, apply_rmsnorm, gain, eps, out, N, G);
-    return err == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+    // large m: the input-dependent compressor without Z rows, the logits as its
+    // bias (read as float4: 16-byte aligned)
+    if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return CSA_ERR_UNSUPPORTED;
+    return launch_compress_dynamic(A, B, nullptr, nullptr, logits, batch, T, d, m, apply_rmsnorm, gain, eps, 0, N,
+                                   N, out, st);
 }
 
 }  // namespace csa

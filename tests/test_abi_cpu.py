@@ -61,6 +61,8 @@ def test_compress_validation(lib):
     assert f(A16, A16, A16, 1, 64, 64, 4, 1, NULL, -1.0, A16b, NULL) == csa.CSA_ERR_INVALID   # eps
     assert f(A16, A16, A16, 1, 4096, 2048, 4, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
     assert f(A16, A16, A16, 1, 4096, 64, 512, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
+    # large m reads the logits as float4: 4-byte aligned logits are refused before any launch
+    assert f(A16, A16, ctypes.c_void_p(0x10004), 1, 4096, 64, 128, 1, NULL, 1e-6, A16b, NULL) == csa.CSA_ERR_UNSUPPORTED
 
 
 def test_compress_dynamic_validation(lib):
