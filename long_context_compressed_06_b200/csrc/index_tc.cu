@@ -10,14 +10,18 @@
 // sum_h w_h * ReLU(.) is a loop over columns inside one thread, and a warp
 // stores 32 consecutive scores.
 //
-// Warp roles (320 threads):  warp 0 -- TMA producer (key tiles into a STAGES
-// ring, query tile once per query group); warp 1 -- TMEM owner and MMA issuer
-// (lane 0 issues; tcgen05.mma kind::f16, fp32 accumulate, four accumulator
-// buffers when N <= 128, else two); warps 2..9 -- two epilogue groups of four
-// warps taking alternate tiles (tcgen05.ld, ReLU, weighted head sum, causal
-// mask, store).  Every mbarrier wait is bounded (csa_sync_status reports a
-// timeout).  Decode streams the key cache from HBM; prefill is bound by the
-// epilogue (64 FMAs per key per query) rather than the tensor cores.
+// Warp roles:  warp 0 -- TMA producer (key tiles into a STAGES ring, query
+// tile once per query group); warp 1 -- TMEM owner and MMA issuer (lane 0
+// issues; tcgen05.mma kind::f16, fp32 accumulate, four accumulator buffers when
+// N <= 128, else two); then two epilogue groups of EW warps taking alternate
+// tiles (tcgen05.ld, ReLU, weighted head sum, causal mask, store).  Every
+// mbarrier wait is bounded (csa_sync_status reports a timeout).  Decode (one
+// query per tile) streams the key cache from HBM: EW = 4, one warp per TMEM
+// lane quarter.  Prefill is bound by the epilogue (64 FMAs per key per query)
+// rather than the tensor cores: with four queries per tile one warp's pass
+// over 256 accumulator columns took longer than the MMAs of two tiles, so
+// EW = 8 splits the queries between two warps of the same lanes (1.69 ->
+// 1.35 ms on the 4096-query prefill); at decode the extra warps cost ~1 us.
 #include <algorithm>
 
 #include "common.cuh"
@@ -27,7 +31,6 @@
 namespace csa {
 namespace {
 
-constexpr int kThreads = 320;  // producer warp, MMA warp, two epilogue groups of four warps
 constexpr int kTileKeys = 128;
 constexpr int kMaxStages = 6;
 constexpr int kMaxAcc = 4;   // TMEM accumulators (two when N = NQ x H_pad > 128)
@@ -76,12 +79,10 @@ CSA_DEVINL void advance(const IndexTcParams &p, Cursor &c) {
     }
 }
 
-// Named barrier of one epilogue group (128 threads).
+// Named barrier of one epilogue group of EW warps.
+template <int EW>
 CSA_DEVINL void group_bar(int eg) {
-    if (eg == 0)
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-    else
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(eg + 1), "n"(EW * 32) : "memory");
 }
 
 // Slot and phase of a ring of n barriers.
@@ -96,7 +97,8 @@ struct Ring {
     }
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int EW>  // warps per epilogue group: 4 (one per TMEM lane quarter) or 8 (two)
+__global__ void __launch_bounds__(64 + 64 * EW, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const IndexTcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < p.n_acc; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 4);
+            mbar_init(tempty + a, EW);
         }
         mbar_init(qfull, 1);
         mbar_init(qempty, 1);
@@ -218,12 +220,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------------------ epilogue
-        // Two groups of four warps take alternate tiles (tile i -> group i & 1,
-        // accumulator i % n_acc), doubling the epilogue rate.
-        const int eg = (warp - 2) >> 2;
+        // Two groups of EW warps take alternate tiles (tile i -> group i & 1,
+        // accumulator i % n_acc), doubling the epilogue rate; with EW = 8 the two
+        // warps of a lane quarter take the even and the odd queries of a tile.
+        constexpr int kLoads = EW == 4 ? 4 : 2;  // 16-column TMEM loads per wait (registers)
+        const int eg = (warp - 2) / EW;
+        const int half = ((warp - 2) % EW) >> 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
-        const int et = (threadIdx.x - 64) & 127;
+        const int et = (threadIdx.x - 64) % (EW * 32);
         float *ws_g = w_s + eg * p.NQ * p.H_pad;
         int *nv_g = nvis_s + eg * p.NQ;
         int loaded_b = -1, loaded_g = -1;
@@ -232,17 +237,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if ((li & 1) != eg) continue;
             const int b = cu.b, g = cu.g;
             if (b != loaded_b || g != loaded_g) {
-                group_bar(eg);
-                for (int i = et; i < p.NQ * p.H_pad; i += 128) {
+                group_bar<EW>(eg);
+                for (int i = et; i < p.NQ * p.H_pad; i += EW * 32) {
                     const int qi = i / p.H_pad, h = i - qi * p.H_pad;
                     const int q = g * p.NQ + qi;
                     ws_g[i] = (q < p.nq && h < p.H_I) ? __ldg(p.w + ((size_t)b * p.nq + q) * p.H_I + h) : 0.f;
                 }
-                for (int qi = et; qi < p.NQ; qi += 128) {
+                for (int qi = et; qi < p.NQ; qi += EW * 32) {
                     const int q = g * p.NQ + qi;
                     nv_g[qi] = q < p.nq ? (int)n_visible(__ldg(p.q_pos + (size_t)b * p.nq + q), p.m, p.N) : 0;
                 }
-                group_bar(eg);
+                group_bar<EW>(eg);
                 loaded_b = b;
                 loaded_g = g;
             }
@@ -255,30 +260,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_after_sync();
             const long long s = (long long)cu.kt * kTileKeys + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.n_cols);
-            for (int qi = 0; qi < p.NQ; ++qi) {
+            for (int qi = half; qi < p.NQ; qi += EW / 4) {
                 const int q = g * p.NQ + qi;
                 if (q >= p.nq) break;
-                // four independent partial sums (one per 16-column load) keep the
-                // FMA chains short
-                float part[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int hc = 0; hc < p.H_pad; hc += 64) {
-                    // up to four 16-column loads in flight per wait
-                    float v[64];
-                    const int nl = min(4, (p.H_pad - hc) >> 4);
+                // independent partial sums (one per 16-column load) keep the FMA
+                // chains short
+                float part[kLoads];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < kLoads; ++u) part[u] = 0.f;
+                for (int hc = 0; hc < p.H_pad; hc += 16 * kLoads) {
+                    float v[16 * kLoads];
+                    const int nl = min(kLoads, (p.H_pad - hc) >> 4);
+#pragma unroll
+                    for (int u = 0; u < kLoads; ++u)
                         if (u < nl) tc::tmem_ld16(tbase + (uint32_t)(qi * p.H_pad + hc + 16 * u), v + 16 * u);
                     tc::tmem_wait_ld();
                     const float *ws = ws_g + qi * p.H_pad + hc;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < kLoads; ++u)
                         if (u < nl) {
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
                                 part[u] = fmaf(ws[16 * u + i], fmaxf(v[16 * u + i], 0.f), part[u]);
                         }
                 }
-                const float score = (part[0] + part[1]) + (part[2] + part[3]);
+                float score = 0.f;
+#pragma unroll
+                for (int u = 0; u < kLoads; ++u) score += part[u];
                 if (s < p.N) p.scores[((size_t)b * p.nq + q) * p.N + s] = s < nv_g[qi] ? score : -INFINITY;
             }
             tc::fence_before_sync();
@@ -352,10 +360,14 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
     }
     const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + p.q_bytes + 2 * ((size_t)NQ * p.H_pad * 4 + NQ * 4) +
                         8 + (2 * kMaxStages + 2 * kMaxAcc + 2) * 8 + 16;
-    if (cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    // several queries per tile: two warps per TMEM lane quarter split them
+    const int EW = NQ >= 2 ? 8 : 4;
+    void (*kern)(const CUtensorMap, const CUtensorMap, const IndexTcParams) =
+        EW == 8 ? index_tc_kernel<8> : index_tc_kernel<4>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
     const int grid = (int)std::min<long long>(p.total_work, num_sms());
-    index_tc_kernel<<<grid, kThreads, smem, st>>>(kmap, qmap, p);
+    kern<<<grid, 64 + 64 * EW, smem, st>>>(kmap, qmap, p);
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
