@@ -24,9 +24,11 @@
 // n % 32, column n / 32 of the block, copied into each of the four lane
 // quarters (the rows of A in a quarter read B's scale factors there).
 //
-// Warp roles (704 threads): warp 0 -- TMA producer (key tiles into a ring of
+// Warp roles (736 threads): warp 0 -- TMA producer (key tiles into a ring of
 // stages, the query group's codes once per group); warp 1 -- TMEM owner and
-// MMA issuer (lane 0 issues through guarded instructions); warps 2..5 -- scale
+// MMA issuer of sub-tile 0, warp 22 -- MMA issuer of sub-tile 1 (lane 0 issues
+// through guarded instructions; one thread issues a tcgen05.mma only every
+// ~100 cycles, two threads twice as fast); warps 2..5 -- scale
 // movers (each thread stages its key row's scale bytes with cp.async several
 // tiles ahead and writes them into the tile's tensor-memory slot; the
 // query-head scales once per group); warps 6..21 -- up to four epilogue
@@ -44,7 +46,8 @@ namespace csa {
 namespace {
 
 constexpr int kEpiGroups = 4;  // epilogue groups of four warps, taking tiles in turn
-constexpr int kThreads = 192 + 128 * kEpiGroups;
+constexpr int kMma2Warp = 6 + 4 * kEpiGroups;  // the second MMA issuer (sub-tile 1)
+constexpr int kThreads = 192 + 128 * kEpiGroups + 32;
 constexpr int kSubKeys = 128;   // keys of one MMA (M); a tile holds p.sub of them
 constexpr int kMaxStages = 20;
 constexpr int kMaxAcc = 4;
@@ -170,20 +173,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);
+            mbar_init(empty + s, p.sub);  // one commit per MMA issuer
         }
         for (int a = 0; a < p.n_acc; ++a) {
-            mbar_init(tfull + a, 1);
+            mbar_init(tfull + a, p.sub);
             mbar_init(tempty + a, 4);
         }
         for (int s = 0; s < kSfSlots; ++s) {
             mbar_init(sfull + s, 4);
-            mbar_init(sempty + s, 1);
+            mbar_init(sempty + s, p.sub);
         }
         mbar_init(qfull, 1);
-        mbar_init(qempty, 1);
+        mbar_init(qempty, p.sub);
         mbar_init(qsfull, 4);
-        mbar_init(qsempty, 1);
+        mbar_init(qsempty, p.sub);
         for (int s = 0; s < kSfAhead; ++s) mbar_init(sfld + s, 128);  // one cp.async arrival per mover thread
         *abort_flag = 0;
         fence_mbar_init();
@@ -226,8 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(smem_u32(full + (j % p.stages)), (uint32_t)((j / p.stages) & 1), p.ctx, nullptr);
         if (gi > 0) mbar_wait(smem_u32(qfull), (uint32_t)((gi - 1) & 1), p.ctx, nullptr);
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || (warp == kMma2Warp && p.sub == 2)) {
+        // ------------------------------------------------------------ MMA issuers
+        // One warp per sub-tile (warp 1: sub-tile 0, the last warp: sub-tile 1):
+        // a single thread issues a tcgen05.mma every ~100 cycles at best
+        // (measured), so the two sub-tiles' independent accumulators are fed
+        // by two issuing threads.  Both wait on the same barriers and each
+        // commits to the ones the tile releases (counts of two).
+        const int h = warp == 1 ? 0 : 1;
         long long gi = 0;
         Ring kr, ar, sr;
         const uint64_t kdesc0 = tc::smem_desc(smem_u32(k_smem), p.sbo, p.layout);
@@ -247,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_all(sfull + sl, sr.phase)) break;
             tc::fence_after_sync();
             const uint64_t kd = kdesc0 + ((uint64_t)(st * p.stage_bytes) >> 4);
-            for (int h = 0; h < p.sub; ++h) {
+            {
                 // sub-tile h: keys 128h.. of the tile into its own accumulator
                 const uint32_t d_tmem = tmem_base + (uint32_t)((acc * p.sub + h) * p.n_cols);
                 for (int ks = 0; ks < NKS; ++ks)
@@ -357,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (pf.w < w1) advance(p, pf);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else {
+    } else if (warp < kMma2Warp) {
         // ------------------------------------------------------------ epilogue (warps 6..21)
         // Groups of four warps, one per accumulator (n_acc <= kEpiGroups; the rest
         // idle): tile i -> accumulator and group i % n_acc.  Each accumulator's
