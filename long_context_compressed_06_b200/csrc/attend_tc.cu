@@ -49,7 +49,8 @@
 namespace csa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kMma2Warp = 8;   // the second MMA issuer
+constexpr int kThreads = 288;
 constexpr int kTileKeys = 64;
 constexpr int kHeads = 64;          // heads per CTA (M of every MMA)
 constexpr int kSoftmaxWarp0 = 4;
@@ -349,20 +350,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < p.stages; ++i) {
             // one cp.async completion arrive per producer thread + the key-mask arrive
             mbar_init(s.kfull + i, kProducerWarps * 32 + 1);
-            mbar_init(s.kempty + i, 1);
+            mbar_init(s.kempty + i, 2);  // one commit per MMA issuer
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(s.sfull + i, 1);
+            mbar_init(s.sfull + i, 2);
             mbar_init(s.sempty + i, 128);
             mbar_init(s.pfull + i, 128);
-            mbar_init(s.pempty + i, 1);
+            mbar_init(s.pempty + i, 2);
         }
-        mbar_init(s.oready, 1);
-        mbar_init(s.oready + 1, 1);
+        mbar_init(s.oready, 2);
+        mbar_init(s.oready + 1, 2);
         mbar_init(s.qready, 128);
-        mbar_init(s.qempty, 1);
+        mbar_init(s.qempty, 2);
         mbar_init(s.qfull, 1);
-        mbar_init(s.qqready, 1);
+        mbar_init(s.qqready, 2);
         *s.abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&qmap);
@@ -390,6 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_o = tmem;                  // lanes 0-15 of each sub-partition, columns 0..D-1
     const uint32_t tmem_s = tmem + (16u << 16);    // lanes 16-31, columns 0..127 (two S buffers)
     const uint32_t tmem_qq = tmem_s + 128;          // lanes 16-31, columns 128..191 (Q Q^T of the item)
+    // the second MMA issuer's halves of S and Q Q^T: lanes 16-31, columns 192..383
+    constexpr uint32_t kIss2Cols = 192;
     // the query tile is rewritten in shared memory only for a gain or partial RoPE
     const bool q_rw = a.q_gain != nullptr || a.rope_cos != nullptr;
 
@@ -510,14 +513,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             jt += it.ntiles;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 0) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 0 || warp == kMma2Warp) {
+        // ------------------------------------------------------------ MMA issuers
         // Event driven: P.V for tile i as soon as P_i is written, QK for the
         // next tile as soon as its keys have landed and an S buffer is free.
         // The whole warp runs the loop and polls (decisions are lane 0's, made
         // warp-uniform by a shuffle); lane 0 issues through guarded
         // instructions, never a branch.  Descriptors are built
         // once and advanced by constant offsets.
+        // Two issuers (warp 0 and warp 8) run the same loop: one thread issues a
+        // tcgen05.mma only every ~100 cycles (measured), so each issues half of
+        // every product -- Q Q^T and QK split along the head dimension into two
+        // accumulators that the softmax adds, P.V by the two 256-column halves
+        // of O (D = 512; below that the first issuer takes all of P.V) -- and
+        // commits to every barrier the products release (counts of two).
+        const int iss = warp == 0 ? 0 : 1;
+        constexpr int kQkSteps = Lt::kChunks * 4;  // K steps of 16 over the head dimension
+        const int qk0 = iss * (kQkSteps / 2), qk1 = qk0 + kQkSteps / 2;
+        constexpr bool kPvSplit = D == 512;
+        const int pv0 = kPvSplit ? iss * (D / 2) : (iss == 0 ? 0 : D), pv1 = kPvSplit ? pv0 + D / 2 : D;
+        const uint32_t s_off = iss ? kIss2Cols : 0u;
         const uint64_t qdesc = tc::smem_desc(smem_u32(s.q), 1024, tc::kLayoutSw128);
         const uint64_t kdesc0 = tc::smem_desc(smem_u32(s.k), 1024, tc::kLayoutSw128);
         const uint64_t vdesc0 = tc::smem_desc_lbo(smem_u32(s.k), kTileKeys * 128, 1024, tc::kLayoutSw128);
@@ -532,21 +547,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n_items > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qempty), (n_items - 1) & 1u, p.ctx,
                                                                  s.abort_flag)))
                 break;
-            mbar_arrive_expect_tx(smem_u32(s.qfull), Lt::kQBytes, lane == 0);
+            mbar_arrive_expect_tx(smem_u32(s.qfull), Lt::kQBytes, lane == 0 && iss == 0);
             for (int c = 0; c < Lt::kChunks; ++c)
                 tc::tma_load_3d(smem_u32(s.q + (size_t)c * kHeads * 128), &qmap, smem_u32(s.qfull), c * 64,
-                                it.head0, (int)it.bq, lane == 0);
+                                it.head0, (int)it.bq, lane == 0 && iss == 0);
             // Q Q^T of the raw rows: its diagonal gives every head's sum of squares
             // for the RMSNorm (applied to the scores in fp32)
             if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s.qfull), n_items & 1u, p.ctx, s.abort_flag))) break;
             tc::fence_after_sync();
-#pragma unroll
-            for (int c = 0; c < Lt::kChunks; ++c)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(tmem_qq, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
-                                qdesc + ((c * kHeads * 128 + kk * 32) >> 4), p.idesc_qk, (c | kk) ? 1u : 0u,
-                                lane == 0);
+            for (int t = qk0; t < qk1; ++t) {
+                const int c = t >> 2, kk = t & 3;
+                tc::mma_f16(tmem_qq + s_off, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                            qdesc + ((c * kHeads * 128 + kk * 32) >> 4), p.idesc_qk, t > qk0 ? 1u : 0u, lane == 0);
+            }
             tc::mma_commit(smem_u32(s.qqready), lane == 0);
             // the softmax warps have read the diagonal (so the next item's Q Q^T may
             // overwrite it) and, with a gain or RoPE, rewritten the tile
@@ -567,13 +580,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::fence_proxy_async_smem();  // cp.async data -> tensor-core reads
                         tc::fence_after_sync();
                         const uint64_t kd = kdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
-#pragma unroll
-                        for (int c = 0; c < Lt::kChunks; ++c)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc::mma_f16(tmem_s + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
-                                            kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk,
-                                            (c | kk) ? 1u : 0u, issuer);
+                        for (int t = qk0; t < qk1; ++t) {
+                            const int c = t >> 2, kk = t & 3;
+                            tc::mma_f16(tmem_s + s_off + sb * kTileKeys, qdesc + ((c * kHeads * 128 + kk * 32) >> 4),
+                                        kd + ((c * kTileKeys * 128 + kk * 32) >> 4), p.idesc_qk, t > qk0 ? 1u : 0u,
+                                        issuer);
+                        }
                         tc::mma_commit(smem_u32(s.sfull + sb), issuer);
                         if (nqk + 1 == it.ntiles) tc::mma_commit(smem_u32(s.qempty), issuer);  // query tile no longer read
                         ++nqk;
@@ -590,8 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t vd = vdesc0 + ((uint64_t)(st * Lt::kStageBytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kTileKeys / 16; ++kk)
-#pragma unroll
-                            for (int n0 = 0; n0 < D; n0 += Lt::kPvN)
+                            for (int n0 = pv0; n0 < pv1; n0 += Lt::kPvN)
                                 // V[keys][dims] read MN-major: 64-dim groups kTileKeys*128 bytes
                                 // apart (LBO), 8-key groups 1024 bytes apart (SBO); K step = 16 keys
                                 tc::mma_f16(tmem_o + n0, pd + ((kk * 32) >> 4),
@@ -646,14 +657,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_after_sync();
             float rq;
             {
-                float v[32];
+                float v[32], v2[32];
                 tmem_ld_half32(tmem_qq + lane_base, v);
+                tmem_ld_half32(tmem_qq + kIss2Cols + lane_base, v2);  // the second issuer's half
                 tc::tmem_wait_ld();
                 // select v[hl & 31] without an indexed (local-memory) access
                 const int di = hl & 31;
                 float d = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) d += (i == di) ? v[i] : 0.f;
+                for (int i = 0; i < 32; ++i) d += (i == di) ? v[i] + v2[i] : 0.f;
                 const float other = __shfl_xor_sync(0xffffffffu, d, 16);
                 const float ss = kh == (hl >> 5) ? d : other;
                 rq = (1.0f / sqrtf(ss / (float)D + a.eps)) * a.scale * 1.4426950408889634f;
@@ -681,9 +693,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint64_t vmask = s.kmask[st] >> (32 * kh);
                 tc::fence_after_sync();
-                float sc[32];
+                float sc[32], sc2[32];
                 tmem_ld_half32(tmem_s + lane_base + sb * kTileKeys, sc);
+                tmem_ld_half32(tmem_s + kIss2Cols + lane_base + sb * kTileKeys, sc2);  // second issuer's half
                 tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sc[i] += sc2[i];
                 tc::fence_before_sync();
                 mbar_arrive(smem_u32(s.sempty + sb));
                 float mt = -INFINITY;
