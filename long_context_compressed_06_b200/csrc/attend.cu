@@ -19,13 +19,34 @@ namespace {
 // then their bf16 rows in split order, 8 splits' loads in flight at a time.
 //   out = sum_s 2^(m_s - M) l_s O_s / (sum_s 2^(m_s - M) l_s + sink)
 // with O_s the split's row already divided by its own sum l_s.
+//
+// Partial layout.  Standard: [H][D] per (split, query).  Warp-store order
+// (part_perm, H % 64 == 0): the attention's softmax warp of lane quarter sp
+// holds 16 heads x 64 columns of each 64-column slab, a thread 8 columns per
+// store; it stores them as one contiguous 2 KiB block per warp and slab (16-byte
+// piece j*32 + lane, lane = head%16 + 16 * (column half)), so that every store
+// instruction writes whole sectors.  Piece P of a (split, query) region then
+// holds head hh*64 + sp*16 + (lane & 15), columns slab*64 + (lane >> 4)*32 + j*8
+// with (hh*slabs + slab, sp, j, lane) = P's digits (slabs = D/64); the merge
+// takes one piece per thread, so its loads of the partials are coalesced.
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendArgs a) {
     const int tph = a.D / 8;                              // threads per head
     const long long bq = blockIdx.x;
-    const int h = blockIdx.y * (kCombineThreads / tph) + threadIdx.x / tph;
-    const int c0 = (threadIdx.x % tph) * 8;
+    int h, c0;
+    long long piece;  // 16-byte piece of the (split, query) region this thread merges
+    if (a.part_perm) {
+        const int P = blockIdx.y * kCombineThreads + threadIdx.x;
+        const int ln = P & 31, j = (P >> 5) & 3, sp = (P >> 7) & 3, rest = P >> 9, slabs = a.D / 64;
+        h = (rest / slabs) * 64 + sp * 16 + (ln & 15);
+        c0 = (rest % slabs) * 64 + (ln >> 4) * 32 + j * 8;
+        piece = P;
+    } else {
+        h = blockIdx.y * (kCombineThreads / tph) + threadIdx.x / tph;
+        c0 = (threadIdx.x % tph) * 8;
+        piece = (long long)h * tph + c0 / 8;
+    }
     const bool active = h < a.H;  // no early exit: the RoPE shuffles need whole warps
     // launched as a programmatic dependent of the attention kernel: its partials
     // are complete only once that grid is
@@ -43,7 +64,8 @@ __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendA
         for (int j = 0; j < 8; ++j)
             if (j < ns) {
                 ml[j] = a.part_ml[(s0 + j) * stride + row];
-                v[j] = *reinterpret_cast<const uint4 *>(a.part_o + ((s0 + j) * stride + row) * a.D + c0);
+                v[j] = *reinterpret_cast<const uint4 *>(
+                    a.part_o + ((s0 + j) * stride + (size_t)bq * a.H) * a.D + (size_t)(active ? piece : 0) * 8);
             }
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -64,10 +86,12 @@ __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendA
     for (int e = 0; e < 8; ++e) o[e] = acc[e] * inv;
     if (a.rope_cos) {
         // conjugate rotation of the trailing kRopeDim channels: channel D-64+j pairs
-        // with D-32+j, held by the thread 4 lanes away (32 channels)
+        // with D-32+j, held by the thread 4 lanes away (32 channels; 16 lanes in
+        // the warp-store order)
         float pv[8];
+        const int pl = a.part_perm ? 16 : 4;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], 4);
+        for (int e = 0; e < 8; ++e) pv[e] = __shfl_xor_sync(0xffffffffu, o[e], pl);
         if (c0 >= a.D - kRopeDim) {
             const long long t = __ldg(a.q_pos + bq);
             const bool first = c0 < a.D - kRopeDim / 2;
@@ -79,7 +103,7 @@ __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendA
             }
         }
     }
-    if (active) *reinterpret_cast<uint4 *>(a.out + row * a.D + c0) = pack8(o);
+    if (active) *reinterpret_cast<uint4 *>(a.out + row * a.D + c0) = pack8(o);  // row = bq * H + h
 }
 
 // [splits][n_bq][H][D] bf16 rows, then [splits][n_bq][H] float2 (max, sum)
@@ -153,6 +177,7 @@ int launch_attend(const uint16_t *q, const float *q_gain, const float *sinks, co
     if (need > 0) {
         if (!ws || ws_bytes < need) return CSA_ERR_WORKSPACE;
         a.part_o = reinterpret_cast<uint16_t *>(ws);
+        a.part_perm = H % 64 == 0 ? 1 : 0;
         a.part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) +
                                                (size_t)a.splits * a.n_bq * H * D * sizeof(uint16_t));
     }

@@ -39,6 +39,7 @@ struct AttendArgs {
     float scale, eps;
     uint16_t *out;          // [n_bq][H][D]
     uint16_t *part_o;       // [splits][n_bq][H][D] bf16 partial outputs, each divided by its own sum
+    int part_perm;          // part_o rows of one (split, query) in warp-store order (see attend_combine)
     float2 *part_ml;        // [splits][n_bq][H] (running max in log2 units, sum)
     int splits;
     long long keys_per_split;

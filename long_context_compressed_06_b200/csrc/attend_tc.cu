@@ -798,7 +798,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v[i] = first ? v[i] * cs.x + pv * cs.y : v[i] * cs.x - pv * cs.y;
                     }
                 }
-                if (h < a.H) {
+                if (a.splits > 1 && a.part_perm) {
+                    // split partials in warp-store order (the merge reads them so): this
+                    // warp's 16 heads x 64 columns of the slab as one 2 KiB block, piece
+                    // j * 32 + lane, so that every store writes whole sectors
+                    uint8_t *blk = reinterpret_cast<uint8_t *>(a.part_o + ((size_t)orow * a.H + it.head0) * D) +
+                                   (size_t)(c / 64) * 8192 + (size_t)sp * 2048;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) reinterpret_cast<uint4 *>(blk)[j * 32 + lane] = pack8(v + 8 * j);
+                } else if (h < a.H) {
                     uint16_t *dst = (a.splits == 1 ? a.out : a.part_o) + ((size_t)orow * a.H + h) * D + c + 32 * kh;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) reinterpret_cast<uint4 *>(dst)[j] = pack8(v + 8 * j);
