@@ -54,9 +54,36 @@ __global__ void __launch_bounds__(kCombineThreads) attend_combine_kernel(AttendA
     const size_t stride = (size_t)a.n_bq * a.H;          // between splits, in rows
     const size_t row = (size_t)bq * a.H + (active ? h : 0);
     float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[s * stride + row].x);
     float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < a.splits; s0 += 8) {
+    const uint16_t *src0 = a.part_o + (size_t)bq * a.H * a.D + (size_t)(active ? piece : 0) * 8;
+    if (a.splits <= 16) {
+        // every split's (max, sum) and row issued before any is used: one L2 round
+        // trip instead of two (same arithmetic, same order as below)
+        float2 ml[16];
+        uint4 v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < a.splits) {
+                ml[j] = a.part_ml[j * stride + row];
+                v[j] = *reinterpret_cast<const uint4 *>(src0 + (size_t)j * stride * a.D);
+            }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < a.splits) M = fmaxf(M, ml[j].x);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < a.splits) {
+                const float wl = ml[j].x == -INFINITY ? 0.f : exp2f(ml[j].x - M) * ml[j].y;
+                L += wl;
+                float f[8];
+                unpack8(v[j], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wl, f[e], acc[e]);
+            }
+    }
+    if (a.splits > 16)
+        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[s * stride + row].x);
+    for (int s0 = 0; a.splits > 16 && s0 < a.splits; s0 += 8) {
         const int ns = a.splits - s0 < 8 ? a.splits - s0 : 8;
         float2 ml[8];
         uint4 v[8];
