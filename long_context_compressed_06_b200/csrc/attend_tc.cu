@@ -174,18 +174,26 @@ CSA_DEVINL Keys query_keys(const AttendArgs &a, long long t) {
     return k;
 }
 
+// The selection index of key e as stored (loaded only: the value is consumed
+// by key_row_index, so that the load can be issued a tile ahead).
+CSA_DEVINL int key_index_raw(const AttendArgs &a, const Keys &ks, long long bq, long long e, long long e_end) {
+    if (e >= e_end) e = e_end - 1;
+    return (!a.dense && e >= 0 && e < ks.nsel) ? __ldg(a.idx + bq * a.k + e) : 0;
+}
+
 // Row of key e -- its index in kv (win == false) or in the window buffer --
 // and whether it takes part (keys past e_end, selection padding and
-// out-of-range indices read a valid row; their scores are masked).
-CSA_DEVINL size_t key_row_index(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
-                                long long e_end, bool &valid, bool &win) {
+// out-of-range indices read a valid row; their scores are masked).  jraw is
+// key_index_raw(e).
+CSA_DEVINL size_t key_row_index(const AttendArgs &a, const Keys &ks, long long b, long long e, long long e_end,
+                                int jraw, bool &valid, bool &win) {
     win = false;
     valid = e < e_end;
     if (!valid) e = e_end - 1;  // e_end >= 1 whenever a tile exists
     if (e < ks.nsel4) {
         long long j = 0;
         if (e < ks.nsel) {
-            j = a.dense ? e : (long long)__ldg(a.idx + bq * a.k + e);
+            j = a.dense ? e : (long long)jraw;
             if (j < 0 || j >= a.N) {
                 j = 0;
                 valid = false;
@@ -203,18 +211,18 @@ CSA_DEVINL size_t key_row_index(const AttendArgs &a, const Keys &ks, long long b
     return (size_t)b * a.win_rows + (ks.u0 - a.win_pos0) + w;
 }
 
-CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
-                                    long long e_end, bool &valid) {
+CSA_DEVINL const uint16_t *key_slot(const AttendArgs &a, const Keys &ks, long long b, long long e, long long e_end,
+                                    int jraw, bool &valid) {
     bool win;
-    const size_t r = key_row_index(a, ks, b, bq, e, e_end, valid, win);
+    const size_t r = key_row_index(a, ks, b, e, e_end, jraw, valid, win);
     return (win ? a.win : a.kv) + r * a.D;
 }
 
 // FP8 rows: the codes of key e (the row's exponent bytes follow from the same index)
-CSA_DEVINL const uint8_t *key_slot8(const AttendArgs &a, const Keys &ks, long long b, long long bq, long long e,
-                                    long long e_end, bool &valid, const uint8_t *&exps) {
+CSA_DEVINL const uint8_t *key_slot8(const AttendArgs &a, const Keys &ks, long long b, long long e, long long e_end,
+                                    int jraw, bool &valid, const uint8_t *&exps) {
     bool win;
-    const size_t r = key_row_index(a, ks, b, bq, e, e_end, valid, win);
+    const size_t r = key_row_index(a, ks, b, e, e_end, jraw, valid, win);
     exps = (win ? a.win8e : a.kv8e) + r * (a.D / 128);
     return (win ? a.win8 : a.kv8) + r * a.D;
 }
@@ -424,19 +432,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("griddepcontrol.wait;" ::: "memory");
                 dep_done = true;
             }
+            // Row pointers of the tile's 64 keys, two per lane.  The selection
+            // indices of tile j + 1 are loaded while tile j is issued (an L2 round
+            // trip that would otherwise separate the tiles' gathers); only the next
+            // iteration uses them.
+            int nraw0 = 0, nraw1 = 0;
+            if (it.ntiles > 0) {
+                nraw0 = key_index_raw(a, it.ks, it.bq, it.e0 + lane, it.e1);
+                nraw1 = key_index_raw(a, it.ks, it.bq, it.e0 + 32 + lane, it.e1);
+            }
             for (int j = 0; j < it.ntiles; ++j) {
                 const long long g = jt + j;
                 const int st = (int)(g % p.stages);
                 const long long ebase = it.e0 + (long long)j * kTileKeys;
+                const int raw0 = nraw0, raw1 = nraw1;
+                if (j + 1 < it.ntiles) {
+                    nraw0 = key_index_raw(a, it.ks, it.bq, ebase + kTileKeys + lane, it.e1);
+                    nraw1 = key_index_raw(a, it.ks, it.bq, ebase + kTileKeys + 32 + lane, it.e1);
+                }
                 bool v0, v1;
                 const uint16_t *r0 = nullptr, *r1 = nullptr;
                 const uint8_t *c0 = nullptr, *c1 = nullptr, *x0 = nullptr, *x1 = nullptr;
                 if constexpr (FP8) {
-                    c0 = key_slot8(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0, x0);
-                    c1 = key_slot8(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1, x1);
+                    c0 = key_slot8(a, it.ks, it.b, ebase + lane, it.e1, raw0, v0, x0);
+                    c1 = key_slot8(a, it.ks, it.b, ebase + 32 + lane, it.e1, raw1, v1, x1);
                 } else {
-                    r0 = key_slot(a, it.ks, it.b, it.bq, ebase + lane, it.e1, v0);
-                    r1 = key_slot(a, it.ks, it.b, it.bq, ebase + 32 + lane, it.e1, v1);
+                    r0 = key_slot(a, it.ks, it.b, ebase + lane, it.e1, raw0, v0);
+                    r1 = key_slot(a, it.ks, it.b, ebase + 32 + lane, it.e1, raw1, v1);
                 }
                 const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
                 if (!warp_wait(smem_u32(s.kempty + st), (uint32_t)(((g / p.stages) & 1) ^ 1), p.ctx, s.abort_flag)) {
