@@ -22,9 +22,10 @@
 // no exchange; each streams the gathered rows itself (the second read of a
 // row is an L2 hit).
 //
-// Warp roles (256 threads): warp 0 TMEM owner, TMA loader of each work
-// item's raw query rows and MMA issuer (lane 0 issues through guarded
-// instructions); warps 1..3 gather the key rows with 16-byte cp.async into
+// Warp roles (352 threads): warp 0 TMEM owner, TMA loader of each work
+// item's raw query rows and, with warp 8, MMA issuer (lane 0 issues through
+// guarded instructions; each issuer takes half of every product); warps 1..3
+// and 9..10 gather the key rows with 16-byte cp.async into
 // the 128-byte swizzled layout (one 512-byte coalesced row segment per warp
 // instruction; HCA tiles of consecutive entries arrive as TMA tiles instead)
 // from kernel entry on, each tile's key-validity mask travelling with it;
@@ -50,11 +51,15 @@ namespace csa {
 namespace {
 
 constexpr int kMma2Warp = 8;   // the second MMA issuer
-constexpr int kThreads = 288;
+constexpr int kThreads = 352;  // warp 0 and 8: MMA; 1-3 and 9-10: gathers; 4-7: softmax
 constexpr int kTileKeys = 64;
 constexpr int kHeads = 64;          // heads per CTA (M of every MMA)
 constexpr int kSoftmaxWarp0 = 4;
-constexpr int kProducerWarp0 = 1, kProducerWarps = 3;
+// gather warps 1, 2, 3, 9, 10 (five: issuing a tile's 4096 16-byte copies took ~0.8 us
+// with three, on the critical path between a stage's release and its next tile)
+constexpr int kProducerWarps = 5;
+CSA_DEVINL bool is_producer_warp(int w) { return (w >= 1 && w < 4) || w >= 9; }
+CSA_DEVINL int producer_index(int w) { return w < 4 ? w - 1 : w - 6; }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxStages = 4;
 
@@ -413,12 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P.V g-2 is known complete (the P buffer it read was released before P_g
     // was written).  jt counts the tiles this CTA has processed, identically in
     // every role.
-    if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
+    if (is_producer_warp(warp)) {
         // ------------------------------------------------------------ producers (cp.async gather)
         // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l, l+32,
         // .. of the row (coalesced 512 B per instruction).  Row pointers of the
         // tile's 64 keys are computed once per tile, two per lane.
-        const int pw = warp - kProducerWarp0;
+        const int pw = producer_index(warp);
         long long jt = 0;
         bool ok = true;
         bool dep_done = false;
