@@ -444,7 +444,7 @@ def e2e_csa_decode(csa, states, args, device, world, rank):
     del graphs
     return {"value": job_rate(wl.batch * wl.nq, args.steps, world, t_max), "unit": "queries/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "method": "every step: H2D of its inputs from pinned memory, csa_index -> csa_topk -> csa_attend, "
+            "method": "every step: H2D of its inputs from pinned memory, csa_decode_step (csa_index -> csa_topk -> csa_attend), "
                       "D2H of the output, captured once per decode state in a CUDA graph; %d states rotate on "
                       "%d streams (inputs exceed L2, no flush), so copies overlap neighbouring steps"
                       % (E2E_STATES, E2E_STATES)}
