@@ -97,8 +97,8 @@ struct Ring {
     }
 };
 
-template <int EW>  // warps per epilogue group: 4 (one per TMEM lane quarter) or 8 (two)
-__global__ void __launch_bounds__(64 + 64 * EW, 1)
+template <int EW, int OCC>  // warps per epilogue group (4: one per TMEM lane quarter, 8: two); CTAs per SM
+__global__ void __launch_bounds__(64 + 64 * EW, OCC)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const IndexTcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(64 + 64 * EW, 1)
         // Two groups of EW warps take alternate tiles (tile i -> group i & 1,
         // accumulator i % n_acc), doubling the epilogue rate; with EW = 8 the two
         // warps of a lane quarter take the even and the odd queries of a tile.
-        constexpr int kLoads = EW == 4 ? 4 : 2;  // 16-column TMEM loads per wait (registers)
+        constexpr int kLoads = (EW == 4 && OCC == 1) ? 4 : 2;  // 16-column TMEM loads per wait (registers)
         const int eg = (warp - 2) / EW;
         const int half = ((warp - 2) % EW) >> 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -331,7 +331,12 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
     p.NQ = NQ;
     p.n_cols = NQ * p.H_pad;
     p.q_bytes = (uint32_t)(p.n_cols * d_I * 2);
-    p.stages = (int)std::min<size_t>(kMaxStages, (smem_cap - p.q_bytes) / p.stage_bytes);
+    // One query per tile (decode): two CTAs per SM, two stages each -- finer work
+    // ranges and two independent pipelines per SM even out the CTAs' finishing
+    // times (decode 128K: 21.0 -> 18.6 us).
+    const bool two_per_sm = NQ == 1 && (size_t)p.q_bytes + 2 * (size_t)p.stage_bytes + 4096 <= 108 * 1024;
+    const size_t cta_cap = two_per_sm ? 108 * 1024 : smem_cap;
+    p.stages = (int)std::min<size_t>(kMaxStages, (cta_cap - p.q_bytes) / p.stage_bytes);
     if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
     p.idesc = tc::idesc_f16(p.n_cols, true);
     p.n_acc = p.n_cols <= 128 ? 4 : 2;
@@ -363,10 +368,10 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
     // several queries per tile: two warps per TMEM lane quarter split them
     const int EW = NQ >= 2 ? 8 : 4;
     void (*kern)(const CUtensorMap, const CUtensorMap, const IndexTcParams) =
-        EW == 8 ? index_tc_kernel<8> : index_tc_kernel<4>;
+        EW == 8 ? index_tc_kernel<8, 1> : (two_per_sm ? index_tc_kernel<4, 2> : index_tc_kernel<4, 1>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
-    const int grid = (int)std::min<long long>(p.total_work, num_sms());
+    const int grid = (int)std::min<long long>(p.total_work, (two_per_sm ? 2 : 1) * num_sms());
     kern<<<grid, 64 + 64 * EW, smem, st>>>(kmap, qmap, p);
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
