@@ -55,10 +55,13 @@ CSA_DEVINL float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Inclusive scan over the 1024 threads of the block; returns this thread's
-// inclusive prefix and writes the block total to *total.
+// Inclusive scan over the 1024 threads (32 warps) of the block; returns this
+// thread's inclusive prefix and writes the block total to *total.  One block
+// barrier: every warp scans the 32 warp totals itself.  The caller places a
+// block barrier between this scan and the next write of warp_buf.
 template <typename T>
 CSA_DEVINL T block_scan_incl(T v, T *warp_buf, T *total) {
+    static_assert(kTopkThreads == 1024, "one warp total per lane");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -67,21 +70,15 @@ CSA_DEVINL T block_scan_incl(T v, T *warp_buf, T *total) {
     }
     if (lane == 31) warp_buf[warp] = v;
     __syncthreads();
-    if (warp == 0) {
-        T w = warp_buf[lane];
+    T w = warp_buf[lane];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const T n = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += n;
-        }
-        warp_buf[lane] = w;  // inclusive over warps
+    for (int o = 1; o < 32; o <<= 1) {
+        const T n = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += n;
     }
-    __syncthreads();
-    if (warp > 0) v += warp_buf[warp - 1];
-    const T tot = warp_buf[31];
-    __syncthreads();  // warp_buf is reused by the next scan
-    *total = tot;
-    return v;
+    const T before = __shfl_sync(0xffffffffu, w, (warp + 31) & 31);  // warps below this one
+    *total = __shfl_sync(0xffffffffu, w, 31);
+    return warp > 0 ? v + before : v;
 }
 
 // Value-linear digit of a key: floor((v - vmin) * scale), capped at the last bin.
@@ -150,7 +147,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
 #pragma unroll
         for (int r = 0; r < R; ++r) key[r] = r < nrow ? order_key(__ldg(row + seg0 + r)) : 0u;
     }
-    const long long nv = q_pos ? n_visible(t_q, m, N) : N;  // no q_pos: every entry is eligible
+    // visible entries floor((t + 1) / m) clipped to [0, N] (no q_pos: every entry), in 32-bit arithmetic
+    long long nv = N;
+    if (q_pos) {
+        const long long v = t_q < 0 ? 0 : (long long)(((uint32_t)t_q + 1u) / (uint32_t)m);
+        nv = v < N ? v : N;
+    }
     const long long kk = nv < k ? nv : k;
     const int nloc = (int)(nv - seg0 <= 0 ? 0 : (nv - seg0 >= R ? R : nv - seg0));
 
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
             vmin = key_value(gmin);
             const float vmax = key_value(gmax);
             const float range = __fsub_rn(vmax, vmin);
-            lscale = __fdiv_rn((float)kLinBins, range);
+            lscale = __fdividef((float)kLinBins, range);  // any value: every thread computes the same
             // Only with few keys per thread (their digits then stay in registers):
             // at 16 or 32 keys per thread the radix passes measured faster
             // (prefill rows 0.28 vs 0.37 ms, 262144-entry rows 29 vs 45 us).
@@ -270,12 +272,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         sync_all();  // every CTA's histogram is complete
         // cluster-wide count of bin threadIdx.x (one bin per thread)
         uint32_t c = 0u;
-        for (int r0 = 0; r0 < CS; r0 += 4) {
-            uint32_t v[4];
+        for (int r0 = 0; r0 < CS; r0 += 8) {
+            uint32_t v[8];  // up to eight ranks' loads in flight
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = r0 + j < CS ? *peer(&hist[0][threadIdx.x], r0 + j) : 0u;
+            for (int j = 0; j < 8; ++j) v[j] = r0 + j < CS ? *peer(&hist[0][threadIdx.x], r0 + j) : 0u;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) c += v[j];
+            for (int j = 0; j < 8; ++j) c += v[j];
         }
         uint32_t tot;
         const uint32_t incl = block_scan_incl<uint32_t>(c, warp_u32, &tot);
@@ -305,21 +307,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
                 n_above += d > t1;
                 n_in += d == t1;
             }
-        unsigned long long blk_tot;
-        const unsigned long long mine = ((unsigned long long)n_above << 32) | n_in;
-        const unsigned long long excl = block_scan_incl<unsigned long long>(mine, warp_u64, &blk_tot) - mine;
+        // (above << 16) | in-bin: a CTA holds at most 1024 * 8 keys on this path
+        uint32_t blk_tot;
+        const uint32_t mine = (n_above << 16) | n_in;
+        const uint32_t excl = block_scan_incl<uint32_t>(mine, warp_u32, &blk_tot) - mine;
         // this CTA's candidates into its segment of every rank's list, in index order
-        uint32_t cp = (uint32_t)excl;
+        uint32_t cp = excl & 0xffffu;
 #pragma unroll
         for (int r = 0; r < R; ++r)
             if (r < nloc && digit(r) == t1) {
                 for (int r2 = 0; r2 < CS; ++r2) *peer(&seg_key[rank][cp], r2) = key[r];
                 ++cp;
             }
-        if ((int)threadIdx.x < CS) *peer(&r_tot[rank], (int)threadIdx.x) = blk_tot;
+        if ((int)threadIdx.x < CS)
+            *peer(&r_tot[rank], (int)threadIdx.x) = ((unsigned long long)(blk_tot >> 16) << 32) | (blk_tot & 0xffffu);
         // every rank's candidates and counts delivered; from here on no CTA
         // touches another's shared memory, so none waits for the others to exit
         sync_all();
+        // the candidate count, the same in every CTA
+        uint32_t C = 0u;
+        for (int r2 = 0; r2 < CS; ++r2) C += (uint32_t)r_tot[r2];
         if (warp == 0) {
             // prefix over ranks of the (above, in-bin) counts: list offsets, and the
             // keys above the bin in lower ranks (this rank's first output slot)
@@ -333,55 +340,80 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
             if (lane < CS) s_off[lane] = (uint32_t)(inc - t);
             if (lane == CS - 1) s_off[CS] = (uint32_t)inc;
             if (lane == rank) s_above_before = (long long)((inc - t) >> 32);
-        }
-        __syncthreads();
-        const int C = (int)s_off[CS];
-        for (int i = threadIdx.x; i < C; i += kTopkThreads) {
-            int r2 = 0;
-            while (r2 + 1 < CS && s_off[r2 + 1] <= (uint32_t)i) ++r2;
-            all_key[i] = seg_key[r2][i - (int)s_off[r2]];
-        }
-        __syncthreads();
-        {
-            // candidates preceding candidate i in (score desc, index asc), counted
-            // over four slices of the list by four threads
-            constexpr int kParts = kTopkThreads / kCandCap;
-            const int i = threadIdx.x % kCandCap, part = threadIdx.x / kCandCap;
-            if (i < C) {
-                const int chunk = (C + kParts - 1) / kParts;
-                const int j0 = part * chunk, j1 = min(C, j0 + chunk);
-                const uint32_t ki = all_key[i];
-                uint32_t cnt = 0u;
-                for (int j = j0; j < j1; ++j) {
-                    const uint32_t kj = all_key[j];
-                    cnt += (kj > ki) || (kj == ki && j < i);
+            if (C <= 32u) {
+                // up to 32 candidates: one warp gathers, ranks and counts them
+                __syncwarp();
+                // candidate `lane` lies in the segment of the last rank whose offset is <= lane
+                const uint32_t my_off = (uint32_t)(inc - t);
+                int r2 = 0;
+#pragma unroll
+                for (int j = 1; j < kMaxCluster; ++j) {
+                    const uint32_t off_j = __shfl_sync(0xffffffffu, my_off, j);
+                    r2 += j < CS && off_j <= (uint32_t)lane;
                 }
-                rank_part[part][i] = cnt;
+                const int seg_start = (int)__shfl_sync(0xffffffffu, my_off, r2);  // every lane takes part
+                const uint32_t ki = (uint32_t)lane < C ? seg_key[r2][lane - seg_start] : 0u;
+                uint32_t rk = 0u;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t kj = __shfl_sync(0xffffffffu, ki, j);
+                    rk += j < (int)C && ((kj > ki) || (kj == ki && j < lane));
+                }
+                const uint32_t selb = __ballot_sync(0xffffffffu, (uint32_t)lane < C && (long long)rk < krem);
+                if ((uint32_t)lane < C) sel_pre[lane + 1] = __popc(selb & (0xffffffffu >> (31 - lane)));
+                if (lane == 0) sel_pre[0] = 0u;
             }
         }
         __syncthreads();
-        uint32_t sel = 0u;
-        if ((int)threadIdx.x < C) {
-            uint32_t rk = 0u;
+        if (C > 32u) {
+            for (int i = threadIdx.x; i < (int)C; i += kTopkThreads) {
+                int r2 = 0;
+                while (r2 + 1 < CS && s_off[r2 + 1] <= (uint32_t)i) ++r2;
+                all_key[i] = seg_key[r2][i - (int)s_off[r2]];
+            }
+            __syncthreads();
+            {
+                // candidates preceding candidate i in (score desc, index asc), counted
+                // over four slices of the list by four threads
+                constexpr int kParts = kTopkThreads / kCandCap;
+                const int i = threadIdx.x % kCandCap, part = threadIdx.x / kCandCap;
+                if (i < (int)C) {
+                    const int chunk = ((int)C + kParts - 1) / kParts;
+                    const int j0 = part * chunk, j1 = min((int)C, j0 + chunk);
+                    const uint32_t ki = all_key[i];
+                    uint32_t cnt = 0u;
+                    for (int j = j0; j < j1; ++j) {
+                        const uint32_t kj = all_key[j];
+                        cnt += (kj > ki) || (kj == ki && j < i);
+                    }
+                    rank_part[part][i] = cnt;
+                }
+            }
+            __syncthreads();
+            uint32_t sel = 0u;
+            if ((int)threadIdx.x < (int)C) {
+                uint32_t rk = 0u;
 #pragma unroll
-            for (int q = 0; q < kTopkThreads / kCandCap; ++q) rk += rank_part[q][threadIdx.x];
-            sel = (long long)rk < krem;
+                for (int q = 0; q < kTopkThreads / kCandCap; ++q) rk += rank_part[q][threadIdx.x];
+                sel = (long long)rk < krem;
+            }
+            uint32_t sel_tot;
+            const uint32_t sel_incl = block_scan_incl<uint32_t>(sel, warp_u32, &sel_tot);
+            if ((int)threadIdx.x < (int)C) sel_pre[threadIdx.x + 1] = sel_incl;
+            if (threadIdx.x == 0) sel_pre[0] = 0u;
+            __syncthreads();
         }
-        uint32_t sel_tot;
-        const uint32_t sel_incl = block_scan_incl<uint32_t>(sel, warp_u32, &sel_tot);
-        if ((int)threadIdx.x < C) sel_pre[threadIdx.x + 1] = sel_incl;
-        if (threadIdx.x == 0) sel_pre[0] = 0u;
-        __syncthreads();
         // outputs in index order: keys above the threshold bin and selected candidates
-        uint32_t ci = s_off[rank] + (uint32_t)excl;
-        long long pos = s_above_before + (long long)(excl >> 32) + sel_pre[ci];
+        uint32_t ci = s_off[rank] + (excl & 0xffffu);
+        int pos = (int)s_above_before + (int)(excl >> 16) + (int)sel_pre[ci];
+        const int kk32 = (int)kk;
 #pragma unroll
         for (int r = 0; r < R; ++r)
             if (r < nloc) {
                 const int d = digit(r);
                 // pos < kk by construction (kk - krem keys above the bin, krem selected in it)
                 if (d > t1 || (d == t1 && sel_pre[ci + 1] != sel_pre[ci])) {
-                    if (pos < kk) out[pos] = (int)(seg0 + r);
+                    if (pos < kk32) out[pos] = (int)(seg0 + r);
                     ++pos;
                 }
                 ci += d == t1;
@@ -466,10 +498,10 @@ TopkPlan plan(long long n_queries, long long N) {
     int R = 4;
     while ((long long)R * CS < need) R *= 2;
     // Spread small batches over more SMs: measured on the 8-query decode batch
-    // at 32768 entries, clusters of 4 (8 keys per thread) take 13.7 us per
-    // launch against 19.9 us for one CTA per query (32 keys per thread), and
-    // beat clusters of 2 and 8.
-    while (n_queries * CS < 148 && CS < 4 && R > 4) {
+    // at 32768 entries, clusters of 8 (4 keys per thread) take 10.4 us per
+    // launch against 12.4 us for clusters of 4 (8 keys per thread) and 19.9 us
+    // for one CTA per query (32 keys per thread).
+    while (n_queries * CS < 148 && CS < 8 && R > 4) {
         CS *= 2;
         R /= 2;
     }

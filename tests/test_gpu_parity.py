@@ -251,6 +251,8 @@ def test_topk_exact_on_identical_scores(cuda, batch, nq, N, m, k, ts, levels):
 
 @pytest.mark.parametrize("batch,nq,N,k,mode", [
     (8, 1, 32768, 1024, "threshold_ties"),   # ties inside the threshold bin (ranked directly)
+    (4, 1, 32768, 1024, "crowded_bin"),      # 33..256 keys in the threshold bin (block-wide ranking)
+    (2, 1, 65536, 2048, "crowded_bin"),
     (2, 1, 32768, 1024, "outlier"),          # one huge score: linear bins collapse, radix passes
     (2, 1, 4096, 256, "neg_inf"),            # -inf among the visible scores
     (2, 80, 16384, 1024, "normal"),          # one CTA per query (many queries)
@@ -268,6 +270,14 @@ def test_topk_exact_value_cases(cuda, batch, nq, N, k, mode):
         for q in np.ndindex(batch, nq):
             kth = np.sort(s[q])[-k]
             s[q][r.choice(N, 6, replace=False)] = kth      # six more copies of the k-th largest score
+    elif mode == "crowded_bin":
+        for q in np.ndindex(batch, nq):
+            kth = np.sort(s[q])[-k]
+            pick = r.choice(N, 100, replace=False)
+            # distinct scores within 1e-3 of the k-th largest (one value-linear bin spans ~8e-3),
+            # every fifth an exact copy of it
+            s[q][pick] = (kth + r.uniform(-1e-3, 1e-3, 100)).astype(np.float32)
+            s[q][pick[::5]] = kth
     elif mode == "outlier":
         s[:, :, 100] = 1e30
     elif mode == "neg_inf":
