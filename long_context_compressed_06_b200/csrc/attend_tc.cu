@@ -427,6 +427,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         long long jt = 0;
         bool ok = true;
         bool dep_done = false;
+        // FP8 rows: a tile's codes are copied (cp.async) into its stage as they
+        // are stored -- the 64 codes of a key's 64-dimension chunk in the first
+        // half of the 128-byte row that chunk's bf16 values will fill -- and
+        // expanded in place once the next tile's copies are issued, so that the
+        // copies of one tile overlap the conversion of the other.  f8_st is the
+        // stage waiting for its conversion (-1: none), with its key mask and this
+        // lane's block exponent of every key the warp copies.
+        constexpr int kKeysPerWarp = (kTileKeys + kProducerWarps - 1) / kProducerWarps;
+        int f8_st = -1;
+        uint64_t f8_mask = 0;
+        uint32_t f8_e[kKeysPerWarp];
+#pragma unroll
+        for (int i = 0; i < kKeysPerWarp; ++i) f8_e[i] = 0u;
+        // expands the codes of stage f8_st (after the copies of this thread are
+        // complete up to the newest `newer` groups) and marks the tile full
+        const auto f8_convert = [&](bool newer) {
+            if constexpr (FP8) {
+                if (newer) asm volatile("cp.async.wait_group 1;" ::: "memory");
+                else asm volatile("cp.async.wait_group 0;" ::: "memory");
+                __syncwarp();
+                const uint32_t stage = smem_u32(s.k + (size_t)f8_st * Lt::kStageBytes);
+                // keys in batches of kBatch: their codes read, then (after every lane has
+                // read its own) the rows overwritten with the bf16 values
+                constexpr int kBatch = 4;
+#pragma unroll
+                for (int i0 = 0; i0 < kKeysPerWarp; i0 += kBatch) {
+                    uint4 c[kBatch];
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) {
+                        const int key = pw + kProducerWarps * (i0 + j);
+                        c[j] = make_uint4(0u, 0u, 0u, 0u);
+                        // lane l holds codes 16l..16l+15: chunk l / 4, bytes 16 (l % 4).. of its row
+                        if (i0 + j < kKeysPerWarp && key < kTileKeys && lane < D / 16)
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(c[j].x), "=r"(c[j].y), "=r"(c[j].z), "=r"(c[j].w)
+                                         : "r"(stage + (lane >> 2) * (kTileKeys * 128) + key * 128 + (lane & 3) * 16));
+                    }
+                    __syncwarp();  // every lane has its codes before any lane overwrites the rows
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) {
+                        const int key = pw + kProducerWarps * (i0 + j);
+                        if (i0 + j < kKeysPerWarp && key < kTileKeys && lane < D / 16) {
+                            const uint32_t row = stage + (lane >> 2) * (kTileKeys * 128) + key * 128;
+                            const uint4 lo = e4m3x8_bf16x8(make_uint2(c[j].x, c[j].y), f8_e[i0 + j]);
+                            const uint4 hi = e4m3x8_bf16x8(make_uint2(c[j].z, c[j].w), f8_e[i0 + j]);
+                            const int u0 = (lane & 3) * 2;  // the 16-byte units of these 16 values
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((u0 ^ (key & 7)) << 4)),
+                                         "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                         : "memory");
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                         ::"r"(row + (((u0 + 1) ^ (key & 7)) << 4)), "r"(hi.x), "r"(hi.y), "r"(hi.z),
+                                         "r"(hi.w)
+                                         : "memory");
+                        }
+                    }
+                }
+                tc::fence_proxy_async_smem();  // the generic stores before the MMA's reads
+                mbar_arrive(smem_u32(s.kfull + f8_st));
+                if (pw == 0) {  // the mask travels with the tile (release by lane 0's arrive)
+                    if (lane == 0) s.kmask[f8_st] = f8_mask;
+                    mbar_arrive(smem_u32(s.kfull + f8_st), lane == 0);
+                }
+                f8_st = -1;
+            }
+        };
         for (long long wi = blockIdx.x; wi < p.n_work && ok; wi += gridDim.x) {
             const Item it = work_item(p, wi);
             // As a programmatic dependent (csa_decode_step) the selection is
@@ -488,32 +553,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 if constexpr (FP8) {
-                    // FP8 rows: lane l converts the 8 codes of each of its 16-byte output units
-                    // (8 bytes in, 8 bf16 out) and stores them where cp.async would have put the
-                    // bf16 row; the async-proxy fence orders the stores before the MMA reads them.
-#pragma unroll 2
-                    for (int key = pw; key < kTileKeys; key += kProducerWarps) {
-                        const uint8_t *crow = reinterpret_cast<const uint8_t *>(
-                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? c0 : c1), key & 31));
-                        const uint8_t *xrow = reinterpret_cast<const uint8_t *>(
-                            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? x0 : x1), key & 31));
-                        const uint32_t krow = stage + key * 128;
+                    // this tile's codes and block exponents in flight, then the previous
+                    // tile's expansion
+                    uint32_t e_new[kKeysPerWarp];
 #pragma unroll
-                        for (int u = lane; u < D / 8; u += 32) {
-                            const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(crow + u * 8));
-                            const uint4 v = e4m3x8_bf16x8(raw, __ldg(xrow + (u >> 4)));
-                            const uint32_t dst = krow + (u >> 3) * (kTileKeys * 128) + (((u & 7) ^ (key & 7)) << 4);
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
-                                         "r"(v.z), "r"(v.w)
-                                         : "memory");
+                    for (int i = 0; i < kKeysPerWarp; ++i) {
+                        const int key = pw + kProducerWarps * i;
+                        e_new[i] = 0u;
+                        if (key < kTileKeys) {
+                            const uint8_t *crow = reinterpret_cast<const uint8_t *>(
+                                __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? c0 : c1), key & 31));
+                            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(
+                                __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(key < 32 ? x0 : x1), key & 31));
+                            if (lane < D / 16) {
+                                const uint32_t dst = stage + (lane >> 2) * (kTileKeys * 128) + key * 128 + (lane & 3) * 16;
+                                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(crow + lane * 16)
+                                             : "memory");
+                                e_new[i] = __ldg(xrow + (lane >> 3));  // the block of 128 codes holding 16l..16l+15
+                            }
                         }
                     }
-                    tc::fence_proxy_async_smem();
-                    mbar_arrive(smem_u32(s.kfull + st));
-                    if (pw == 0) {  // the mask travels with the tile (release by lane 0's arrive)
-                        if (lane == 0) s.kmask[st] = ((uint64_t)mhi << 32) | mlo;
-                        mbar_arrive(smem_u32(s.kfull + st), lane == 0);
-                    }
+                    asm volatile("cp.async.commit_group;" ::: "memory");
+                    if (f8_st >= 0) f8_convert(true);
+                    f8_st = st;
+                    f8_mask = ((uint64_t)mhi << 32) | mlo;
+#pragma unroll
+                    for (int i = 0; i < kKeysPerWarp; ++i) f8_e[i] = e_new[i];
                 } else {
                     // Each warp copies keys pw, pw+3, ...: lane l moves 16-byte units l,
                     // l+32, .. of the row (coalesced 512 B per instruction).
@@ -539,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             jt += it.ntiles;
         }
+        if (ok && f8_st >= 0) f8_convert(false);  // the last tile's expansion
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 0 || warp == kMma2Warp) {
         // ------------------------------------------------------------ MMA issuers
