@@ -6,7 +6,7 @@ query per sequence at position 131071, m = 4 (32768 compressed entries), 64x128
 indexer, top-k 1024, 128 heads x 512, window 128.  A step is one pass of the
 decode hot path over the resident cache: csa_decode_step, i.e. csa_index ->
 csa_topk -> csa_attend (+ split combine) with the top-k and attention kernels
-launched as programmatic dependents, replayed as a CUDA graph per decode state.  Six decode
+launched as programmatic dependents; the K timed steps are one CUDA graph.  Six decode
 states rotate (each has 79 MB of step inputs; 5 x 79 MB pass through the
 126 MB L2 between two uses of one state), so no step finds its inputs in L2
 and no flush is needed between steps.
@@ -274,31 +274,32 @@ DEVICE_STATES = 6
 
 
 def bench_csa_decode(csa, args, device, world, rank, peaks):
-    """The headline: the 128K decode step, one CUDA graph per decode state.
-    DEVICE_STATES states (each 79 MB of step inputs, together more than the
-    126 MB L2) rotate, so every step reads its keys and rows from HBM without
-    an L2 flush between steps (a write flush would leave dirty lines whose
-    write-back shares DRAM with the step).  The K timed steps run back to back
-    between two events on the launch stream."""
+    """The headline: the 128K decode step.  The K timed steps are captured in
+    one CUDA graph (as consecutive attention layers of a decode forward would
+    be), each step complete before the next starts, and replayed once between
+    two events on the launch stream.  DEVICE_STATES states (each 79 MB of step
+    inputs, together more than the 126 MB L2) rotate, so every step reads its
+    keys and rows from HBM without an L2 flush between steps (a write flush
+    would leave dirty lines whose write-back shares DRAM with the step)."""
     wl = W.CSA_DECODE
     states = [decode_cache_state(csa, wl, device, rank_seed(0 if i == 0 else 101 + i, rank))
               for i in range(DEVICE_STATES)]
     st = states[0]
-    graphs = []
     for S in states:
         decode_step(csa, S)  # eager first (lazy initialisation outside the capture)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            decode_step(csa, S)
-        graphs.append(g)
     torch.cuda.synchronize()
 
-    def replay(n, first):
-        for i in range(first, first + n):
-            graphs[i % len(graphs)].replay()
+    def capture(n, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(first, first + n):
+                decode_step(csa, states[i % len(states)])
+        return g
 
-    replay(args.warmup, 0)
+    g_warm, g_timed = capture(args.warmup, 0), capture(args.steps, args.warmup)
+    graphs = [g_warm, g_timed]
+    torch.cuda.synchronize()
+    g_warm.replay()
     torch.cuda.synchronize()
     barrier(world)
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -306,21 +307,21 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
         torch.cuda._sleep(2_000_000)  # lets the host enqueue ahead of the GPU (outside the events)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        replay(args.steps, args.warmup)
+        g_timed.replay()
         e1.record()
         torch.cuda.synchronize()
         t_graph = e0.elapsed_time(e1) / 1e3
         # keep the GPU under the same load until the sampler has seen >= 1 s of it
         while time.perf_counter() - t0 < 1.5:
-            replay(50, 0)
+            for _ in range(5):
+                g_timed.replay()
             torch.cuda.synchronize()
     torch.cuda.synchronize()
     barrier(world)
     t_max = max_over_ranks(t_graph, world, device)
     value = job_rate(wl.batch * wl.nq, args.steps, world, t_max)
-    # per-kernel breakdown: each kernel of the step captured alone in a graph per
-    # decode state; K back-to-back replays over the same rotation between two
-    # events on the launch stream (no host launch gaps inside the interval)
+    # per-kernel breakdown: each kernel of the step launched n times over the
+    # rotation inside one graph, between two events on the launch stream
     seg = kernel_breakdown(csa, states, args)
     t_index = seg[0]
     idx_bytes = index_bytes(wl)
@@ -332,7 +333,7 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
             "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": round(t_index * 1e3, 4)}
     step_bytes = decode_step_bytes(wl)
     step_s = t_max / args.steps
-    del graphs
+    del graphs, g_warm, g_timed
     e2e = e2e_csa_decode(csa, states, args, device, world, rank)
     return dict(value=value, ms_per_step=step_s * 1e3, roofline=roof, clocks=clk.summary(), e2e=e2e,
                 launches=st["launches"] * args.steps,
@@ -345,40 +346,40 @@ def bench_csa_decode(csa, args, device, world, rank, peaks):
 
 def kernel_breakdown(csa, states, args):
     """Seconds per launch of csa_index, csa_topk and csa_attend (+ its split
-    combine) in the decode step: each captured alone per decode state and
-    replayed back to back over the rotation, timed by events around the run."""
-    parts = []
-    for S in states:
-        wl = S["wl"]
-        gs = []
-        for k in range(3):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                if k == 0:
-                    csa.csa_index(S["qI"], S["w"], S["kI"], S["qp"], wl.m, scores=S["S"])
-                elif k == 1:
-                    csa.csa_topk(S["S"], S["qp"], wl.m, wl.k, idx=S["idx"])
-                else:
-                    csa.csa_attend(S["q"], S["C"], S["idx"], S.get("win", S.get("A")), S["qp"], wl.W, wl.scale,
-                                   wl.eps, out=S["out"], workspace=S["ws"], win_pos0=S.get("win_pos0", 0))
-            gs.append(g)
-        parts.append(gs)
-    torch.cuda.synchronize()
-    seg = []
+    combine) in the decode step: n launches of one kernel, cycling over the
+    decode states (inputs larger than L2), captured in one graph and timed by
+    events around its replay, so that no graph-launch gap sits between them."""
     n = max(args.steps, 6)
+    n = (n + len(states) - 1) // len(states) * len(states)
+
+    def launch(k, S):
+        wl = S["wl"]
+        if k == 0:
+            csa.csa_index(S["qI"], S["w"], S["kI"], S["qp"], wl.m, scores=S["S"])
+        elif k == 1:
+            csa.csa_topk(S["S"], S["qp"], wl.m, wl.k, idx=S["idx"])
+        else:
+            csa.csa_attend(S["q"], S["C"], S["idx"], S.get("win", S.get("A")), S["qp"], wl.W, wl.scale,
+                           wl.eps, out=S["out"], workspace=S["ws"], win_pos0=S.get("win_pos0", 0))
+
+    seg = []
     for k in range(3):
-        for i in range(args.warmup):
-            parts[i % len(parts)][k].replay()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                launch(k, states[i % len(states)])
+        torch.cuda.synchronize()
+        for i in range(max(1, args.warmup // 2)):
+            g.replay()
         torch.cuda.synchronize()
         torch.cuda._sleep(2_000_000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for i in range(n):
-            parts[i % len(parts)][k].replay()
+        g.replay()
         e1.record()
         torch.cuda.synchronize()
         seg.append(e0.elapsed_time(e1) / 1e3 / n)
-    del parts
+        del g
     return seg
 
 
@@ -432,6 +433,7 @@ def e2e_csa_decode(csa, states, args, device, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(2_000_000)  # lets the host enqueue every step ahead of the GPU (outside the events)
     e0.record(main)
     for s_ in streams:
         s_.wait_stream(main)
