@@ -12,13 +12,21 @@
 //     weights are static, so each CTA computes them once into shared memory
 //     and every element costs one FMA; one warp per entry, the whole row in
 //     registers, RMSNorm by a warp reduction;
-//   * large m (HCA, m = 128): the input-dependent compressor with no Z rows
-//     (its logits Z + bias reduce to the static logits as the bias), a thread
-//     per (entry, 8 channels) with an online softmax over the 2m rows: the
-//     weights of all d channels do not fit in shared memory, and a cluster
-//     that split the channels and exchanged the RMSNorm sums measured 1.18
-//     TB/s against this kernel's rate.
+//   * large m (HCA, m = 128): the 2m x d weights do not fit in shared memory;
+//     a small kernel writes them once per call into a stream-ordered
+//     allocation (a pool of the library that keeps its memory between calls),
+//     and a thread per (entry, 8 channels) reads them through L1
+//     (shared by the CTA's entries), one FMA per element with kStepRows rows'
+//     loads in flight; an entry's channels stay in one CTA for the RMSNorm.
+//     Entry 0 of each sequence (its A half only, other weights) runs the
+//     input-dependent compressor with no Z rows, whose logits reduce to the
+//     static ones.  That compressor alone (an online softmax per element)
+//     measured 1.43 ms on the 1M-token cache; weights recomputed per CTA in
+//     row chunks, 0.85 ms; a channel-split cluster 1.18 TB/s.
 #include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -129,6 +137,120 @@ __global__ void __launch_bounds__(256) compress_small_kernel(
     }
 }
 
+// ------------------------------------------------------------------ large m
+constexpr int kTableThreads = 256;
+constexpr int kStepRows = 8;  // rows whose loads are in flight together
+
+// Softmax weights of the 2m logits of every channel: w[j][c] (one warp per
+// channel; the lanes' partial maxima and sums are combined in a fixed order).
+__global__ void pool_weight_table_kernel(const float *__restrict__ logits, int d, int m, float *__restrict__ w) {
+    const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (c >= d) return;  // warp-uniform
+    const float *L = logits + c;
+    float mx = -INFINITY;
+    for (int j = lane; j < 2 * m; j += 32) mx = fmaxf(mx, L[(size_t)j * d]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float den = 0.f;
+    for (int j = lane; j < 2 * m; j += 32) den += expf(L[(size_t)j * d] - mx);
+    den = warp_sum(den);
+    for (int j = lane; j < 2 * m; j += 32) w[(size_t)j * d + c] = expf(L[(size_t)j * d] - mx) / den;
+}
+
+// Entries 1..N-1 of every sequence, one entry per tpe = d / 8 threads (whole
+// warps), 256 / tpe entries per CTA; every element costs one FMA with its
+// weight from the table (read through L1, shared by the CTA's entries).
+__global__ void __launch_bounds__(kTableThreads, 4) compress_table_kernel(
+    const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, const float *__restrict__ w, int batch,
+    long long T, int d, int m, int apply_rms, const float *__restrict__ gain, float eps,
+    uint16_t *__restrict__ out, long long N) {
+    __shared__ float red[kTableThreads / 32];
+    const int tpe = d >> 3;
+    const int el_n = kTableThreads / tpe;
+    const int el = threadIdx.x / tpe;
+    const int c0 = (threadIdx.x - el * tpe) * 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long per_seq = N - 1;
+    const long long e = (long long)blockIdx.x * el_n + el;
+    const bool act = e < (long long)batch * per_seq;
+    const long long b = act ? e / per_seq : 0;
+    const long long i = act ? 1 + (e - b * per_seq) : 1;
+    const uint16_t *brow = B + ((size_t)b * T + (size_t)(i - 1) * m) * d + c0;  // previous block, stream B
+    const uint16_t *arow = A + ((size_t)b * T + (size_t)i * m) * d + c0;        // this block, stream A
+    const int two_m = 2 * m;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    if (act) {
+        for (int r0 = 0; r0 < two_m; r0 += kStepRows) {
+            uint4 xv[kStepRows];
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u) {
+                const int r = r0 + u;
+                xv[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (r < two_m) xv[u] = ldg_stream(r < m ? brow + (size_t)r * d : arow + (size_t)(r - m) * d);
+            }
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u)
+                if (r0 + u < two_m) {
+                    const float *wr = w + (size_t)(r0 + u) * d + c0;
+                    float wv[8];
+                    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(wr));
+                    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(wr + 4));
+                    wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+                    wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+                    fma8(acc, wv, xv[u]);
+                }
+        }
+    }
+    // RMSNorm over the entry's d channels: its tpe threads are whole warps
+    float rn = 1.f;
+    if (apply_rms) {
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ss = fmaf(acc[q], acc[q], ss);
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        const int w0 = el * (tpe >> 5);
+        float t = 0.f;
+        for (int k = 0; k < (tpe >> 5); ++k) t += red[w0 + k];
+        rn = 1.0f / sqrtf(t / (float)d + eps);
+    }
+    if (act) {
+        float o[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q] = acc[q] * rn * ((apply_rms && gain) ? __ldg(gain + c0 + q) : 1.f);
+        *reinterpret_cast<uint4 *>(out + ((size_t)b * N + i) * d + c0) = pack8(o);
+    }
+}
+
+// Stream-ordered pool of the current device for the weight table: it keeps its
+// memory between calls (release threshold at the maximum), so that a call does
+// not map memory while its kernels are queued.
+cudaMemPool_t table_pool() {
+    static cudaMemPool_t cache[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return nullptr;
+        }
+        cache[dev] = pool;
+    }
+    return cache[dev];
+}
+
 template <int MT, int CPL>
 cudaError_t run_small(const uint16_t *A, const uint16_t *B, const float *logits, int batch, long long T,
                       int d, int m, int apply_rms, const float *gain, float eps, uint16_t *out,
@@ -166,11 +288,33 @@ int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, i
             err = run_small<0, 4>(A, B, logits, batch, T, d, m, apply_rmsnorm, gain, eps, out, N, small_smem, grid, st);
         return err == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
     }
-    // large m: the input-dependent compressor without Z rows, the logits as its
-    // bias (read as float4: 16-byte aligned)
+    // large m.  Entry 0 of every sequence: the input-dependent compressor
+    // without Z rows, the logits as its bias (read as float4: 16-byte aligned)
     if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return CSA_ERR_UNSUPPORTED;
-    return launch_compress_dynamic(A, B, nullptr, nullptr, logits, batch, T, d, m, apply_rmsnorm, gain, eps, 0, N,
-                                   N, out, st);
+    const int tpe = d / 8;
+    const bool tabled = (tpe == 32 || tpe == 64 || tpe == 128 || tpe == 256) && N > 1;
+    float *table = nullptr;
+    cudaMemPool_t pool = tabled ? table_pool() : nullptr;
+    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&table), (size_t)2 * m * d * sizeof(float), pool,
+                                         st) != cudaSuccess) {
+        cudaGetLastError();  // no table: the online-softmax kernel does every entry
+        return launch_compress_dynamic(A, B, nullptr, nullptr, logits, batch, T, d, m, apply_rmsnorm, gain, eps, 0,
+                                       N, N, out, st);
+    }
+    int rcode = launch_compress_dynamic(A, B, nullptr, nullptr, logits, batch, T, d, m, apply_rmsnorm, gain, eps, 0,
+                                        1, N, out, st);
+    if (rcode == CSA_OK) {
+        pool_weight_table_kernel<<<(d + 3) / 4, 128, 0, st>>>(logits, d, m, table);
+        const int el_n = kTableThreads / tpe;
+        const long long blocks = ((long long)batch * (N - 1) + el_n - 1) / el_n;
+        if (blocks > INT_MAX) rcode = CSA_ERR_UNSUPPORTED;
+        else
+            compress_table_kernel<<<(unsigned)blocks, kTableThreads, 0, st>>>(A, B, table, batch, T, d, m,
+                                                                               apply_rmsnorm, gain, eps, out, N);
+        if (rcode == CSA_OK && cudaGetLastError() != cudaSuccess) rcode = CSA_ERR_CUDA;
+    }
+    if (cudaFreeAsync(table, st) != cudaSuccess && rcode == CSA_OK) rcode = CSA_ERR_CUDA;
+    return rcode;
 }
 
 }  // namespace csa

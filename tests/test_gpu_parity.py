@@ -50,12 +50,14 @@ def positions(batch, nq, ts):
     (1, 2048, 64, 4, True, False),      # tiny workload shape
     (2, 1037, 512, 4, True, True),      # ragged T, V4 width
     (2, 777, 64, 3, False, False),      # odd m, no norm
-    (1, 4 * 128 + 77, 512, 128, True, False),   # HCA ratio (cluster kernel), ragged tail
+    (1, 4 * 128 + 77, 512, 128, True, False),   # HCA ratio (chunked large-m kernel), ragged tail
     (2, 300, 256, 16, True, True),
     (3, 5, 64, 4, True, False),         # N = 1
-    (1, 1000, 1024, 64, True, False),   # cluster kernel, dc = 128
-    (1, 1000, 256, 20, True, True),     # cluster kernel, m not a multiple of the row groups
-    (1, 3 * 160 + 50, 128, 160, True, False),   # cluster kernel, two row batches per entry
+    (1, 1000, 1024, 64, True, False),   # chunked large-m kernel, 8-row chunks
+    (1, 1000, 256, 20, True, True),     # chunked large-m kernel, a partial last chunk
+    (1, 3 * 160 + 50, 128, 160, True, False),   # online-softmax kernel (d = 128)
+    (2, 128 * 37 + 5, 512, 128, True, True),    # chunked large-m kernel: two sequences, a partial entry group
+    (3, 40 * 9 + 3, 1024, 40, True, False),     # chunked large-m kernel, three sequences, 8-row chunks
 ])
 def test_compress_parity(cuda, batch, T, d, m, rms, use_gain):
     A = seeded((batch, T, d), 11)
