@@ -80,9 +80,14 @@ int csa_version(void);
  *   out     [batch][floor(T/m)][d] bf16
  * Requirements: batch >= 1, T >= m >= 1, d % 8 == 0, 8 <= d <= 1024, m <= 256
  * (m > 16 or 24*m*d > 96 KiB additionally needs logits 16-byte aligned;
- * CSA_ERR_UNSUPPORTED otherwise).  Those shapes run the csa_compress_dynamic
- * kernel with no Z rows (its logits Z + bias are then these logits): results
- * agree with the small-m kernel up to fp32 rounding order.
+ * CSA_ERR_UNSUPPORTED otherwise).  Those shapes write the 2m x d softmax
+ * weights into a table taken from a memory pool of the library (stream
+ * ordered; the pool keeps its memory, 2m*d*4 bytes at most per device, between
+ * calls) and pool every entry but the first with them; entry 0 runs the
+ * csa_compress_dynamic kernel with no Z rows (its logits Z + bias are then
+ * these logits); where the pool cannot be had, and for d / 8 not in {32, 64,
+ * 128}, that kernel computes every entry.  Results agree with the small-m
+ * kernel up to fp32 rounding order.
  */
 int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,
                  int batch, long long T, int d, int m,
