@@ -29,11 +29,11 @@
 namespace csa {
 namespace {
 
-constexpr int kRows = 8;                         // rows whose loads are in flight together
+constexpr int kRows = 4;                         // rows whose loads are in flight together (three CTAs per SM)
 constexpr int kMaxThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__global__ void __launch_bounds__(kMaxThreads) compress_dynamic_kernel(
+__global__ void __launch_bounds__(kMaxThreads, 3) compress_dynamic_kernel(
     const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, const uint16_t *__restrict__ Za,
     const uint16_t *__restrict__ Zb, const float *__restrict__ bias, int batch, long long T, int d, int m,
     int apply_rms, const float *__restrict__ gain, float eps, long long i0, long long ni, long long n_out,
