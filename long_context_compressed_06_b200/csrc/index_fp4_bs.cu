@@ -142,6 +142,27 @@ CSA_DEVINL void cp_async_row(uint32_t dst, const uint8_t *src, bool valid) {
         asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(dst), "l"(src), "n"(KB), "r"(n) : "memory");
 }
 
+// Query-head scales of group g of sequence b for head rows n = 32 gq + lane:
+// v[gq][j] = the j-th 32-bit word of row n's scale bytes (zero past the heads).
+template <int NKS>
+CSA_DEVINL void load_qscales(const Fp4BsParams &p, int b, int g, int lane, uint32_t (&v)[4][NKS]) {
+    constexpr int KB = 4 * NKS;
+#pragma unroll
+    for (int gq = 0; gq < 4; ++gq) {
+        const int n = 32 * gq + lane;
+#pragma unroll
+        for (int j = 0; j < NKS; ++j) v[gq][j] = 0u;
+        if (n < p.n_cols) {
+            const int qi = n / p.H_pad, h = n - qi * p.H_pad, q = g * p.NQ + qi;
+            if (q < p.nq && h < p.H_I) {
+                const uint8_t *src = p.q4s + (((size_t)b * p.nq + q) * p.H_I + h) * KB;
+#pragma unroll
+                for (int j = 0; j < NKS; ++j) v[gq][j] = __ldg(reinterpret_cast<const uint32_t *>(src) + j);
+            }
+        }
+    }
+}
+
 template <int KB>
 __global__ void __launch_bounds__(kThreads, 1)
     index_fp4_bs_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -196,6 +217,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc::tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
         tc::tmem_relinquish();
+    }
+    // Scale movers (warps 2..5): thread r owns row r of every sub-tile and query-head
+    // row r of every group.  The first kSfAhead tiles' key scales and the first
+    // group's query-head scales are requested before the setup barrier, i.e.
+    // before the producer fills its ring: issued after it, they waited behind the
+    // ring's key tiles in the memory queues and the first MMA came ~6.8 us after
+    // entry.  (The copies' barrier arrivals follow the barrier initialisation.)
+    const int mv_r = (warp & 3) * 32 + lane;
+    const uint32_t mv_row = smem_u32(sf_smem + mv_r * KB);
+    const auto prefetch_copies = [&](const Cursor &c, long long i) {
+        for (int h = 0; h < p.sub; ++h) {
+            const long long key = (long long)c.kt * p.tile_keys + h * kSubKeys + mv_r;
+            const bool valid = key < p.N;
+            cp_async_row<KB>(mv_row + (uint32_t)(((i % kSfAhead) * p.tile_keys + h * kSubKeys) * KB),
+                             p.k4s + ((size_t)c.b * p.N + (valid ? key : 0)) * KB, valid);
+        }
+    };
+    uint32_t q_first[4][NKS];
+    if (warp >= 2 && warp < 6 && w0 < w1) {
+        Cursor pf0 = cursor_at(p, w0);
+        load_qscales<NKS>(p, pf0.b, pf0.g, lane, q_first);
+        for (int i = 0; i < kSfAhead && pf0.w < w1; ++i, advance(p, pf0)) prefetch_copies(pf0, i);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -287,25 +330,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // memory queues and set the pace.  A thread reads and refills only its own
         // row of a slot, so a slot needs no barrier between the movers.
         const int sub = warp & 3;  // tensor-memory lanes this warp may access
-        const int r = sub * 32 + lane;
+        const int r = mv_r;
         const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
-        const uint32_t stage_row = smem_u32(sf_smem + r * KB);
         const auto prefetch = [&](const Cursor &c, long long i) {
             if (c.w < w1) {
-                for (int h = 0; h < p.sub; ++h) {
-                    const long long key = (long long)c.kt * p.tile_keys + h * kSubKeys + r;
-                    const bool valid = key < p.N;
-                    cp_async_row<KB>(stage_row + (uint32_t)(((i % kSfAhead) * p.tile_keys + h * kSubKeys) * KB),
-                                     p.k4s + ((size_t)c.b * p.N + (valid ? key : 0)) * KB, valid);
-                }
+                prefetch_copies(c, i);
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
                              ::"r"(smem_u32(sfld + (int)(i % kSfAhead))) : "memory");
             }
         };
+        // the arrivals of the copies issued before the setup barrier (each tracks
+        // all of this thread's copies so far)
         Cursor pf = cursor_at(p, w0);
         for (int i = 0; i < kSfAhead; ++i) {
-            prefetch(pf, i);
-            if (pf.w < w1) advance(p, pf);
+            if (pf.w < w1) {
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                             ::"r"(smem_u32(sfld + i)) : "memory");
+                advance(p, pf);
+            }
         }
         long long gi = 0, i = 0;
         Ring sr;
@@ -317,23 +359,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // factors from the lanes of s), so each warp writes its own copy
                 if (!wait_all(qsempty, (uint32_t)((gi & 1) ^ 1))) break;
                 tc::fence_after_sync();
-                for (int gq = 0; gq < 4; ++gq) {
-                    const int n = 32 * gq + lane;
-                    uint32_t v[NKS];
+                uint32_t v[4][NKS];
+                if (cu.w == w0) {
 #pragma unroll
-                    for (int j = 0; j < NKS; ++j) v[j] = 0u;
-                    if (n < p.n_cols) {
-                        const int qi = n / p.H_pad, h = n - qi * p.H_pad, q = cu.g * p.NQ + qi;
-                        if (q < p.nq && h < p.H_I) {
-                            const uint8_t *src = p.q4s + (((size_t)cu.b * p.nq + q) * p.H_I + h) * KB;
+                    for (int gq = 0; gq < 4; ++gq)
 #pragma unroll
-                            for (int j = 0; j < NKS; ++j) v[j] = __ldg(reinterpret_cast<const uint32_t *>(src) + j);
-                        }
-                    }
+                        for (int j = 0; j < NKS; ++j) v[gq][j] = q_first[gq][j];
+                } else {
+                    load_qscales<NKS>(p, cu.b, cu.g, lane, v);
+                }
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq)
 #pragma unroll
                     for (int j = 0; j < NKS; ++j)
-                        tmem_st1(tmem_base + lane_off + p.sfb_col + (uint32_t)(4 * j + gq), v[j]);
-                }
+                        tmem_st1(tmem_base + lane_off + p.sfb_col + (uint32_t)(4 * j + gq), v[gq][j]);
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
