@@ -31,8 +31,9 @@
 // ~100 cycles, two threads twice as fast); warps 2..5 -- scale
 // movers (each thread stages its key row's scale bytes with cp.async several
 // tiles ahead and writes them into the tile's tensor-memory slot; the
-// query-head scales once per group); warps 6..21 -- up to four epilogue
-// groups of four warps, one per accumulator, taking the tiles in turn
+// query-head scales once per group); warps 6..21 -- four epilogue groups of
+// four warps (a tile's two sub-tiles to a pair of groups, the pairs taking
+// the tiles in turn; one-sub-tile tiles: one group per accumulator)
 // (tcgen05.ld, ReLU, weighted head sum, causal mask, store).  Every wait is
 // bounded and every role warp stays converged.
 #include <algorithm>
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < p.n_acc; ++a) {
             mbar_init(tfull + a, p.sub);
-            mbar_init(tempty + a, 4);
+            mbar_init(tempty + a, p.sub == 2 ? 8 : 4);  // the warps of the groups that read it
         }
         for (int s = 0; s < kSfSlots; ++s) {
             mbar_init(sfull + s, 4);
@@ -407,11 +408,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kMma2Warp) {
         // ------------------------------------------------------------ epilogue (warps 6..21)
-        // Groups of four warps, one per accumulator (n_acc <= kEpiGroups; the rest
-        // idle): tile i -> accumulator and group i % n_acc.  Each accumulator's
-        // tiles then reach one group in order, so a group never waits on a
-        // tfull phase parity two phases ahead of the one it means.
+        // Groups of four warps.  Two-sub-tile tiles: tile i -> accumulator i % n_acc
+        // and the group pair i % 2, sub-tile h to group 2 (i % 2) + h, so that a
+        // tile's two sub-tiles are summed in parallel (one group per tile took
+        // ~2 us per tile, the accumulators' turnaround set the pace).  One
+        // sub-tile: tile i -> accumulator and group i % n_acc.  A group never
+        // waits on a tfull phase two phases ahead of the one it means: the next
+        // use of its accumulator needs this group's tempty arrival.
         const int eg = (warp - 6) >> 2;
+        const bool pairs = p.sub == 2;
+        const int pair = eg >> 1, hsel = eg & 1;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
         const int et = (threadIdx.x - 192) & 127;  // thread within its group
@@ -420,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int loaded_b = -1, loaded_g = -1;
         for (Cursor cu = cursor_at(p, w0); cu.w < w1; advance(p, cu)) {
             const int li = (int)(cu.w - w0);
-            if (li % p.n_acc != eg) continue;
+            if (pairs ? ((li & 1) != pair) : (li % p.n_acc != eg)) continue;
             const int b = cu.b, g = cu.g;
             if (b != loaded_b || g != loaded_g) {
                 group_bar(eg);
@@ -443,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc::fence_after_sync();
             for (int h = 0; h < p.sub; ++h) {
+                if (pairs && h != hsel) continue;
                 const long long s = (long long)cu.kt * p.tile_keys + h * kSubKeys + row;
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * p.sub + h) * p.n_cols);
                 for (int qi = 0; qi < p.NQ; ++qi) {
