@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256) compress_small_kernel(
 
 // ------------------------------------------------------------------ large m
 constexpr int kTableThreads = 256;
-constexpr int kStepRows = 8;  // rows whose loads are in flight together
+constexpr int kStepRows = 6;  // rows whose loads are in flight together (64 registers: four CTAs per SM)
 
 // Softmax weights of the 2m logits of every channel: w[j][c] (one warp per
 // channel; the lanes' partial maxima and sums are combined in a fixed order).
