@@ -48,6 +48,8 @@ struct IndexTcParams {
     int n_cols;           // N of the MMA = NQ * H_pad
     int n_acc;            // TMEM accumulators (2 or 4)
     uint32_t tmem_cols;   // allocated columns (n_acc accumulators)
+    int split;            // MMA-issuing warps (2: each issues half of the N columns)
+    uint32_t idesc_half;  // instruction descriptor of N = n_cols / 2
     DevCtx ctx;
 };
 
@@ -97,8 +99,12 @@ struct Ring {
     }
 };
 
+// Threads: producer and MMA warps, two epilogue groups of EW warps, and with
+// EW = 8 (several queries per tile) a second MMA-issuing warp.
+constexpr int index_threads(int EW) { return 64 + 64 * EW + (EW == 8 ? 32 : 0); }
+
 template <int EW, int OCC>  // warps per epilogue group (4: one per TMEM lane quarter, 8: two); CTAs per SM
-__global__ void __launch_bounds__(64 + 64 * EW, OCC)
+__global__ void __launch_bounds__(index_threads(EW), OCC)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const IndexTcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -126,14 +132,14 @@ __global__ void __launch_bounds__(64 + 64 * EW, OCC)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);
+            mbar_init(empty + s, p.split);  // one commit per MMA issuer
         }
         for (int a = 0; a < p.n_acc; ++a) {
-            mbar_init(tfull + a, 1);
+            mbar_init(tfull + a, p.split);
             mbar_init(tempty + a, EW);
         }
         mbar_init(qfull, 1);
-        mbar_init(qempty, 1);
+        mbar_init(qempty, p.split);
         *abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&kmap);
@@ -182,8 +188,15 @@ __global__ void __launch_bounds__(64 + 64 * EW, OCC)
             mbar_wait(smem_u32(full + (j % p.stages)), (uint32_t)((j / p.stages) & 1), p.ctx, nullptr);
         if (gi > 0) mbar_wait(smem_u32(qfull), (uint32_t)((gi - 1) & 1), p.ctx, nullptr);
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || (EW == 8 && p.split == 2 && warp == 2 + 2 * EW)) {
+        // ------------------------------------------------------------ MMA issuers
+        // With several queries per tile two warps issue, each the N / 2 columns
+        // of its half of the query heads (a thread issues a tcgen05.mma only
+        // every ~100-160 cycles, which held the tensor pipe to ~37 % at N = 256);
+        // both wait on the same barriers and commit to the ones the tile releases.
+        const int half = (p.split == 2 && warp != 1) ? 1 : 0;
+        const int ncol = p.n_cols / p.split;
+        const uint32_t idesc = p.split == 2 ? p.idesc_half : p.idesc;
         long long gi = 0;
         Ring kr, ar;
         const uint32_t sbo = 8u * p.row_bytes;
@@ -201,13 +214,14 @@ __global__ void __launch_bounds__(64 + 64 * EW, OCC)
             const int st = kr.idx;
             if (!wait_all(full + st, kr.phase)) break;
             tc::fence_after_sync();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols);
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.n_cols + half * ncol);
             const uint64_t kd = kdesc0 + ((uint64_t)(st * p.stage_bytes) >> 4);
             uint32_t accumulate = 0;
             for (int c = 0; c < p.nchunk; ++c) {
                 for (int kk = 0; kk < p.chunk_elems / 16; ++kk) {
                     tc::mma_f16(d_tmem, kd + ((uint32_t)(c * kTileKeys * p.row_bytes + kk * 32) >> 4),
-                                qdesc0 + ((uint32_t)(c * p.n_cols * p.row_bytes + kk * 32) >> 4), p.idesc, accumulate,
+                                qdesc0 + ((uint32_t)((c * p.n_cols + half * ncol) * p.row_bytes + kk * 32) >> 4), idesc,
+                                accumulate,
                                 issuer);
                     accumulate = 1;
                 }
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(64 + 64 * EW, OCC)
             kr.next(p.stages);
             ar.next(p.n_acc);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 2 + 2 * EW) {
         // ------------------------------------------------------------ epilogue
         // Two groups of EW warps take alternate tiles (tile i -> group i & 1,
         // accumulator i % n_acc), doubling the epilogue rate; with EW = 8 the two
@@ -367,12 +381,16 @@ int launch_index_tc(const uint16_t *q_idx, const float *w, const uint16_t *k_idx
                         8 + (2 * kMaxStages + 2 * kMaxAcc + 2) * 8 + 16;
     // several queries per tile: two warps per TMEM lane quarter split them
     const int EW = NQ >= 2 ? 8 : 4;
+    // two MMA issuers when each half of N is a valid MMA width starting on an
+    // 8-row swizzle atom of the query tile
+    p.split = (EW == 8 && (p.n_cols / 2) % 16 == 0) ? 2 : 1;
+    p.idesc_half = tc::idesc_f16(std::max(16, p.n_cols / 2), true);
     void (*kern)(const CUtensorMap, const CUtensorMap, const IndexTcParams) =
         EW == 8 ? index_tc_kernel<8, 1> : (two_per_sm ? index_tc_kernel<4, 2> : index_tc_kernel<4, 1>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CSA_ERR_CUDA;
     const int grid = (int)std::min<long long>(p.total_work, (two_per_sm ? 2 : 1) * num_sms());
-    kern<<<grid, 64 + 64 * EW, smem, st>>>(kmap, qmap, p);
+    kern<<<grid, index_threads(EW), smem, st>>>(kmap, qmap, p);
     return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
