@@ -524,6 +524,9 @@ def _dev(a, dtype=None):
     (1, 64, 128, 512, 1024, 4096, 64, 32, 4, [4095 - 5 * i for i in range(64)]),   # one split
     (2, 1, 40, 128, 97, 400, 33, 7, 4, [399, 13]),                     # ragged heads, D = 128
     (1, 3, 128, 256, 300, 1200, 64, 16, 4, [1199, 700, 5]),
+    # 400 work items on at most 148 CTAs: a CTA's last tile of one item is expanded
+    # while the next item's first tile is copied
+    (1, 200, 128, 512, 2048, 8192, 64, 32, 4, [8191 - 7 * i for i in range(200)]),
 ])
 def test_csa_attend_fp8kv_parity(cuda, batch, nq, H, D, N, T, k, Wn, m, ts):
     """The FP8 cache (quantised by the oracle) against the oracle's attention on
