@@ -6,9 +6,12 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  * Buffers are caller-owned DEVICE memory unless stated otherwise,
- *    row-major and contiguous, base pointers 16-byte aligned.  The library
- *    never allocates or frees device memory; calls that need scratch take a
- *    caller workspace sized by the matching *_workspace_bytes() query.
+ *    row-major and contiguous, base pointers 16-byte aligned.  Calls that
+ *    need scratch take a caller workspace sized by the matching
+ *    *_workspace_bytes() query.  The one allocation the library makes is the
+ *    weight table of csa_compress at large m (stream ordered, from a memory
+ *    pool of the library that keeps its memory: 2m*d*4 bytes, at most 2 MiB,
+ *    per call in flight).
  *  * bf16 tensors are passed as `const uint16_t *` holding bf16 bit patterns.
  *  * `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *    asynchronous on that stream and returns after enqueueing its kernels.
@@ -82,8 +85,8 @@ int csa_version(void);
  * (m > 16 or 24*m*d > 96 KiB additionally needs logits 16-byte aligned;
  * CSA_ERR_UNSUPPORTED otherwise).  Those shapes write the 2m x d softmax
  * weights into a table taken from a memory pool of the library (stream
- * ordered; the pool keeps its memory, 2m*d*4 bytes at most per device, between
- * calls) and pool every entry but the first with them; entry 0 runs the
+ * ordered, 2m*d*4 bytes per call in flight; the pool keeps its memory
+ * between calls) and pool every entry but the first with them; entry 0 runs the
  * csa_compress_dynamic kernel with no Z rows (its logits Z + bias are then
  * these logits); where the pool cannot be had, and for d / 8 not in {32, 64,
  * 128}, that kernel computes every entry.  Results agree with the small-m
