@@ -16,8 +16,10 @@
 // holds the k-th largest score -- then has few keys: every key above it is
 // selected, and the keys inside it (at most 256) are pushed, with the per-CTA
 // counts, into every CTA's shared memory, where each CTA ranks them directly
-// (score descending, index ascending) and writes its own selected indices in
-// index order.  After that barrier no CTA touches another's memory.
+// (score descending, index ascending; up to 32 of them by one warp with
+// shuffles and a ballot, more by the whole block) and writes its own selected
+// indices in index order.  After that barrier no CTA touches another's memory.
+// Every block scan takes one block barrier (each warp scans the warp totals).
 //
 // The value-linear pass runs at up to 8 keys per thread (the decode batches);
 // longer rows per thread, a non-finite score range, or a threshold bin above
