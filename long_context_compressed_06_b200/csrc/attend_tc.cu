@@ -28,7 +28,9 @@
 // and 9..10 gather the key rows with 16-byte cp.async into
 // the 128-byte swizzled layout (one 512-byte coalesced row segment per warp
 // instruction; HCA tiles of consecutive entries arrive as TMA tiles instead)
-// from kernel entry on, each tile's key-validity mask travelling with it;
+// from kernel entry on, each tile's key-validity mask travelling with it
+// (FP8 rows: the e4m3 codes are copied the same way and expanded to bf16 in
+// place once the next tile's copies are issued);
 // warps 4..7 take each head's 1/RMS from the diagonal of Q Q^T (rewriting the
 // query tile only for a gain or RoPE), then run the softmax, two threads per
 // head (keys 0-31 / 32-63, D/2 output columns each), and store the output
