@@ -88,8 +88,9 @@ int csa_version(void);
  * ordered, 2m*d*4 bytes per call in flight; the pool keeps its memory
  * between calls) and pool every entry but the first with them; entry 0 runs the
  * csa_compress_dynamic kernel with no Z rows (its logits Z + bias are then
- * these logits); where the pool cannot be had, and for d / 8 not in {32, 64,
- * 128}, that kernel computes every entry.  Results agree with the small-m
+ * these logits); where the pool cannot be had, on a stream being captured
+ * into a CUDA graph, and for d / 8 not in {32, 64, 128}, that kernel computes
+ * every entry.  Results agree with the small-m
  * kernel up to fp32 rounding order.
  */
 int csa_compress(const uint16_t *A, const uint16_t *B, const float *logits,

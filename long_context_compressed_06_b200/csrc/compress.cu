@@ -294,7 +294,16 @@ int launch_compress(const uint16_t *A, const uint16_t *B, const float *logits, i
     const int tpe = d / 8;
     const bool tabled = (tpe == 32 || tpe == 64 || tpe == 128 || tpe == 256) && N > 1;
     float *table = nullptr;
-    cudaMemPool_t pool = tabled ? table_pool() : nullptr;
+    // a stream being captured into a graph takes the allocation-free path
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    bool capturing = false;
+    if (cudaStreamIsCapturing(st, &capture) != cudaSuccess) {
+        cudaGetLastError();  // the query failed (e.g. the legacy stream during a capture): treat as capturing
+        capturing = true;
+    } else {
+        capturing = capture != cudaStreamCaptureStatusNone;
+    }
+    cudaMemPool_t pool = (tabled && !capturing) ? table_pool() : nullptr;
     if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&table), (size_t)2 * m * d * sizeof(float), pool,
                                          st) != cudaSuccess) {
         cudaGetLastError();  // no table: the online-softmax kernel does every entry
